@@ -1,0 +1,94 @@
+"""Seeded synthetic inputs for the attention workloads.
+
+This module only draws random numbers and casts them; it holds none of the
+attention arithmetic.  Both the CUDA path's tests and the CPU oracle's tests
+take their inputs from here.
+
+Recipe (one CPU generator per workload, ``torch.Generator().manual_seed(seed)``):
+
+1. ragged workload only: valid key lengths ``seqlens[b]`` drawn uniformly
+   from {1, ..., N} (``torch.randint``);
+2. Q, K, V, then dO, each an iid N(0, 1) float32 draw of shape [B, H, N, d];
+3. ragged workload only: K row j multiplied by (1 + 3 j / N) in float32, so
+   that the running row max keeps growing across K tiles;
+4. each tensor cast round-to-nearest-even to the workload's 16-bit dtype.
+
+The pages name no dataset or benchmark suite; these shapes stand in for the
+workloads they discuss (n = 8192 fp16 sizing, 32k context, short training
+shapes, padded batches).
+"""
+
+import math
+from dataclasses import dataclass, field
+
+import torch
+
+__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_inputs_shape"]
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    H: int
+    N: int
+    d: int
+    causal: bool
+    dtypes: tuple            # 16-bit dtypes the kernels run in
+    ragged: bool = False     # key-padding with drawn valid lengths
+    draw_dtype: str = "f32"  # inputs drawn in float32, then cast
+    description: str = field(default="", compare=False)
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+
+WORKLOADS = {
+    "tiny": Workload("tiny", 1, 1, 128, 64, False, (torch.bfloat16, torch.float16),
+                     description="B1 H1 N128 d64, fp32 draws cast to bf16 and fp16, non-causal"),
+    "small": Workload("small", 4, 16, 1024, 64, True, (torch.bfloat16,),
+                      description="B4 H16 N1024 d64 bf16 causal (short training shape)"),
+    "mid": Workload("mid", 2, 32, 8192, 128, True, (torch.bfloat16, torch.float16),
+                    description="B2 H32 N8192 d128 causal, bf16 and fp16"),
+    "long": Workload("long", 1, 32, 32768, 128, True, (torch.bfloat16,),
+                     description="B1 H32 N32768 d128 bf16 causal (no NxN buffer)"),
+    "ragged": Workload("ragged", 8, 16, 4099, 128, False, (torch.bfloat16,), ragged=True,
+                       description="B8 H16 N4099 d128 bf16, key padding with seqlens ~ U{1..N}, "
+                                   "K row j scaled by (1 + 3j/N)"),
+}
+
+
+def make_inputs_shape(B, H, N, d, dtype, seed=0, ragged=False, with_do=True,
+                      seqlens=None):
+    """Draw q, k, v (and dO) of shape [B, H, N, d] on the CPU.
+
+    Returns a dict with 16-bit tensors ``q, k, v, do`` and ``seqlens``
+    (int32 [B] or None).  ``ragged`` draws seqlens and grows K along the
+    sequence as in the module docstring; an explicit ``seqlens`` sequence
+    overrides the drawn one.
+    """
+    g = torch.Generator().manual_seed(seed)
+    sl = None
+    if ragged:
+        sl = torch.randint(1, N + 1, (B,), generator=g, dtype=torch.int64).to(torch.int32)
+    if seqlens is not None:
+        sl = torch.as_tensor(seqlens, dtype=torch.int32)
+    q = torch.randn(B, H, N, d, generator=g, dtype=torch.float32)
+    k = torch.randn(B, H, N, d, generator=g, dtype=torch.float32)
+    v = torch.randn(B, H, N, d, generator=g, dtype=torch.float32)
+    do = torch.randn(B, H, N, d, generator=g, dtype=torch.float32) if with_do else None
+    if ragged:
+        grow = 1.0 + 3.0 * torch.arange(N, dtype=torch.float32) / N
+        k = k * grow[None, None, :, None]
+    out = {"q": q.to(dtype), "k": k.to(dtype), "v": v.to(dtype),
+           "do": do.to(dtype) if do is not None else None, "seqlens": sl}
+    return out
+
+
+def make_inputs(name, dtype=None, seed=0, with_do=True):
+    """Inputs of a named workload (``WORKLOADS``) in ``dtype`` (default: its first)."""
+    w = WORKLOADS[name]
+    dt = dtype if dtype is not None else w.dtypes[0]
+    return make_inputs_shape(w.B, w.H, w.N, w.d, dt, seed=seed, ragged=w.ragged,
+                             with_do=with_do)

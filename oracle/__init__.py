@@ -1,0 +1,13 @@
+"""CPU float64 oracle for exact tiled attention.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+the CPU-baseline leg of ``bench.py`` may import it.  The CUDA library and its
+Python binding never import it, and it imports nothing from them.
+"""
+
+from .attention import (allowed_mask, ref_bwd, ref_bwd_slice, ref_fwd,
+                        ref_fwd_slice)
+from .online_model import tiled_fwd_slice
+
+__all__ = ["allowed_mask", "ref_fwd_slice", "ref_fwd", "ref_bwd_slice",
+           "ref_bwd", "tiled_fwd_slice"]
