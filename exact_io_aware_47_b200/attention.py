@@ -1,0 +1,110 @@
+"""torch-facing calls of the CUDA library: allocate outputs, pass pointers.
+
+``forward`` and ``backward`` validate tensor properties that ctypes cannot
+see (device, dtype, contiguity, shapes), allocate the outputs and the
+backward workspace with torch, and call ``fa_fwd`` / ``fa_bwd`` on the
+current CUDA stream.  No arithmetic of the method happens here.
+"""
+
+import math
+
+import torch
+
+from . import _lib
+
+_DTYPES = {torch.bfloat16: _lib.FA_BF16, torch.float16: _lib.FA_FP16}
+
+
+def _stream_handle(device):
+    return ctypes_void(torch.cuda.current_stream(device).cuda_stream)
+
+
+def ctypes_void(x):
+    return x if x else None
+
+
+def _check_inputs(tensors, shape, dtype, device):
+    for name, t in tensors.items():
+        if t is None:
+            raise ValueError(f"{name} is None")
+        if not t.is_cuda or t.device != device:
+            raise ValueError(f"{name} must be a CUDA tensor on {device}")
+        if t.dtype != dtype:
+            raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous [B, H, N, d]")
+
+
+def _seqlens_arg(seqlens, B, device):
+    if seqlens is None:
+        return None, None
+    sl = seqlens
+    if not (torch.is_tensor(sl) and sl.is_cuda and sl.dtype == torch.int32 and sl.is_contiguous()):
+        sl = torch.as_tensor(seqlens, dtype=torch.int32).to(device).contiguous()
+    if sl.shape != (B,):
+        raise ValueError(f"seqlens must have shape ({B},)")
+    return sl, sl.data_ptr()
+
+
+def forward(q, k, v, scale=None, causal=False, seqlens=None, out=None, lse=None):
+    """O, LSE = attention(q, k, v) on the GPU ([B, H, N, d] bf16/fp16)."""
+    if q.dim() != 4:
+        raise ValueError("q must be [B, H, N, d]")
+    B, H, N, d = q.shape
+    dev = q.device
+    if q.dtype not in _DTYPES:
+        raise ValueError("dtype must be bfloat16 or float16")
+    _check_inputs({"q": q, "k": k, "v": v}, (B, H, N, d), q.dtype, dev)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    _check_inputs({"out": out}, (B, H, N, d), q.dtype, dev)
+    _check_inputs({"lse": lse}, (B, H, N), torch.float32, dev)
+    sl, sl_ptr = _seqlens_arg(seqlens, B, dev)
+    with torch.cuda.device(dev):
+        st = _lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                         B, H, N, d, scale, int(bool(causal)), sl_ptr, _DTYPES[q.dtype],
+                         _stream_handle(dev))
+    _lib.check("fa_fwd", st)
+    return out, lse
+
+
+def workspace_bytes(B, H, N, d):
+    return _lib.fa_bwd_workspace_size(B, H, N, d)
+
+
+def backward(q, k, v, o, lse, do, scale=None, causal=False, seqlens=None, workspace=None,
+             dq=None, dk=None, dv=None):
+    """dQ, dK, dV of the loss <dO, O> on the GPU."""
+    B, H, N, d = q.shape
+    dev = q.device
+    _check_inputs({"q": q, "k": k, "v": v, "o": o, "do": do}, (B, H, N, d), q.dtype, dev)
+    _check_inputs({"lse": lse}, (B, H, N), torch.float32, dev)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check_inputs({"dq": dq, "dk": dk, "dv": dv}, (B, H, N, d), q.dtype, dev)
+    need = workspace_bytes(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    sl, sl_ptr = _seqlens_arg(seqlens, B, dev)
+    with torch.cuda.device(dev):
+        st = _lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                         lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                         workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                         B, H, N, d, scale, int(bool(causal)), sl_ptr, _DTYPES[q.dtype],
+                         _stream_handle(dev))
+    _lib.check("fa_bwd", st)
+    return dq, dk, dv
+
+
+def device_status(device=None):
+    """Synchronise and return (status, raw word) of the device status word."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        return _lib.fa_device_status(_stream_handle(dev))

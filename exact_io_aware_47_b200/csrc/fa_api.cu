@@ -1,0 +1,223 @@
+// C ABI of the library: argument checks, TMA descriptors, launches.
+//
+// Every check here runs on the host before anything is enqueued, so a bad
+// call returns a status and leaves the device untouched.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/fa.h"
+#include "fa_internal.h"
+#include "sm100.cuh"
+
+namespace fa {
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  bool probed = false;
+  bool is_sm100 = false;
+  int num_sms = 0;
+};
+
+DeviceInfo g_devices[kMaxDevices];
+std::mutex g_mutex;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn g_encode = nullptr;
+
+int current_device_info(DeviceInfo* out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceInfo& di = g_devices[dev];
+  if (!di.probed) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return FA_ERR_CUDA;
+    di.is_sm100 = (major == 10 && minor == 0);
+    di.num_sms = sms;
+    di.probed = true;
+  }
+  if (g_encode == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return FA_ERR_CUDA;
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  *out = di;
+  return di.is_sm100 ? FA_OK : FA_ERR_ARCH;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_common(int B, int H, int N, int d, float scale, int dtype) {
+  if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const long long elems = static_cast<long long>(B) * H * N * d;
+  if (elems >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+// [B*H, N, d] view of a [B, H, N, d] 16-bit tensor; box = 64 columns x 128 rows,
+// 128-byte swizzle (the layout the tcgen05 descriptors expect).  Rows past N
+// inside a head read as zero.
+int make_map(CUtensorMap* map, const void* ptr, int BH, int N, int d, int dtype) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                                 static_cast<cuuint64_t>(N) * d * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r =
+      g_encode(map, dtype == FA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+               3, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+}  // namespace
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                      int H, int N, int d, float scale, int causal, const int32_t* seqlens,
+                      int dtype, void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  int st = check_common(B, H, N, d, scale, dtype);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      (seqlens && (reinterpret_cast<uintptr_t>(seqlens) & 3u)))
+    return FA_ERR_ALIGNMENT;
+  DeviceInfo di;
+  st = current_device_info(&di);
+  if (st != FA_OK) return st;
+
+  CUtensorMap tq, tk, tv;
+  const int BH = B * H;
+  if (make_map(&tq, q, BH, N, d, dtype) != FA_OK || make_map(&tk, k, BH, N, d, dtype) != FA_OK ||
+      make_map(&tv, v, BH, N, d, dtype) != FA_OK)
+    return FA_ERR_CUDA;
+
+  FwdParams p;
+  p.o = o;
+  p.lse = lse;
+  p.seqlens = seqlens;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = causal ? 1 : 0;
+  p.n_qtiles = (N + kBlockM - 1) / kBlockM;
+  p.n_pairs = (p.n_qtiles + 1) / 2;
+  p.n_units = BH * p.n_pairs;
+  const cudaError_t e =
+      launch_fwd(d, dtype == FA_BF16, tq, tk, tv, p, di.num_sms, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+extern "C" size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  if (check_common(B, H, N, d, 1.f, FA_BF16) != FA_OK) return 0;
+  const size_t rows = static_cast<size_t>(B) * H * N;
+  return round256(rows * sizeof(float)) + round256(rows * d * sizeof(float));
+}
+
+extern "C" int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                      const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                      size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
+                      const int32_t* seqlens, int dtype, void* stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  int st = check_common(B, H, N, d, scale, dtype);
+  if (st != FA_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (seqlens && (reinterpret_cast<uintptr_t>(seqlens) & 3u)))
+    return FA_ERR_ALIGNMENT;
+  const size_t need = fa_bwd_workspace_size(B, H, N, d);
+  if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FA_ERR_ALIGNMENT;
+  DeviceInfo di;
+  st = current_device_info(&di);
+  if (st != FA_OK) return st;
+
+  CUtensorMap tq, tk, tv, tdo;
+  const int BH = B * H;
+  if (make_map(&tq, q, BH, N, d, dtype) != FA_OK || make_map(&tk, k, BH, N, d, dtype) != FA_OK ||
+      make_map(&tv, v, BH, N, d, dtype) != FA_OK || make_map(&tdo, dout, BH, N, d, dtype) != FA_OK)
+    return FA_ERR_CUDA;
+
+  const size_t rows = static_cast<size_t>(BH) * N;
+  BwdParams p;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.o = o;
+  p.dout = dout;
+  p.lse = lse;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.dsum = static_cast<float*>(workspace);
+  p.dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round256(rows * sizeof(float)));
+  p.seqlens = seqlens;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = causal ? 1 : 0;
+  p.n_ktiles = (N + kBlockN - 1) / kBlockN;
+  p.n_units = BH * p.n_ktiles;
+  const cudaError_t e = launch_bwd(d, dtype == FA_BF16, tq, tk, tv, tdo, p, di.num_sms,
+                                   static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+extern "C" int fa_device_status(void* stream, uint32_t* detail) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+  unsigned int word = 0;
+  const unsigned int zero = 0;
+  if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return FA_ERR_CUDA;
+  if (word != 0 && cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess)
+    return FA_ERR_CUDA;
+  if (detail) *detail = word;
+  const unsigned code = word & 0xffu;
+  if (code == kErrDeviceTimeout) return FA_ERR_DEVICE_TIMEOUT;
+  if (code == kErrDeviceSeqlen) return FA_ERR_DEVICE_SEQLEN;
+  return word == 0 ? FA_OK : FA_ERR_CUDA;
+}
+
+extern "C" const char* fa_status_string(int status) {
+  switch (status) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID_ARG: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported shape (d must be 64 or 128; B*H*N*d < 2^31)";
+    case FA_ERR_ALIGNMENT: return "pointer not aligned (16 bytes; workspace 256 bytes)";
+    case FA_ERR_ARCH: return "current device is not sm_100 (B200)";
+    case FA_ERR_CUDA: return "CUDA call or launch failed";
+    case FA_ERR_DEVICE_TIMEOUT: return "device pipeline wait timed out";
+    case FA_ERR_DEVICE_SEQLEN: return "seqlens value outside [1, N] (clamped on device)";
+    case FA_ERR_WORKSPACE: return "backward workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+extern "C" int fa_version(void) { return 100; }

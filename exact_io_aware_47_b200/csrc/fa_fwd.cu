@@ -1,0 +1,441 @@
+// Forward exact attention on sm_100a: tiled, online softmax, nothing N x N
+// ever leaves the SM.
+//
+// What is computed follows "How Flash Attention Works" (swarnava.dev):
+//  * section "Tiling Q, K, and V for Fast On-Chip Memory": a block of query
+//    rows stays on chip while K and V blocks stream past it; causal and
+//    padding masks are applied per tile, boundary tiles take the ragged edge;
+//  * section "Online Softmax Without the Full Score Matrix": each K/V tile
+//    updates a running row max and row sum, and the partial output is
+//    rescaled when the max grows;
+//  * section "Kernel Fusion and Incremental Output Accumulation": scores,
+//    masking, softmax statistics and the V-weighted accumulation all happen
+//    in one kernel, and only O and per-row statistics (here the log-sum-exp)
+//    reach HBM.
+//
+// B200 mapping (one persistent CTA per SM, 384 threads):
+//  * a work unit is (batch*head, pair of 128-row query tiles); the two tiles
+//    share every K/V tile that is loaded, and their softmax work ping-pongs
+//    so the tensor core always has the other tile's MMA to run;
+//  * warp 9 (one thread) issues TMA loads: Q tiles once per unit, K and V
+//    tiles through a ring of shared-memory slots guarded by mbarriers;
+//  * warp 8 (one thread) issues tcgen05 MMAs: S = Q K^T into TMEM, then
+//    O += P V with P read straight from TMEM;
+//  * warps 0-3 and 4-7 are the softmax warpgroups of query tile 0 and 1: a
+//    thread owns one query row (TMEM lane), so row max and row sum need no
+//    shuffles; they write P (16-bit) over S in TMEM, rescale O in TMEM when
+//    the running max moves by more than the lazy threshold, and finally
+//    normalise O and store O and LSE with 16-byte vector stores.
+//
+// TMEM columns: S0 [0,128), S1 [128,256), O0 and O1 at 256 + t*d.
+#include "fa_internal.h"
+#include "sm100.cuh"
+
+namespace fa {
+
+template <int D>
+struct FwdLayout {
+  static constexpr int kTileBytes = kBlockM * D * 2;  // one 128-row, d-wide 16-bit tile
+  static constexpr int kPanelBytes = 128 * 64 * 2;    // one 64-column swizzle panel (16 KB)
+  static constexpr int kPanels = D / 64;
+  static constexpr int kSlots = (D == 128) ? 4 : 8;   // K/V ring depth
+  static constexpr int kQ0 = 0;
+  static constexpr int kSlot0 = 2 * kTileBytes;
+  static constexpr int kBar = kSlot0 + kSlots * kTileBytes;
+  static constexpr int kBarBytes = 512;
+  static constexpr int kSmemBytes = kBar + kBarBytes + 1024;  // + slack to align to 1024
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColO = 256;
+};
+
+struct FwdUnit {
+  int bh, qt0, L, jend0, jend1;
+};
+
+__device__ __forceinline__ FwdUnit fwd_decode(int u, const FwdParams& p) {
+  FwdUnit w;
+  const int r = u % p.n_pairs;
+  w.bh = u / p.n_pairs;
+  // causal units of one head run longest-first; heads stay contiguous so the
+  // CTAs running at the same time share K/V in L2
+  const int pair = p.causal ? (p.n_pairs - 1 - r) : r;
+  const int b = w.bh / p.H;
+  int L = p.N;
+  if (p.seqlens != nullptr) {
+    L = p.seqlens[b];
+    L = L < 1 ? 1 : (L > p.N ? p.N : L);
+  }
+  w.L = L;
+  const int nkb = (L + kBlockN - 1) / kBlockN;
+  w.qt0 = 2 * pair;
+  int je[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int qt = w.qt0 + t;
+    if (qt < p.n_qtiles) je[t] = p.causal ? min(nkb, qt + 1) : nkb;
+    else je[t] = 0;
+  }
+  w.jend0 = je[0];
+  w.jend1 = je[1];
+  return w;
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(384, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                  const __grid_constant__ CUtensorMap tmv, const FwdParams p) {
+  using Lay = FwdLayout<D>;
+  constexpr int kSlots = Lay::kSlots;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sq = smem + Lay::kQ0;        // Q0, Q1 tiles
+  uint8_t* skv = smem + Lay::kSlot0;    // K/V ring
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
+  uint64_t* q_full = bars;              // [2]
+  uint64_t* q_empty = bars + 2;         // [2]
+  uint64_t* kv_full = bars + 4;         // [kSlots]
+  uint64_t* kv_empty = kv_full + kSlots;
+  uint64_t* s_full = kv_empty + kSlots; // [2]
+  uint64_t* p_full = s_full + 2;        // [2]
+  uint64_t* o_full = p_full + 2;        // [2]
+  uint64_t* drain = o_full + 2;         // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&q_full[t], 1);
+      mbar_init(&q_empty[t], 1);
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 128);
+      mbar_init(&o_full[t], 1);
+    }
+    for (int s = 0; s < kSlots; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(tmem_slot, Lay::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 9) {
+    // ------------------------------------------------------------- TMA loads
+    if (lane == 0) {
+      tma_prefetch_desc(&tmq);
+      tma_prefetch_desc(&tmk);
+      tma_prefetch_desc(&tmv);
+      int qload[2] = {0, 0};
+      int kv_seq = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        const FwdUnit w = fwd_decode(u, p);
+        const int je[2] = {w.jend0, w.jend1};
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (je[t] == 0) continue;
+          ok = mbar_wait(&q_empty[t], (qload[t] & 1) ^ 1, abort_flag, 1);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&q_full[t], Lay::kTileBytes);
+#pragma unroll
+          for (int pn = 0; pn < Lay::kPanels; ++pn)
+            tma_load_3d(sq + t * Lay::kTileBytes + pn * Lay::kPanelBytes, &tmq, &q_full[t],
+                        pn * 64, (w.qt0 + t) * kBlockM, w.bh);
+          ++qload[t];
+        }
+        const int jmax = max(je[0], je[1]);
+        for (int j = 0; j < jmax && ok; ++j) {
+          for (int kv = 0; kv < 2; ++kv) {
+            const int slot = kv_seq % kSlots;
+            const int round = kv_seq / kSlots;
+            ok = mbar_wait(&kv_empty[slot], (round & 1) ^ 1, abort_flag, 2);
+            if (!ok) break;
+            mbar_arrive_expect_tx(&kv_full[slot], Lay::kTileBytes);
+            uint8_t* dst = skv + slot * Lay::kTileBytes;
+#pragma unroll
+            for (int pn = 0; pn < Lay::kPanels; ++pn)
+              tma_load_3d(dst + pn * Lay::kPanelBytes, kv ? &tmv : &tmk, &kv_full[slot], pn * 64,
+                          j * kBlockN, w.bh);
+            ++kv_seq;
+          }
+        }
+      }
+      // Never leave with copies in flight: wait for the last load issued into
+      // every barrier (already complete on the normal path).
+      for (int t = 0; t < 2; ++t)
+        if (qload[t] > 0) mbar_wait_drain(&q_full[t], (qload[t] - 1) & 1, 200000000ull);
+      for (int s = 0; s < kSlots; ++s) {
+        if (kv_seq > s) {
+          const int last = kv_seq - 1 - ((kv_seq - 1 - s) % kSlots);
+          mbar_wait_drain(&kv_full[s], (last / kSlots) & 1, 200000000ull);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 8) {
+    // ------------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      constexpr uint32_t kIdescQK = idesc_f16(BF16, 128, 128, false, false);
+      constexpr uint32_t kIdescPV = idesc_f16(BF16, 128, D, false, true);
+      const uint32_t sq_addr = smem_addr(sq);
+      const uint32_t skv_addr = smem_addr(skv);
+      int qload[2] = {0, 0};
+      int pcnt[2] = {0, 0};
+      int kv_seq = 0;
+      bool ok = true;
+
+      // S_t = Q_t K^T: A = Q tile (K-major), B = K tile (K-major); the
+      // 16-element K steps walk 32 bytes inside a 128-byte swizzle panel.
+      auto issue_s = [&](int t, int kslot) {
+        const uint32_t d_tmem = tmem + t * 128;
+        const uint32_t qa = sq_addr + t * Lay::kTileBytes;
+        const uint32_t kb = skv_addr + kslot * Lay::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * Lay::kPanelBytes + (kk & 3) * 32;
+          umma_ss(d_tmem, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024),
+                  kIdescQK, kk > 0 ? 1u : 0u);
+        }
+      };
+      // O_t += P_t V: A = P (16-bit, TMEM, over S_t), B = V tile read
+      // MN-major (d contiguous): 16 keys = 2048 bytes, 64-column panels
+      // 16 KB apart.
+      auto issue_pv = [&](int t, int vslot, bool acc) {
+        const uint32_t d_tmem = tmem + Lay::kColO + t * D;
+        const uint32_t vb = skv_addr + vslot * Lay::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kBlockN / 16; ++kk) {
+          umma_ts(d_tmem, tmem + t * 128 + kk * 8, sdesc_sw128(vb + kk * 2048, Lay::kPanelBytes, 1024),
+                  kIdescPV, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        const FwdUnit w = fwd_decode(u, p);
+        const int je[2] = {w.jend0, w.jend1};
+        const int jmax = max(je[0], je[1]);
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (je[t] == 0) continue;
+          ok = mbar_wait(&q_full[t], qload[t] & 1, abort_flag, 3);
+          ++qload[t];
+        }
+        if (!ok) break;
+        tc_fence_after();
+        // first K tile
+        {
+          const int slot = kv_seq % kSlots;
+          ok = mbar_wait(&kv_full[slot], (kv_seq / kSlots) & 1, abort_flag, 4);
+          if (!ok) break;
+          tc_fence_after();
+          for (int t = 0; t < 2; ++t) {
+            if (je[t] == 0) continue;
+            issue_s(t, slot);
+            umma_commit(&s_full[t]);
+            if (je[t] == 1) umma_commit(&q_empty[t]);
+          }
+          umma_commit(&kv_empty[slot]);
+          ++kv_seq;
+        }
+        for (int j = 0; j < jmax && ok; ++j) {
+          const int vslot = kv_seq % kSlots;
+          ok = mbar_wait(&kv_full[vslot], (kv_seq / kSlots) & 1, abort_flag, 5);
+          if (!ok) break;
+          tc_fence_after();
+          ++kv_seq;
+          const int kslot = kv_seq % kSlots;
+          bool k_ready = false;
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (j < je[t]) {
+              ok = mbar_wait(&p_full[t], pcnt[t] & 1, abort_flag, 6);
+              if (!ok) break;
+              ++pcnt[t];
+              tc_fence_after();
+              issue_pv(t, vslot, j > 0);
+              if (j == je[t] - 1) umma_commit(&o_full[t]);
+            }
+            if (j + 1 < je[t]) {
+              if (!k_ready) {
+                ok = mbar_wait(&kv_full[kslot], (kv_seq / kSlots) & 1, abort_flag, 7);
+                if (!ok) break;
+                tc_fence_after();
+                k_ready = true;
+              }
+              issue_s(t, kslot);
+              umma_commit(&s_full[t]);
+              if (j + 1 == je[t] - 1) umma_commit(&q_empty[t]);
+            }
+          }
+          if (!ok) break;
+          umma_commit(&kv_empty[vslot]);
+          if (j + 1 < jmax) {
+            umma_commit(&kv_empty[kslot]);
+            ++kv_seq;
+          }
+        }
+      }
+      // every MMA issued must be complete before TMEM is released
+      umma_commit(drain);
+      mbar_wait_drain(drain, 0, 200000000ull);
+    }
+    __syncwarp();
+  } else if (warp < 8) {
+    // ------------------------------------------------------------- softmax
+    const int t = warp >> 2;                 // query tile of the pair
+    const int r = ((warp & 3) << 5) | lane;  // row inside the tile = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + t * 128;
+    const uint32_t tO = tmem + lane_off + Lay::kColO + t * D;
+    const float c = p.scale_log2;
+    int scnt = 0, ocnt = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      const FwdUnit w = fwd_decode(u, p);
+      const int jend = t == 0 ? w.jend0 : w.jend1;
+      if (jend == 0) continue;
+      const int qt = w.qt0 + t;
+      const int row = qt * kBlockM + r;
+      if (t == 0 && r == 0 && p.seqlens != nullptr) {
+        const int raw = p.seqlens[w.bh / p.H];
+        if (raw < 1 || raw > p.N) record_error(kErrDeviceSeqlen, 0);
+      }
+      float m = -INFINITY;  // running max, log2 units
+      float l = 0.f;        // running sum of unnormalised probabilities
+      for (int j = 0; j < jend; ++j) {
+        ok = mbar_wait_warp(&s_full[t], scnt & 1, abort_flag, 8);
+        if (!ok) break;
+        ++scnt;
+        tc_fence_after();
+        float x[128];
+        {
+          uint32_t rr[32];
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            tmem_ld32(tS + cc * 32, rr);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[cc * 32 + i] = __uint_as_float(rr[i]) * c;
+          }
+        }
+        const int kbase = j * kBlockN;
+        const bool need_mask = (p.causal && j == qt) || (kbase + kBlockN > w.L);
+        if (need_mask) {
+          const int lim = p.causal ? min(w.L, row + 1) : w.L;  // keys < lim are visible
+#pragma unroll
+          for (int i = 0; i < 128; ++i)
+            if (kbase + i >= lim) x[i] = -INFINITY;
+        }
+        float mx = x[0];
+#pragma unroll
+        for (int i = 1; i < 128; ++i) mx = fmaxf(mx, x[i]);
+        const float m_new = (mx > m + kRescaleThreshold) ? mx : m;
+        const bool moved = m_new != m;
+        const float alpha = moved ? ex2_approx(m - m_new) : 1.f;  // 0 when m was -inf
+        l *= alpha;
+        if (j > 0 && __any_sync(0xffffffffu, moved)) {
+          // O_t holds the sum up to tile j-1 (its MMA completed before S_t(j)
+          // was committed); rows that did not move multiply by 1.
+          uint32_t ro[32];
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            tmem_ld32(tO + cc * 32, ro);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ro[i] = __float_as_uint(__uint_as_float(ro[i]) * alpha);
+            tmem_st32(tO + cc * 32, ro);
+          }
+        }
+        m = m_new;
+        const float mu = (m == -INFINITY) ? 0.f : m;
+        float sum = 0.f;
+        uint32_t pk[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const float p0 = ex2_approx(x[2 * i] - mu);
+          const float p1 = ex2_approx(x[2 * i + 1] - mu);
+          sum += p0 + p1;
+          pk[i] = pack2<BF16>(p0, p1);
+        }
+        l += sum;
+        {
+          uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
+          uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
+          tmem_st32(tS, lo);
+          tmem_st32(tS + 32, hi);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_full[t]);
+      }
+      if (!ok) break;
+      // epilogue: O / l -> 16-bit, LSE
+      ok = mbar_wait_warp(&o_full[t], ocnt & 1, abort_flag, 9);
+      if (!ok) break;
+      ++ocnt;
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      const bool store = row < p.N;
+      uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) +
+                      (static_cast<size_t>(w.bh) * p.N + (store ? row : 0)) * (D * 2);
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t ro[32];
+        tmem_ld32(tO + cc * 32, ro);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pk[i] = pack2<BF16>(__uint_as_float(ro[2 * i]) * inv_l, __uint_as_float(ro[2 * i + 1]) * inv_l);
+        if (store) {
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            st_global_v4(orow + cc * 64 + v4 * 16, pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2],
+                         pk[4 * v4 + 3]);
+        }
+      }
+      if (store) p.lse[static_cast<size_t>(w.bh) * p.N + row] = (m + log2f(l)) * 0.69314718055994531f;
+    }
+  }
+  // warps 10 and 11 have no role
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Lay::kTmemCols);
+  }
+}
+
+template <int D, bool BF16>
+static cudaError_t launch_fwd_t(const CUtensorMap& tmq, const CUtensorMap& tmk,
+                                const CUtensorMap& tmv, const FwdParams& p, int num_sms,
+                                cudaStream_t stream) {
+  using Lay = FwdLayout<D>;
+  auto kern = fa_fwd_kernel<D, BF16>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Lay::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int grid = p.n_units < num_sms ? p.n_units : num_sms;
+  kern<<<grid, 384, Lay::kSmemBytes, stream>>>(tmq, tmk, tmv, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fwd(int d, bool bf16, const CUtensorMap& tmq, const CUtensorMap& tmk,
+                       const CUtensorMap& tmv, const FwdParams& p, int num_sms,
+                       cudaStream_t stream) {
+  if (d == 128) {
+    return bf16 ? launch_fwd_t<128, true>(tmq, tmk, tmv, p, num_sms, stream)
+                : launch_fwd_t<128, false>(tmq, tmk, tmv, p, num_sms, stream);
+  }
+  return bf16 ? launch_fwd_t<64, true>(tmq, tmk, tmv, p, num_sms, stream)
+              : launch_fwd_t<64, false>(tmq, tmk, tmv, p, num_sms, stream);
+}
+
+}  // namespace fa

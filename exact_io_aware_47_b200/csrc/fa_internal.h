@@ -1,0 +1,63 @@
+// Parameters shared between the host launchers and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace fa {
+
+constexpr int kBlockM = 128;  // query rows per tile (TMEM lanes)
+constexpr int kBlockN = 128;  // keys per tile
+
+// Lazy-rescale threshold in log2 units: the running row max is only moved
+// when a tile's max exceeds it by more than this, so unnormalised
+// probabilities stay below 2^8 and the final division by the row sum (taken
+// with the same max) still yields the exact softmax.
+constexpr float kRescaleThreshold = 8.0f;
+
+struct FwdParams {
+  void* o;                  // [B, H, N, d] 16-bit
+  float* lse;               // [B, H, N] natural-log log-sum-exp
+  const int32_t* seqlens;   // [B] valid key lengths, or nullptr
+  int B, H, N;
+  float scale_log2;         // scale * log2(e)
+  int causal;
+  int n_qtiles;             // ceil(N / 128)
+  int n_pairs;              // ceil(n_qtiles / 2): a CTA work unit is two query tiles
+  int n_units;              // B * H * n_pairs
+};
+
+struct BwdParams {
+  const void* q;            // [B, H, N, d] 16-bit
+  const void* k;
+  const void* v;
+  const void* o;
+  const void* dout;
+  const float* lse;         // [B, H, N]
+  void* dq;                 // [B, H, N, d] 16-bit outputs
+  void* dk;
+  void* dv;
+  float* dsum;              // workspace [B, H, N]: D_i = <dO_i, O_i>
+  float* dq_acc;            // workspace [B, H, N, d] fp32 accumulator
+  const int32_t* seqlens;
+  int B, H, N;
+  float scale;
+  float scale_log2;
+  int causal;
+  int n_ktiles;             // ceil(N / 128)
+  int n_units;              // B * H * n_ktiles
+};
+
+// Host launchers (defined in the .cu files).  They assume validated
+// arguments and return a cudaError_t from the launch.
+cudaError_t launch_fwd(int d, bool bf16, const CUtensorMap& tmq, const CUtensorMap& tmk,
+                       const CUtensorMap& tmv, const FwdParams& p, int num_sms,
+                       cudaStream_t stream);
+
+cudaError_t launch_bwd(int d, bool bf16, const CUtensorMap& tmq, const CUtensorMap& tmk,
+                       const CUtensorMap& tmv, const CUtensorMap& tmdo, const BwdParams& p,
+                       int num_sms, cudaStream_t stream);
+
+}  // namespace fa

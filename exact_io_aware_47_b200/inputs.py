@@ -4,7 +4,10 @@ This module only draws random numbers and casts them; it holds none of the
 attention arithmetic.  Both the CUDA path's tests and the CPU oracle's tests
 take their inputs from here.
 
-Recipe (one CPU generator per workload, ``torch.Generator().manual_seed(seed)``):
+Recipe (one generator per workload, ``torch.Generator(device).manual_seed(seed)``;
+large workloads are drawn on the GPU, where torch's counter-based generator is
+fast, small ones on the CPU; the two devices give different draws, and a test
+always hands both the kernel and the oracle the same tensors):
 
 1. ragged workload only: valid key lengths ``seqlens[b]`` drawn uniformly
    from {1, ..., N} (``torch.randint``);
@@ -60,35 +63,38 @@ WORKLOADS = {
 
 
 def make_inputs_shape(B, H, N, d, dtype, seed=0, ragged=False, with_do=True,
-                      seqlens=None):
-    """Draw q, k, v (and dO) of shape [B, H, N, d] on the CPU.
+                      seqlens=None, device="cpu"):
+    """Draw q, k, v (and dO) of shape [B, H, N, d] on ``device``.
 
     Returns a dict with 16-bit tensors ``q, k, v, do`` and ``seqlens``
     (int32 [B] or None).  ``ragged`` draws seqlens and grows K along the
     sequence as in the module docstring; an explicit ``seqlens`` sequence
     overrides the drawn one.
     """
-    g = torch.Generator().manual_seed(seed)
+    device = torch.device(device)
+    g = torch.Generator(device=device).manual_seed(seed)
     sl = None
     if ragged:
-        sl = torch.randint(1, N + 1, (B,), generator=g, dtype=torch.int64).to(torch.int32)
+        sl = torch.randint(1, N + 1, (B,), generator=g, dtype=torch.int64,
+                           device=device).to(torch.int32)
     if seqlens is not None:
-        sl = torch.as_tensor(seqlens, dtype=torch.int32)
-    q = torch.randn(B, H, N, d, generator=g, dtype=torch.float32)
-    k = torch.randn(B, H, N, d, generator=g, dtype=torch.float32)
-    v = torch.randn(B, H, N, d, generator=g, dtype=torch.float32)
-    do = torch.randn(B, H, N, d, generator=g, dtype=torch.float32) if with_do else None
+        sl = torch.as_tensor(seqlens, dtype=torch.int32).to(device)
+    shape = (B, H, N, d)
+    q = torch.randn(shape, generator=g, dtype=torch.float32, device=device)
+    k = torch.randn(shape, generator=g, dtype=torch.float32, device=device)
+    v = torch.randn(shape, generator=g, dtype=torch.float32, device=device)
+    do = torch.randn(shape, generator=g, dtype=torch.float32, device=device) if with_do else None
     if ragged:
-        grow = 1.0 + 3.0 * torch.arange(N, dtype=torch.float32) / N
+        grow = 1.0 + 3.0 * torch.arange(N, dtype=torch.float32, device=device) / N
         k = k * grow[None, None, :, None]
     out = {"q": q.to(dtype), "k": k.to(dtype), "v": v.to(dtype),
            "do": do.to(dtype) if do is not None else None, "seqlens": sl}
     return out
 
 
-def make_inputs(name, dtype=None, seed=0, with_do=True):
+def make_inputs(name, dtype=None, seed=0, with_do=True, device="cpu"):
     """Inputs of a named workload (``WORKLOADS``) in ``dtype`` (default: its first)."""
     w = WORKLOADS[name]
     dt = dtype if dtype is not None else w.dtypes[0]
     return make_inputs_shape(w.B, w.H, w.N, w.d, dt, seed=seed, ragged=w.ragged,
-                             with_do=with_do)
+                             with_do=with_do, device=device)

@@ -1,0 +1,126 @@
+/*
+ * fa.h - C ABI of the B200 (sm_100a) exact tiled attention library
+ *        (libfa_b200.so).
+ *
+ * Operation.  Exact scaled-dot-product attention
+ *
+ *     O = softmax(scale * Q K^T  [+ causal / key-padding mask]) V
+ *
+ * computed tile by tile with an online softmax, so that no N x N score or
+ * probability matrix is ever written to device memory:
+ *   - "How Flash Attention Works" (swarnava.dev), section "The Exact-Attention
+ *     Idea": the result is the unchanged softmax(QK^T/sqrt(d))V, with causal
+ *     masking when asked for;
+ *   - same page, sections "Tiling Q, K, and V", "Online Softmax Without the
+ *     Full Score Matrix" and "Kernel Fusion": query tiles stay on chip, K/V
+ *     tiles stream past them, running row max and row sum rescale the partial
+ *     output, only O and per-row statistics reach memory;
+ *   - same page, section "The Backward Pass: Recomputation Instead of Stored
+ *     Activations": the backward pass keeps only O and the per-row statistics
+ *     and recomputes the score tiles;
+ *   - "attn-flash-equivalence" (zenaique.com), opening answer: the output
+ *     equals naive attention up to floating-point reduction order, so results
+ *     agree with a float64 evaluation within rounding, not bit for bit.
+ *
+ * Conventions shared by every entry point.
+ *   Layout.  Q, K, V, O, dO, dQ, dK, dV are dense, contiguous [B, H, N, d]
+ *     tensors (d innermost), 16-bit (bf16 or fp16, all the same type).
+ *     LSE is [B, H, N] float32, natural log:  LSE_i = ln sum_j exp(scale*s_ij)
+ *     over the visible keys.  seqlens is a device int32 [B] array or NULL.
+ *   Masks.  causal != 0 hides key j from query i when j > i (top-left
+ *     aligned; queries and keys have the same length N).  seqlens[b] = L
+ *     hides keys j >= L of batch b from every query (key padding); query rows
+ *     i >= L are still computed.  1 <= L <= N is required; other values are
+ *     clamped into range on the device and reported by fa_device_status().
+ *   Sizes.  B, H, N >= 1; d in {64, 128}; B*H*N*d < 2^31.
+ *   Scale.  finite and > 0 (typically 1/sqrt(d)).
+ *   Memory.  All pointers are device pointers owned by the caller, 16-byte
+ *     aligned.  The library allocates no device memory and keeps no state
+ *     other than cached driver entry points and per-device properties.
+ *   Streams.  stream is a cudaStream_t (NULL = legacy default stream).  Work
+ *     is enqueued asynchronously; no entry point synchronises except
+ *     fa_device_status().
+ *   Errors.  Return FA_OK or an fa_status code.  Argument errors are found on
+ *     the host before anything is launched.  Device-side conditions (bad
+ *     seqlens values, a pipeline wait that timed out) are written to a device
+ *     status word, read and cleared by fa_device_status().  The library never
+ *     aborts the process and never traps on the device.
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,     /* null pointer, size < 1, bad scale or dtype    */
+  FA_ERR_UNSUPPORTED = 2,     /* head dim not in {64, 128}, sizes too large     */
+  FA_ERR_ALIGNMENT = 3,       /* a pointer is not 16-byte aligned               */
+  FA_ERR_ARCH = 4,            /* current device is not an sm_100 (B200) GPU     */
+  FA_ERR_CUDA = 5,            /* a CUDA runtime/driver call or launch failed    */
+  FA_ERR_DEVICE_TIMEOUT = 6,  /* device: a pipeline wait gave up (fa_device_status) */
+  FA_ERR_DEVICE_SEQLEN = 7,   /* device: seqlens[b] outside [1, N] (fa_device_status) */
+  FA_ERR_WORKSPACE = 8        /* backward workspace missing or too small        */
+} fa_status;
+
+typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
+
+/*
+ * Forward pass.
+ *   in : q, k, v       [B, H, N, d] 16-bit
+ *   out: o             [B, H, N, d] 16-bit, rounded to nearest from fp32
+ *        lse           [B, H, N] float32 log-sum-exp of the scaled scores
+ *   Launches one persistent kernel on `stream`.
+ */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+           int B, int H, int N, int d, float scale, int causal,
+           const int32_t* seqlens, int dtype, void* stream);
+
+/*
+ * Bytes of device workspace fa_bwd needs: the row dots D = rowsum(dO * O)
+ * (float32 [B, H, N]) and the float32 dQ accumulator ([B, H, N, d]), each
+ * padded to 256 bytes.  Returns 0 for arguments fa_bwd would reject.
+ */
+size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Backward pass of the loss <dO, O> (gradients of the forward above).
+ *   in : q, k, v, o, dout  [B, H, N, d] 16-bit (o and lse from fa_fwd with the
+ *        same arguments), lse [B, H, N] float32
+ *   out: dq, dk, dv        [B, H, N, d] 16-bit; keys hidden by key padding get
+ *        exactly zero dK and dV
+ *   workspace: caller-owned device memory of at least
+ *        fa_bwd_workspace_size(B, H, N, d) bytes, 256-byte aligned; its
+ *        contents on entry do not matter and are overwritten.
+ *   Launches three kernels on `stream` (row-dot preprocess, main, dQ convert).
+ */
+int fa_bwd(const void* q, const void* k, const void* v, const void* o,
+           const void* dout, const float* lse, void* dq, void* dk, void* dv,
+           void* workspace, size_t workspace_bytes,
+           int B, int H, int N, int d, float scale, int causal,
+           const int32_t* seqlens, int dtype, void* stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device status word of
+ * the current device: FA_OK, FA_ERR_DEVICE_SEQLEN or FA_ERR_DEVICE_TIMEOUT
+ * (FA_ERR_CUDA if the synchronisation itself failed).  *detail, if not NULL,
+ * receives the raw word (code | site << 8 | block << 16).
+ */
+int fa_device_status(void* stream, uint32_t* detail);
+
+/* Static description of a status code.  Never NULL. */
+const char* fa_status_string(int status);
+
+/* Library ABI version: 100 * major + minor. */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

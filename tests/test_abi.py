@@ -1,0 +1,99 @@
+"""The C ABI library builds, loads and exports what include/fa.h declares;
+host-side argument checks answer without a GPU (no compute calls here)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from exact_io_aware_47_b200 import _lib, build
+    build.build()
+    return _lib.load()
+
+
+def _declared_functions():
+    names = []
+    for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"^\s*(?:[A-Za-z_][\w\s\*]*?)\b(fa_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_functions()
+    for want in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_size", "fa_device_status",
+                 "fa_status_string", "fa_version"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_binding_covers_every_declared_symbol():
+    from exact_io_aware_47_b200 import _lib
+    assert set(_declared_functions()) == set(_lib.SIGNATURES)
+
+
+def test_status_strings_and_version(lib):
+    for code in range(0, 10):
+        s = lib.fa_status_string(code)
+        assert isinstance(s, bytes) and len(s) > 0
+    assert lib.fa_version() == 100
+
+
+def test_workspace_size(lib):
+    B, H, N, d = 2, 3, 1000, 128
+    rows = B * H * N
+    r256 = lambda x: (x + 255) // 256 * 256
+    assert lib.fa_bwd_workspace_size(B, H, N, d) == r256(rows * 4) + r256(rows * d * 4)
+    assert lib.fa_bwd_workspace_size(B, H, N, 96) == 0
+    assert lib.fa_bwd_workspace_size(0, H, N, d) == 0
+
+
+def test_rejections_before_any_cuda_call(lib):
+    from exact_io_aware_47_b200 import _lib
+    P = 1 << 20  # never dereferenced: every case below fails validation first
+    ok = dict(B=1, H=2, N=128, d=64, scale=0.125, causal=1, seqlens=None, dtype=0)
+
+    def fwd(q=P, o=P, **kw):
+        a = {**ok, **kw}
+        return lib.fa_fwd(q, P, P, o, P, a["B"], a["H"], a["N"], a["d"], a["scale"], a["causal"],
+                          a["seqlens"], a["dtype"], None)
+    assert fwd(q=None) == _lib.FA_ERR_INVALID_ARG
+    assert fwd(B=0) == _lib.FA_ERR_INVALID_ARG
+    assert fwd(N=-3) == _lib.FA_ERR_INVALID_ARG
+    assert fwd(scale=0.0) == _lib.FA_ERR_INVALID_ARG
+    assert fwd(scale=float("inf")) == _lib.FA_ERR_INVALID_ARG
+    assert fwd(dtype=2) == _lib.FA_ERR_INVALID_ARG
+    assert fwd(d=32) == _lib.FA_ERR_UNSUPPORTED
+    assert fwd(B=1 << 12, H=1 << 10, N=1 << 10, d=64) == _lib.FA_ERR_UNSUPPORTED
+    assert fwd(q=P + 8) == _lib.FA_ERR_ALIGNMENT
+    assert fwd(seqlens=P + 2) == _lib.FA_ERR_ALIGNMENT
+
+    ws = lib.fa_bwd_workspace_size(1, 2, 128, 64)
+
+    def bwd(wsp=P, wsb=ws, **kw):
+        a = {**ok, **kw}
+        return lib.fa_bwd(P, P, P, P, P, P, P, P, P, wsp, wsb, a["B"], a["H"], a["N"], a["d"],
+                          a["scale"], a["causal"], a["seqlens"], a["dtype"], None)
+    assert bwd(wsp=None) == _lib.FA_ERR_WORKSPACE
+    assert bwd(wsb=ws - 1) == _lib.FA_ERR_WORKSPACE
+    assert bwd(wsp=P + 16) == _lib.FA_ERR_ALIGNMENT
+    assert bwd(d=100) == _lib.FA_ERR_UNSUPPORTED
+    assert bwd(H=0) == _lib.FA_ERR_INVALID_ARG
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    from exact_io_aware_47_b200 import _lib
+    with pytest.raises(RuntimeError, match="missing"):
+        _lib.load(str(tmp_path / "nope.so"))
