@@ -1,0 +1,399 @@
+"""Throughput of exact tiled attention (forward + backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is the whole hot path over one batch: fa_fwd, then the three
+backward stages (row-dot preprocess, main kernel, dQ convert), on the
+mid-context workload B=2, H=32, N=8192, d=128, bf16, causal (synthetic
+N(0,1) inputs, 128 MiB per tensor, so every step's inputs exceed the 126 MB
+L2).  The metric is attention TFLOP/s: forward 4*B*H*N^2*d/2 (causal),
+backward 2.5x that.
+
+With N > 1 (torchrun), every rank runs its own replica of the workload (the
+op has no cross-GPU exchange); the time is the max over ranks and the value
+counts the work of all ranks.
+
+``--impl reference`` times the float64 CPU oracle (test infrastructure, the
+only other place this script runs it) on bounded samples of the same
+workload.
+"""
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd/bwd TFLOP/s on 1 B200 and fraction of bf16 tensor-core peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def flops_fwd(B, H, N, d, causal):
+    f = 4.0 * B * H * N * N * d
+    return f / 2 if causal else f
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="mid")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "exact_io_aware_47_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        if fn.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, fn), "rb") as f:
+                h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, or None if the
+    kernel sources changed since it was captured."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel, {})
+    if e.get("workload") != workload or e.get("source_sha") != kernel_source_sha():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if "Active" in v
+                          and "Not" not in v})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup():
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl" if torch.cuda.is_available() else "gloo",
+                                timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def dist_max(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------- CPU oracle
+def oracle_sample(w, n_rows, seed=0):
+    """Time the float64 oracle (forward + backward) on one (batch, head) slice of
+    the workload cut to its first n_rows queries and keys.  Returns
+    (seconds, algorithmic flops of the sample, threads)."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+    from exact_io_aware_47_b200.inputs import make_inputs_shape
+    from oracle import ref_bwd_slice, ref_fwd_slice
+    inp = make_inputs_shape(1, 1, n_rows, w.d, w.dtypes[0], seed=seed, ragged=False)
+    q, k, v, do = (inp[n][0, 0].double().numpy() for n in ("q", "k", "v", "do"))
+    t0 = time.perf_counter()
+    ref_fwd_slice(q, k, v, w.scale, w.causal)
+    ref_bwd_slice(q, k, v, do, w.scale, w.causal)
+    dt = time.perf_counter() - t0
+    fl = 3.5 * flops_fwd(1, 1, n_rows, w.d, w.causal)
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    return dt, fl, threads
+
+
+def run_reference(args, w):
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return 0
+    n_rows = 2048
+    for _ in range(args.warmup):
+        oracle_sample(w, n_rows)
+    tot_t, tot_f, thr = 0.0, 0.0, 1
+    for s in range(args.steps):
+        dt, fl, thr = oracle_sample(w, n_rows, seed=s)
+        tot_t += dt
+        tot_f += fl
+    value = tot_f / tot_t / 1e12
+    sample = (f"per step: float64 oracle forward+backward of one (batch, head) slice of "
+              f"'{w.name}' cut to its first {n_rows} queries/keys")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.description, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------- CUDA path
+def run_ours(args, w):
+    import torch
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from exact_io_aware_47_b200 import _lib, build
+    build.build()
+    import exact_io_aware_47_b200 as fa
+    from exact_io_aware_47_b200.inputs import make_inputs
+
+    B, H, N, d = w.B, w.H, w.N, w.d
+    dtype = w.dtypes[0]
+    causal, scale = w.causal, w.scale
+    inp = make_inputs(w.name, dtype=dtype, seed=rank, device=dev)
+    q, k, v, do = inp["q"], inp["k"], inp["v"], inp["do"]
+    sl = inp["seqlens"]
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_bytes = fa.workspace_bytes(B, H, N, d)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    dt_code = _lib.FA_BF16 if dtype == torch.bfloat16 else _lib.FA_FP16
+    slp = sl.data_ptr() if sl is not None else None
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        _lib.check("fa_fwd", _lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                         lse.data_ptr(), B, H, N, d, scale, int(causal), slp,
+                                         dt_code, sh))
+        if ev is not None:
+            ev[1].record(stream)
+        _lib.check("pre", _lib.fa_bwd_preprocess(o.data_ptr(), do.data_ptr(), ws.data_ptr(),
+                                                 ws_bytes, B, H, N, d, dt_code, sh))
+        if ev is not None:
+            ev[2].record(stream)
+        _lib.check("main", _lib.fa_bwd_main(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                            do.data_ptr(), lse.data_ptr(), dk.data_ptr(),
+                                            dv.data_ptr(), ws.data_ptr(), ws_bytes, B, H, N, d,
+                                            scale, int(causal), slp, dt_code, sh))
+        if ev is not None:
+            ev[3].record(stream)
+        _lib.check("post", _lib.fa_bwd_postprocess(ws.data_ptr(), ws_bytes, dq.data_ptr(), B, H,
+                                                   N, d, scale, dt_code, sh))
+        if ev is not None:
+            ev[4].record(stream)
+
+    warmup = max(3, args.warmup)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    st, word = _lib.fa_device_status(sh)
+    if st != 0:
+        raise RuntimeError(f"device status {st} ({word:#x}) after warm-up")
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    if not args.no_clocks:
+        clocks.start()
+        time.sleep(0.3)
+    dist_barrier(world)
+    torch.cuda.synchronize(dev)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(K):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    dist_barrier(world)
+    clk = None if args.no_clocks else clocks.stop()
+    st, word = _lib.fa_device_status(sh)
+    if st != 0:
+        raise RuntimeError(f"device status {st} ({word:#x}) after timing")
+
+    total_ms = dist_max(t_start.elapsed_time(t_end), world)
+    parts = {"fa_fwd_kernel": [], "fa_bwd_pre": [], "fa_bwd_kernel": [], "fa_bwd_post": []}
+    for e in evs:
+        parts["fa_fwd_kernel"].append(e[0].elapsed_time(e[1]))
+        parts["fa_bwd_pre"].append(e[1].elapsed_time(e[2]))
+        parts["fa_bwd_kernel"].append(e[2].elapsed_time(e[3]))
+        parts["fa_bwd_post"].append(e[3].elapsed_time(e[4]))
+    avg = {n: sum(v_) / len(v_) for n, v_ in parts.items()}
+
+    f_fwd = flops_fwd(B, H, N, d, causal)
+    f_bwd = 2.5 * f_fwd
+    step_flops = f_fwd + f_bwd
+    ms_per_step = total_ms / K
+    value = world * step_flops * K / (total_ms / 1e3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    dom = max(("fa_fwd_kernel", "fa_bwd_kernel"), key=lambda n: avg[n])
+    dom_flops = f_fwd if dom == "fa_fwd_kernel" else f_bwd
+    achieved = dom_flops / (avg[dom] / 1e3) / 1e12
+    traffic = recorded_traffic(dom, w.name)
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                "peak_source": f"{peak_src} bf16 dense (burst)",
+                "flops_per_launch": dom_flops}
+    fwd_tf = f_fwd / (avg["fa_fwd_kernel"] / 1e3) / 1e12
+    bwd_ms = avg["fa_bwd_pre"] + avg["fa_bwd_kernel"] + avg["fa_bwd_post"]
+    bwd_tf = f_bwd / (bwd_ms / 1e3) / 1e12
+    kernels = {n: {"ms": avg[n], "share": avg[n] / ms_per_step} for n in avg}
+
+    # end to end through the public API: pinned host inputs in, results out
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
+        ho, hdq, hdk, hdv = (torch.empty(q.shape, dtype=dtype, pin_memory=True) for _ in range(4))
+        hlse = torch.empty((B, H, N), dtype=torch.float32, pin_memory=True)
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
+        d2h = sum(t.numel() * t.element_size() for t in (ho, hlse, hdq, hdk, hdv))
+
+        def e2e_step():
+            for src, dst in ((hq, q), (hk, k), (hv, v), (hdo, do)):
+                dst.copy_(src, non_blocking=True)
+            fa.forward(q, k, v, scale=scale, causal=causal, seqlens=sl, out=o, lse=lse)
+            fa.backward(q, k, v, o, lse, do, scale=scale, causal=causal, seqlens=sl,
+                        workspace=ws, dq=dq, dk=dk, dv=dv)
+            for src, dst in ((o, ho), (lse, hlse), (dq, hdq), (dk, hdk), (dv, hdv)):
+                dst.copy_(src, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        ke = max(3, min(K, 10))
+        dist_barrier(world)
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(ke):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        dist_barrier(world)
+        e_ms = dist_max(a.elapsed_time(b), world)
+        e2e = {"value": world * step_flops * ke / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e_ms / ke}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n_rows = 4096
+        dt, fl, thr = oracle_sample(w, n_rows)
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+               "sample": f"float64 oracle forward+backward of one (batch, head) slice of "
+                         f"'{w.name}' cut to its first {n_rows} queries/keys ({dt:.1f} s)"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if dtype == torch.bfloat16 else "f16",
+        "data": "synthetic",
+        "config": {"workload": w.description, "B": B, "H": H, "N": N, "d": d, "causal": causal,
+                   "step": "fa_fwd + fa_bwd_preprocess + fa_bwd_main + fa_bwd_postprocess",
+                   "flops_per_step": step_flops, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (4 x 128 MiB per step), no flush"},
+        "fwd": {"ms": avg["fa_fwd_kernel"], "tflops": fwd_tf, "frac": fwd_tf / peak},
+        "bwd": {"ms": bwd_ms, "tflops": bwd_tf, "frac": bwd_tf / peak},
+        "kernels": kernels,
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": 4 * K,
+        "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    from exact_io_aware_47_b200.inputs import WORKLOADS
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

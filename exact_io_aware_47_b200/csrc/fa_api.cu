@@ -140,55 +140,120 @@ extern "C" size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   return round256(rows * sizeof(float)) + round256(rows * d * sizeof(float));
 }
 
-extern "C" int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
-                      const float* lse, void* dq, void* dk, void* dv, void* workspace,
-                      size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
-                      const int32_t* seqlens, int dtype, void* stream) {
-  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+namespace fa {
+namespace {
+
+// Checks shared by the backward stages; fills the workspace carving.
+int bwd_common(void* workspace, size_t workspace_bytes, int B, int H, int N, int d, float scale,
+               int dtype, const int32_t* seqlens, BwdParams* p, DeviceInfo* di) {
   int st = check_common(B, H, N, d, scale, dtype);
   if (st != FA_OK) return st;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
-      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
-      (seqlens && (reinterpret_cast<uintptr_t>(seqlens) & 3u)))
-    return FA_ERR_ALIGNMENT;
+  if (seqlens && (reinterpret_cast<uintptr_t>(seqlens) & 3u)) return FA_ERR_ALIGNMENT;
   const size_t need = fa_bwd_workspace_size(B, H, N, d);
   if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FA_ERR_ALIGNMENT;
-  DeviceInfo di;
-  st = current_device_info(&di);
+  st = current_device_info(di);
   if (st != FA_OK) return st;
+  const size_t rows = static_cast<size_t>(B) * H * N;
+  std::memset(p, 0, sizeof(*p));
+  p->dsum = static_cast<float*>(workspace);
+  p->dq_acc =
+      reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round256(rows * sizeof(float)));
+  p->seqlens = seqlens;
+  p->B = B;
+  p->H = H;
+  p->N = N;
+  p->scale = scale;
+  p->scale_log2 = scale * 1.4426950408889634f;
+  p->n_ktiles = (N + kBlockN - 1) / kBlockN;
+  p->n_units = B * H * p->n_ktiles;
+  return FA_OK;
+}
 
+}  // namespace
+}  // namespace fa
+
+extern "C" int fa_bwd_preprocess(const void* o, const void* dout, void* workspace,
+                                 size_t workspace_bytes, int B, int H, int N, int d, int dtype,
+                                 void* stream) {
+  if (!o || !dout) return FA_ERR_INVALID_ARG;
+  if (!aligned16(o) || !aligned16(dout)) return FA_ERR_ALIGNMENT;
+  BwdParams p;
+  DeviceInfo di;
+  int st = bwd_common(workspace, workspace_bytes, B, H, N, d, 1.f, dtype, nullptr, &p, &di);
+  if (st != FA_OK) return st;
+  p.o = o;
+  p.dout = dout;
+  const cudaError_t e = launch_bwd_pre(d, dtype == FA_BF16, p, di.num_sms,
+                                       static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+extern "C" int fa_bwd_main(const void* q, const void* k, const void* v, const void* dout,
+                           const float* lse, void* dk, void* dv, void* workspace,
+                           size_t workspace_bytes, int B, int H, int N, int d, float scale,
+                           int causal, const int32_t* seqlens, int dtype, void* stream) {
+  if (!q || !k || !v || !dout || !lse || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(lse) ||
+      !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_ALIGNMENT;
+  BwdParams p;
+  DeviceInfo di;
+  int st = bwd_common(workspace, workspace_bytes, B, H, N, d, scale, dtype, seqlens, &p, &di);
+  if (st != FA_OK) return st;
   CUtensorMap tq, tk, tv, tdo;
   const int BH = B * H;
   if (make_map(&tq, q, BH, N, d, dtype) != FA_OK || make_map(&tk, k, BH, N, d, dtype) != FA_OK ||
       make_map(&tv, v, BH, N, d, dtype) != FA_OK || make_map(&tdo, dout, BH, N, d, dtype) != FA_OK)
     return FA_ERR_CUDA;
-
-  const size_t rows = static_cast<size_t>(BH) * N;
-  BwdParams p;
   p.q = q;
   p.k = k;
   p.v = v;
-  p.o = o;
   p.dout = dout;
   p.lse = lse;
-  p.dq = dq;
   p.dk = dk;
   p.dv = dv;
-  p.dsum = static_cast<float*>(workspace);
-  p.dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round256(rows * sizeof(float)));
-  p.seqlens = seqlens;
-  p.B = B;
-  p.H = H;
-  p.N = N;
-  p.scale = scale;
-  p.scale_log2 = scale * 1.4426950408889634f;
   p.causal = causal ? 1 : 0;
-  p.n_ktiles = (N + kBlockN - 1) / kBlockN;
-  p.n_units = BH * p.n_ktiles;
-  const cudaError_t e = launch_bwd(d, dtype == FA_BF16, tq, tk, tv, tdo, p, di.num_sms,
-                                   static_cast<cudaStream_t>(stream));
+  const cudaError_t e = launch_bwd_main(d, dtype == FA_BF16, tq, tk, tv, tdo, p, di.num_sms,
+                                        static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+extern "C" int fa_bwd_postprocess(void* workspace, size_t workspace_bytes, void* dq, int B, int H,
+                                  int N, int d, float scale, int dtype, void* stream) {
+  if (!dq) return FA_ERR_INVALID_ARG;
+  if (!aligned16(dq)) return FA_ERR_ALIGNMENT;
+  BwdParams p;
+  DeviceInfo di;
+  int st = bwd_common(workspace, workspace_bytes, B, H, N, d, scale, dtype, nullptr, &p, &di);
+  if (st != FA_OK) return st;
+  p.dq = dq;
+  const cudaError_t e = launch_bwd_post(d, dtype == FA_BF16, p, di.num_sms,
+                                        static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+extern "C" int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                      const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                      size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
+                      const int32_t* seqlens, int dtype, void* stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  // validate everything before the first launch, so a rejected call enqueues nothing
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_ALIGNMENT;
+  {
+    BwdParams p;
+    DeviceInfo di;
+    const int st = bwd_common(workspace, workspace_bytes, B, H, N, d, scale, dtype, seqlens, &p, &di);
+    if (st != FA_OK) return st;
+  }
+  int st = fa_bwd_preprocess(o, dout, workspace, workspace_bytes, B, H, N, d, dtype, stream);
+  if (st != FA_OK) return st;
+  st = fa_bwd_main(q, k, v, dout, lse, dk, dv, workspace, workspace_bytes, B, H, N, d, scale,
+                   causal, seqlens, dtype, stream);
+  if (st != FA_OK) return st;
+  return fa_bwd_postprocess(workspace, workspace_bytes, dq, B, H, N, d, scale, dtype, stream);
 }
 
 extern "C" int fa_device_status(void* stream, uint32_t* detail) {
@@ -202,6 +267,7 @@ extern "C" int fa_device_status(void* stream, uint32_t* detail) {
   const unsigned code = word & 0xffu;
   if (code == kErrDeviceTimeout) return FA_ERR_DEVICE_TIMEOUT;
   if (code == kErrDeviceSeqlen) return FA_ERR_DEVICE_SEQLEN;
+  if (code == kErrDeviceLayout) return FA_ERR_DEVICE_LAYOUT;
   return word == 0 ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -216,6 +282,7 @@ extern "C" const char* fa_status_string(int status) {
     case FA_ERR_DEVICE_TIMEOUT: return "device pipeline wait timed out";
     case FA_ERR_DEVICE_SEQLEN: return "seqlens value outside [1, N] (clamped on device)";
     case FA_ERR_WORKSPACE: return "backward workspace missing or too small";
+    case FA_ERR_DEVICE_LAYOUT: return "kernel refused: shared-memory window misaligned";
     default: return "unknown status";
   }
 }

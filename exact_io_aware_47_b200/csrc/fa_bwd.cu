@@ -1,13 +1,584 @@
-// Backward pass (placeholder launcher; kernels follow).
+// Backward exact attention on sm_100a, by recomputation.
+//
+// "How Flash Attention Works" (swarnava.dev), section "The Backward Pass:
+// Recomputation Instead of Stored Activations": only O and the per-row
+// statistics are kept from the forward pass; the score tiles are recomputed
+// tile by tile inside one fused kernel.  The statistic kept here is the
+// log-sum-exp LSE_i, so P_ij = exp(scale * s_ij - LSE_i) is rebuilt exactly.
+// With D_i = <dO_i, O_i> (the softmax-backward row term), the gradients are
+//   dV = P^T dO,  dP = dO V^T,  dS = P * (dP - D),  dQ = scale dS K,
+//   dK = scale dS^T Q.
+//
+// Three kernels:
+//  1. fa_bwd_pre: D_i = sum_c dO_ic O_ic (fp32) and zero the fp32 dQ
+//     accumulator;
+//  2. fa_bwd_kernel (persistent, one CTA per SM, 384 threads): a work unit is
+//     (batch*head, 128-key tile j).  K_j and V_j stay in shared memory while
+//     the query tiles i (i >= j when causal) stream past:
+//       S^T  = K_j Q_i^T      (tcgen05, TMEM, keys on lanes)
+//       dP^T = V_j dO_i^T     (tcgen05, TMEM)
+//       P^T  = exp2(c S^T - LSE_i log2 e), dS^T = P^T * (dP^T - D_i)
+//                              (warps 0-3, one key row per thread; P^T goes
+//                              back to TMEM over S^T as 16-bit, dS^T to a
+//                              swizzled shared-memory tile)
+//       dV_j += P^T dO_i,  dK_j += dS^T Q_i   (TMEM accumulators)
+//       dQ_i  = dS K_j     (TMEM; warps 4-7 reduce-add it into the fp32
+//                           accumulator in global memory)
+//     warp 8 issues the MMAs, warp 9 the TMA loads, warp 10 stages LSE_i and
+//     D_i in shared memory; warps 4-7 also write dK_j (times scale) and dV_j
+//     at the end of the unit;
+//  3. fa_bwd_post: dQ = scale * accumulator, rounded to 16-bit.
+//
+// TMEM columns: S^T/P^T [0,128), dP^T [128,256), dV [256,256+d),
+// dK [256+d,256+2d); dQ_i reuses the dP^T columns when d = 128 (the 512
+// columns are all taken) and [384,448) when d = 64.
+#include <algorithm>
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
 #include "fa_internal.h"
 #include "sm100.cuh"
 
 namespace fa {
 
-cudaError_t launch_bwd(int d, bool bf16, const CUtensorMap& tmq, const CUtensorMap& tmk,
-                       const CUtensorMap& tmv, const CUtensorMap& tmdo, const BwdParams& p,
-                       int num_sms, cudaStream_t stream) {
-  return cudaErrorNotSupported;
+template <int D>
+struct BwdLayout {
+  static constexpr int kTileBytes = 128 * D * 2;
+  static constexpr int kPanelBytes = 128 * 64 * 2;
+  static constexpr int kPanels = D / 64;
+  static constexpr int kK = 0;
+  static constexpr int kV = kTileBytes;
+  static constexpr int kQ = 2 * kTileBytes;            // 2 stages
+  static constexpr int kDO = kQ + 2 * kTileBytes;      // 2 stages
+  static constexpr int kDS = kDO + 2 * kTileBytes;     // dS^T, 128 x 128 16-bit
+  static constexpr int kLSE = kDS + 128 * 128 * 2;     // 2 stages x 128 fp32
+  static constexpr int kDSUM = kLSE + 2 * 128 * 4;     // 2 stages x 128 fp32
+  static constexpr int kBar = kDSUM + 2 * 128 * 4;
+  static constexpr int kBarBytes = 256;
+  static constexpr int kUsed = kBar + kBarBytes;
+  static constexpr int kSmemMax = 232448;              // sm_100 per-block opt-in maximum
+  static constexpr int kSmemBytes = (kUsed + 1024 <= kSmemMax) ? kUsed + 1024 : kSmemMax;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColS = 0;
+  static constexpr uint32_t kColDP = 128;
+  static constexpr uint32_t kColDV = 256;
+  static constexpr uint32_t kColDK = 256 + D;
+  static constexpr uint32_t kColDQ = (D == 128) ? 128 : 256 + 2 * D;
+};
+
+struct BwdUnit {
+  int bh, j, L, i0, ni;
+};
+
+__device__ __forceinline__ BwdUnit bwd_decode(int u, const BwdParams& p) {
+  BwdUnit w;
+  w.bh = u / p.n_ktiles;
+  w.j = u % p.n_ktiles;  // causal: small j has the most query tiles, so runs first
+  const int b = w.bh / p.H;
+  int L = p.N;
+  if (p.seqlens != nullptr) {
+    L = p.seqlens[b];
+    L = L < 1 ? 1 : (L > p.N ? p.N : L);
+  }
+  w.L = L;
+  w.i0 = p.causal ? w.j : 0;
+  w.ni = (w.j * kBlockN < L) ? (p.n_ktiles - w.i0) : 0;  // a key tile past L only gets zeros
+  return w;
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(384, 1)
+    fa_bwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                  const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdo,
+                  const BwdParams p) {
+  using Lay = BwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  if (smem + Lay::kUsed > smem_raw + Lay::kSmemBytes) {
+    // the dynamic shared-memory window is not aligned well enough: refuse
+    if (threadIdx.x == 0) record_error(kErrDeviceLayout, 0);
+    return;
+  }
+  uint8_t* sK = smem + Lay::kK;
+  uint8_t* sV = smem + Lay::kV;
+  uint8_t* sQ = smem + Lay::kQ;
+  uint8_t* sDO = smem + Lay::kDO;
+  uint8_t* sDS = smem + Lay::kDS;
+  float* sLSE = reinterpret_cast<float*>(smem + Lay::kLSE);
+  float* sDSUM = reinterpret_cast<float*>(smem + Lay::kDSUM);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* kv_empty = bars + 1;
+  uint64_t* q_full = bars + 2;     // [2]
+  uint64_t* q_empty = bars + 4;    // [2]
+  uint64_t* ld_full = bars + 6;    // [2]
+  uint64_t* ld_empty = bars + 8;   // [2]
+  uint64_t* s_full = bars + 10;
+  uint64_t* dp_full = bars + 11;
+  uint64_t* p_full = bars + 12;
+  uint64_t* ds_empty = bars + 13;
+  uint64_t* dq_full = bars + 14;
+  uint64_t* dq_empty = bars + 15;
+  uint64_t* dkv_full = bars + 16;
+  uint64_t* dkv_empty = bars + 17;
+  uint64_t* drain = bars + 18;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    mbar_init(kv_empty, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+      mbar_init(&ld_full[s], 32);
+      mbar_init(&ld_empty[s], 128);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(p_full, 128);
+    mbar_init(ds_empty, 1);
+    mbar_init(dq_full, 1);
+    mbar_init(dq_empty, 128);
+    mbar_init(dkv_full, 1);
+    mbar_init(dkv_empty, 128);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(tmem_slot, Lay::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 9) {
+    // ------------------------------------------------------------- TMA loads
+    if (lane == 0) {
+      tma_prefetch_desc(&tmq);
+      tma_prefetch_desc(&tmk);
+      tma_prefetch_desc(&tmv);
+      tma_prefetch_desc(&tmdo);
+      int nunit = 0, qseq = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        const BwdUnit w = bwd_decode(u, p);
+        ok = mbar_wait(kv_empty, (nunit & 1) ^ 1, abort_flag, 20);
+        if (!ok) break;
+        mbar_arrive_expect_tx(kv_full, 2 * Lay::kTileBytes);
+#pragma unroll
+        for (int pn = 0; pn < Lay::kPanels; ++pn) {
+          tma_load_3d(sK + pn * Lay::kPanelBytes, &tmk, kv_full, pn * 64, w.j * kBlockN, w.bh);
+          tma_load_3d(sV + pn * Lay::kPanelBytes, &tmv, kv_full, pn * 64, w.j * kBlockN, w.bh);
+        }
+        ++nunit;
+        for (int idx = 0; idx < w.ni && ok; ++idx) {
+          const int i = w.i0 + idx;
+          const int st = qseq & 1;
+          ok = mbar_wait(&q_empty[st], ((qseq >> 1) & 1) ^ 1, abort_flag, 21);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&q_full[st], 2 * Lay::kTileBytes);
+#pragma unroll
+          for (int pn = 0; pn < Lay::kPanels; ++pn) {
+            tma_load_3d(sQ + st * Lay::kTileBytes + pn * Lay::kPanelBytes, &tmq, &q_full[st],
+                        pn * 64, i * kBlockM, w.bh);
+            tma_load_3d(sDO + st * Lay::kTileBytes + pn * Lay::kPanelBytes, &tmdo, &q_full[st],
+                        pn * 64, i * kBlockM, w.bh);
+          }
+          ++qseq;
+        }
+      }
+      if (nunit > 0) mbar_wait_drain(kv_full, (nunit - 1) & 1, 200000000ull);
+      for (int s = 0; s < 2; ++s) {
+        if (qseq > s) {
+          const int last = qseq - 1 - ((qseq - 1 - s) & 1);
+          mbar_wait_drain(&q_full[s], (last >> 1) & 1, 200000000ull);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 10) {
+    // ------------------------------------------------ LSE_i, D_i -> shared memory
+    int seq = 0;
+    bool ok = true;
+    const float log2e = 1.4426950408889634f;
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      const BwdUnit w = bwd_decode(u, p);
+      const size_t base = static_cast<size_t>(w.bh) * p.N;
+      for (int idx = 0; idx < w.ni && ok; ++idx) {
+        const int i = w.i0 + idx;
+        const int st = seq & 1;
+        ok = mbar_wait_warp(&ld_empty[st], ((seq >> 1) & 1) ^ 1, abort_flag, 22);
+        if (!ok) break;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int ql = lane * 4 + e;
+          const int q = i * kBlockM + ql;
+          // rows past N: LSE = +inf makes P = 0 there, D = 0
+          sLSE[st * 128 + ql] = q < p.N ? p.lse[base + q] * log2e : INFINITY;
+          sDSUM[st * 128 + ql] = q < p.N ? p.dsum[base + q] : 0.f;
+        }
+        mbar_arrive(&ld_full[st]);
+        ++seq;
+      }
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      constexpr uint32_t kIdS = idesc_f16(BF16, 128, 128, false, false);  // S^T, dP^T
+      constexpr uint32_t kIdTS = idesc_f16(BF16, 128, D, false, true);    // dV, dK (B MN-major)
+      constexpr uint32_t kIdDQ = idesc_f16(BF16, 128, D, true, true);     // dQ (A, B MN-major)
+      const uint32_t aK = smem_addr(sK), aV = smem_addr(sV), aQ = smem_addr(sQ),
+                     aDO = smem_addr(sDO), aDS = smem_addr(sDS);
+      int nunit = 0, qseq = 0, it = 0;
+      bool ok = true;
+      // K-major operands (A and B): 16-element steps walk 32 bytes inside a
+      // 64-column panel, panels are 16 KB apart.
+      auto kmaj = [](uint32_t base, int kk) {
+        return sdesc_sw128(base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+      };
+      // MN-major operands: 16 rows of K = 2048 bytes; 64-column MN panels
+      // 16 KB apart (leading byte offset).
+      auto mnmaj = [](uint32_t base, int kk) {
+        return sdesc_sw128(base + kk * 2048, 16384, 1024);
+      };
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        const BwdUnit w = bwd_decode(u, p);
+        ok = mbar_wait(kv_full, nunit & 1, abort_flag, 23);
+        if (!ok) break;
+        tc_fence_after();
+        for (int idx = 0; idx < w.ni && ok; ++idx) {
+          const int st = qseq & 1;
+          ok = mbar_wait(&q_full[st], (qseq >> 1) & 1, abort_flag, 24);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t q_s = aQ + st * Lay::kTileBytes;
+          const uint32_t do_s = aDO + st * Lay::kTileBytes;
+          // S^T = K_j Q_i^T
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            umma_ss(tmem + Lay::kColS, kmaj(aK, kk), kmaj(q_s, kk), kIdS, kk > 0);
+          umma_commit(s_full);
+          if (it > 0) {
+            ok = mbar_wait(dq_empty, (it - 1) & 1, abort_flag, 25);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          // dP^T = V_j dO_i^T
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            umma_ss(tmem + Lay::kColDP, kmaj(aV, kk), kmaj(do_s, kk), kIdS, kk > 0);
+          umma_commit(dp_full);
+          ok = mbar_wait(p_full, it & 1, abort_flag, 26);
+          if (!ok) break;
+          tc_fence_after();
+          if (idx == 0 && nunit > 0) {
+            ok = mbar_wait(dkv_empty, (nunit - 1) & 1, abort_flag, 27);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          // dV_j += P^T dO_i   (A = P^T in TMEM, 16 queries = 8 columns)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_ts(tmem + Lay::kColDV, tmem + Lay::kColS + kk * 8, mnmaj(do_s, kk), kIdTS,
+                    (idx > 0 || kk > 0) ? 1u : 0u);
+          // dK_j += dS^T Q_i   (A = dS^T in shared memory, K-major)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_ss(tmem + Lay::kColDK, kmaj(aDS, kk), mnmaj(q_s, kk), kIdTS,
+                    (idx > 0 || kk > 0) ? 1u : 0u);
+          // dQ_i = dS K_j      (A = the same dS^T tile read MN-major)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_ss(tmem + Lay::kColDQ, mnmaj(aDS, kk), mnmaj(aK, kk), kIdDQ, kk > 0);
+          umma_commit(dq_full);
+          umma_commit(&q_empty[st]);
+          umma_commit(ds_empty);
+          ++qseq;
+          ++it;
+        }
+        if (!ok) break;
+        umma_commit(dkv_full);
+        umma_commit(kv_empty);
+        ++nunit;
+      }
+      umma_commit(drain);
+      mbar_wait_drain(drain, 0, 200000000ull);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ----------------------------------------------- P^T and dS^T (key rows)
+    const int r = (warp << 5) | lane;  // key row in the tile = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tS = tmem + lane_off + Lay::kColS;
+    const uint32_t tDP = tmem + lane_off + Lay::kColDP;
+    const uint32_t ds_row = smem_addr(sDS) + r * 128;
+    const float cl = p.scale_log2;
+    int it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      const BwdUnit w = bwd_decode(u, p);
+      const bool key_ok = w.j * kBlockN + r < w.L;
+      for (int idx = 0; idx < w.ni && ok; ++idx) {
+        const int i = w.i0 + idx;
+        const int st = it & 1;  // LSE/D staging advances with the iteration count
+        ok = mbar_wait_warp(&ld_full[st], (it >> 1) & 1, abort_flag, 28) &&
+             mbar_wait_warp(s_full, it & 1, abort_flag, 29) &&
+             mbar_wait_warp(dp_full, it & 1, abort_flag, 30);
+        if (ok && it > 0) ok = mbar_wait_warp(ds_empty, (it - 1) & 1, abort_flag, 31);
+        if (!ok) break;
+        tc_fence_after();
+        const bool diag = p.causal && i == w.j;
+        const float* lse2 = sLSE + st * 128;
+        const float* dsm = sDSUM + st * 128;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t sr[32], dr[32];
+          tmem_ld32(tS + c * 32, sr);
+          tmem_ld32(tDP + c * 32, dr);
+          uint32_t pp[16], dd[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int q0 = c * 32 + e;
+            const bool v0 = key_ok && (!diag || r <= q0);
+            const bool v1 = key_ok && (!diag || r <= q0 + 1);
+            const float p0 = v0 ? ex2_approx(__uint_as_float(sr[e]) * cl - lse2[q0]) : 0.f;
+            const float p1 = v1 ? ex2_approx(__uint_as_float(sr[e + 1]) * cl - lse2[q0 + 1]) : 0.f;
+            const float g0 = p0 * (__uint_as_float(dr[e]) - dsm[q0]);
+            const float g1 = p1 * (__uint_as_float(dr[e + 1]) - dsm[q0 + 1]);
+            pp[e >> 1] = pack2<BF16>(p0, p1);
+            dd[e >> 1] = pack2<BF16>(g0, g1);
+          }
+          tmem_st16(tS + c * 16, pp);  // P^T over the already-read S^T columns
+          // dS^T row r, queries [32c, 32c+32): four 16-byte units of a 128-byte
+          // swizzled row in panel c/2
+          const uint32_t prow = ds_row + (c >> 1) * 16384;
+#pragma unroll
+          for (int w4 = 0; w4 < 4; ++w4) {
+            const uint32_t unit = ((c & 1) * 4 + w4) ^ (r & 7);
+            st_shared_v4(prow + unit * 16, dd[4 * w4], dd[4 * w4 + 1], dd[4 * w4 + 2],
+                         dd[4 * w4 + 3]);
+          }
+        }
+        tmem_st_wait();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(p_full);
+        mbar_arrive(&ld_empty[st]);
+        ++it;
+      }
+    }
+  } else if (warp < 8) {
+    // ------------------------------- dQ_i reduce-add; dK_j, dV_j at unit end
+    const int r = ((warp & 3) << 5) | lane;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    int it = 0, nunit = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      const BwdUnit w = bwd_decode(u, p);
+      const size_t base = static_cast<size_t>(w.bh) * p.N;
+      for (int idx = 0; idx < w.ni && ok; ++idx) {
+        const int i = w.i0 + idx;
+        ok = mbar_wait_warp(dq_full, it & 1, abort_flag, 32);
+        if (!ok) break;
+        tc_fence_after();
+        const int row = i * kBlockM + r;
+        float* dst = p.dq_acc + (base + (row < p.N ? row : 0)) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_off + Lay::kColDQ + c * 32, v);
+          if (row < p.N) {
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4)
+              red_add_v4(dst + c * 32 + q4 * 4, __uint_as_float(v[4 * q4]),
+                         __uint_as_float(v[4 * q4 + 1]), __uint_as_float(v[4 * q4 + 2]),
+                         __uint_as_float(v[4 * q4 + 3]));
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(dq_empty);
+        ++it;
+      }
+      if (!ok) break;
+      ok = mbar_wait_warp(dkv_full, nunit & 1, abort_flag, 33);
+      if (!ok) break;
+      tc_fence_after();
+      const int key = w.j * kBlockN + r;
+      const bool keep = key < w.L;  // padded keys get exactly zero
+      const bool store = key < p.N;
+      const size_t off = (base + (store ? key : 0)) * (D * 2);
+      uint8_t* dvrow = reinterpret_cast<uint8_t*>(p.dv) + off;
+      uint8_t* dkrow = reinterpret_cast<uint8_t*>(p.dk) + off;
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        const uint32_t col = part == 0 ? Lay::kColDV : Lay::kColDK;
+        const float mul = part == 0 ? 1.f : p.scale;
+        uint8_t* rowp = part == 0 ? dvrow : dkrow;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          if (w.ni > 0) {
+            tmem_ld32(tmem + lane_off + col + c * 32, v);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = 0u;
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float a = keep ? __uint_as_float(v[2 * e]) * mul : 0.f;
+            const float b = keep ? __uint_as_float(v[2 * e + 1]) * mul : 0.f;
+            pk[e] = pack2<BF16>(a, b);
+          }
+          if (store) {
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              st_global_v4(rowp + c * 64 + v4 * 16, pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2],
+                           pk[4 * v4 + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(dkv_empty);
+      ++nunit;
+    }
+  }
+  // warp 11 has no role
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Lay::kTmemCols);
+  }
+}
+
+// D_i = <dO_i, O_i> in fp32 from the stored 16-bit values; zero the fp32 dQ
+// accumulator.  D/8 threads per row, 16-byte loads.
+template <int D, bool BF16>
+__global__ void __launch_bounds__(256) fa_bwd_pre(const uint4* __restrict__ o,
+                                                  const uint4* __restrict__ dout,
+                                                  float* __restrict__ dsum,
+                                                  float4* __restrict__ dq_acc, long long rows) {
+  constexpr int T = D / 8;
+  const long long total = rows * T;
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  // whole warps iterate together so the row-group shuffles see every lane
+  for (long long wbase = blockIdx.x * static_cast<long long>(blockDim.x) + (threadIdx.x & ~31);
+       wbase < total; wbase += stride) {
+    const long long g = wbase + (threadIdx.x & 31);
+    const bool live = g < total;
+    float s = 0.f;
+    if (live) {
+      const uint4 a = o[g];
+      const uint4 b = dout[g];
+      const uint32_t av[4] = {a.x, a.y, a.z, a.w};
+      const uint32_t bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float2 fa, fb;
+        if constexpr (BF16) {
+          fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&av[e]));
+          fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bv[e]));
+        } else {
+          fa = __half22float2(*reinterpret_cast<const __half2*>(&av[e]));
+          fb = __half22float2(*reinterpret_cast<const __half2*>(&bv[e]));
+        }
+        s = fmaf(fa.x, fb.x, s);
+        s = fmaf(fa.y, fb.y, s);
+      }
+      const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+      dq_acc[2 * g] = z;
+      dq_acc[2 * g + 1] = z;
+    }
+#pragma unroll
+    for (int m = T / 2; m > 0; m >>= 1) s += __shfl_xor_sync(0xffffffffu, s, m, T);
+    if (live && (g & (T - 1)) == 0) dsum[g / T] = s;
+  }
+}
+
+// dQ = scale * accumulator -> 16-bit; 8 values per thread.
+template <bool BF16>
+__global__ void __launch_bounds__(256) fa_bwd_post(const float4* __restrict__ acc,
+                                                   uint4* __restrict__ dq, float scale,
+                                                   long long n8) {
+  for (long long g = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; g < n8;
+       g += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float4 a = acc[2 * g];
+    const float4 b = acc[2 * g + 1];
+    uint4 r;
+    r.x = pack2<BF16>(a.x * scale, a.y * scale);
+    r.y = pack2<BF16>(a.z * scale, a.w * scale);
+    r.z = pack2<BF16>(b.x * scale, b.y * scale);
+    r.w = pack2<BF16>(b.z * scale, b.w * scale);
+    dq[g] = r;
+  }
+}
+
+static int elementwise_grid(long long n8, int num_sms) {
+  return static_cast<int>(std::max<long long>(1, std::min<long long>((n8 + 255) / 256, num_sms * 16ll)));
+}
+
+cudaError_t launch_bwd_pre(int d, bool bf16, const BwdParams& p, int num_sms,
+                           cudaStream_t stream) {
+  const long long rows = static_cast<long long>(p.B) * p.H * p.N;
+  const int grid = elementwise_grid(rows * d / 8, num_sms);
+  const uint4* o = static_cast<const uint4*>(p.o);
+  const uint4* dout = static_cast<const uint4*>(p.dout);
+  float4* acc = reinterpret_cast<float4*>(p.dq_acc);
+  if (d == 128) {
+    if (bf16) fa_bwd_pre<128, true><<<grid, 256, 0, stream>>>(o, dout, p.dsum, acc, rows);
+    else fa_bwd_pre<128, false><<<grid, 256, 0, stream>>>(o, dout, p.dsum, acc, rows);
+  } else {
+    if (bf16) fa_bwd_pre<64, true><<<grid, 256, 0, stream>>>(o, dout, p.dsum, acc, rows);
+    else fa_bwd_pre<64, false><<<grid, 256, 0, stream>>>(o, dout, p.dsum, acc, rows);
+  }
+  return cudaGetLastError();
+}
+
+template <int D, bool BF16>
+static cudaError_t launch_bwd_main_t(const CUtensorMap& tmq, const CUtensorMap& tmk,
+                                     const CUtensorMap& tmv, const CUtensorMap& tmdo,
+                                     const BwdParams& p, int num_sms, cudaStream_t stream) {
+  using Lay = BwdLayout<D>;
+  auto kern = fa_bwd_kernel<D, BF16>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int grid = p.n_units < num_sms ? p.n_units : num_sms;
+  kern<<<grid, 384, Lay::kSmemBytes, stream>>>(tmq, tmk, tmv, tmdo, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_main(int d, bool bf16, const CUtensorMap& tmq, const CUtensorMap& tmk,
+                            const CUtensorMap& tmv, const CUtensorMap& tmdo, const BwdParams& p,
+                            int num_sms, cudaStream_t stream) {
+  if (d == 128) {
+    return bf16 ? launch_bwd_main_t<128, true>(tmq, tmk, tmv, tmdo, p, num_sms, stream)
+                : launch_bwd_main_t<128, false>(tmq, tmk, tmv, tmdo, p, num_sms, stream);
+  }
+  return bf16 ? launch_bwd_main_t<64, true>(tmq, tmk, tmv, tmdo, p, num_sms, stream)
+              : launch_bwd_main_t<64, false>(tmq, tmk, tmv, tmdo, p, num_sms, stream);
+}
+
+cudaError_t launch_bwd_post(int d, bool bf16, const BwdParams& p, int num_sms,
+                            cudaStream_t stream) {
+  const long long n8 = static_cast<long long>(p.B) * p.H * p.N * d / 8;
+  const int grid = elementwise_grid(n8, num_sms);
+  const float4* acc = reinterpret_cast<const float4*>(p.dq_acc);
+  uint4* dq = static_cast<uint4*>(p.dq);
+  if (bf16) fa_bwd_post<true><<<grid, 256, 0, stream>>>(acc, dq, p.scale, n8);
+  else fa_bwd_post<false><<<grid, 256, 0, stream>>>(acc, dq, p.scale, n8);
+  return cudaGetLastError();
 }
 
 }  // namespace fa

@@ -56,8 +56,12 @@ cudaError_t launch_fwd(int d, bool bf16, const CUtensorMap& tmq, const CUtensorM
                        const CUtensorMap& tmv, const FwdParams& p, int num_sms,
                        cudaStream_t stream);
 
-cudaError_t launch_bwd(int d, bool bf16, const CUtensorMap& tmq, const CUtensorMap& tmk,
-                       const CUtensorMap& tmv, const CUtensorMap& tmdo, const BwdParams& p,
-                       int num_sms, cudaStream_t stream);
+cudaError_t launch_bwd_pre(int d, bool bf16, const BwdParams& p, int num_sms,
+                           cudaStream_t stream);
+cudaError_t launch_bwd_main(int d, bool bf16, const CUtensorMap& tmq, const CUtensorMap& tmk,
+                            const CUtensorMap& tmv, const CUtensorMap& tmdo, const BwdParams& p,
+                            int num_sms, cudaStream_t stream);
+cudaError_t launch_bwd_post(int d, bool bf16, const BwdParams& p, int num_sms,
+                            cudaStream_t stream);
 
 }  // namespace fa

@@ -65,7 +65,8 @@ typedef enum {
   FA_ERR_CUDA = 5,            /* a CUDA runtime/driver call or launch failed    */
   FA_ERR_DEVICE_TIMEOUT = 6,  /* device: a pipeline wait gave up (fa_device_status) */
   FA_ERR_DEVICE_SEQLEN = 7,   /* device: seqlens[b] outside [1, N] (fa_device_status) */
-  FA_ERR_WORKSPACE = 8        /* backward workspace missing or too small        */
+  FA_ERR_WORKSPACE = 8,       /* backward workspace missing or too small        */
+  FA_ERR_DEVICE_LAYOUT = 9    /* device: shared-memory window misaligned, kernel refused (fa_device_status) */
 } fa_status;
 
 typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
@@ -106,8 +107,29 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* o,
            const int32_t* seqlens, int dtype, void* stream);
 
 /*
+ * The three stages fa_bwd runs, callable one by one (same arguments and
+ * checks; fa_bwd is exactly these three calls in this order on one stream).
+ *   fa_bwd_preprocess : workspace <- D_i = sum_c dO_ic O_ic (float32, from the
+ *                       16-bit O and dO) and a zeroed float32 dQ accumulator.
+ *   fa_bwd_main       : dk, dv written; float32 dQ accumulator reduce-added in
+ *                       the workspace (needs the preprocess result).
+ *   fa_bwd_postprocess: dq <- scale * accumulator, rounded to 16-bit.
+ */
+int fa_bwd_preprocess(const void* o, const void* dout, void* workspace,
+                      size_t workspace_bytes, int B, int H, int N, int d,
+                      int dtype, void* stream);
+int fa_bwd_main(const void* q, const void* k, const void* v, const void* dout,
+                const float* lse, void* dk, void* dv, void* workspace,
+                size_t workspace_bytes, int B, int H, int N, int d, float scale,
+                int causal, const int32_t* seqlens, int dtype, void* stream);
+int fa_bwd_postprocess(void* workspace, size_t workspace_bytes, void* dq,
+                       int B, int H, int N, int d, float scale, int dtype,
+                       void* stream);
+
+/*
  * Synchronises `stream`, then returns and clears the device status word of
- * the current device: FA_OK, FA_ERR_DEVICE_SEQLEN or FA_ERR_DEVICE_TIMEOUT
+ * the current device: FA_OK, FA_ERR_DEVICE_SEQLEN, FA_ERR_DEVICE_TIMEOUT or
+ * FA_ERR_DEVICE_LAYOUT
  * (FA_ERR_CUDA if the synchronisation itself failed).  *detail, if not NULL,
  * receives the raw word (code | site << 8 | block << 16).
  */

@@ -9,6 +9,11 @@ O_MAX_ABS = 2e-2
 O_MEAN_ABS = 2e-3
 LSE_MAX_ABS = 1e-3
 GRAD_REL_MAX = 5e-2   # max |d(grad)| <= GRAD_REL_MAX * max |ref grad|
+# Where the exact gradient vanishes (a row with one visible key: dS = P (dP - D)
+# = 0), fp32 evaluation of D_i = <dO_i, O_i> and of dP_i0 in different
+# summation orders leaves |dS| ~ 2^-23 sum |dO O| ~ 1e-6, so dQ ~ scale |K| 1e-6.
+# The relative bound then gets this absolute floor (GRAD_REL_MAX * 1e-4 = 5e-6).
+GRAD_ABS_FLOOR = 1e-4
 
 
 def f64(t):
@@ -43,5 +48,6 @@ def assert_grad_close(g_gpu, g_ref, what=""):
     assert np.isfinite(g_gpu).all(), f"{what}: non-finite gradient"
     err = np.abs(g_gpu - g_ref).max()
     scale = np.abs(g_ref).max()
-    assert err <= GRAD_REL_MAX * max(scale, 1e-6), f"{what}: max|d| {err:.3e} vs max|ref| {scale:.3e}"
+    assert err <= GRAD_REL_MAX * max(scale, GRAD_ABS_FLOOR), \
+        f"{what}: max|d| {err:.3e} vs max|ref| {scale:.3e}"
     return err / max(scale, 1e-30)
