@@ -288,3 +288,15 @@ extern "C" const char* fa_status_string(int status) {
 }
 
 extern "C" int fa_version(void) { return 100; }
+
+#ifdef FA_TRACE
+// Trace builds only: copy the device timeline (see FA_TRACE_AT) to the host.
+extern "C" int fa_trace_read(unsigned long long* host, int n) {
+  if (n > kTraceSlots) n = kTraceSlots;
+  if (cudaDeviceSynchronize() != cudaSuccess) return FA_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(host, g_trace, n * sizeof(unsigned long long)) != cudaSuccess)
+    return FA_ERR_CUDA;
+  static unsigned long long zeros[kTraceSlots];
+  return cudaMemcpyToSymbol(g_trace, zeros, sizeof(zeros)) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+#endif

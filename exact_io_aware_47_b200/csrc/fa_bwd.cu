@@ -218,6 +218,7 @@ __global__ void __launch_bounds__(384, 1)
         const int st = seq & 1;
         ok = mbar_wait_warp(&ld_empty[st], ((seq >> 1) & 1) ^ 1, abort_flag, 22);
         if (!ok) break;
+        if (lane == 0) FA_TRACE_AT(seq, 8);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int ql = lane * 4 + e;
@@ -227,6 +228,7 @@ __global__ void __launch_bounds__(384, 1)
           sDSUM[st * 128 + ql] = q < p.N ? p.dsum[base + q] : 0.f;
         }
         mbar_arrive(&ld_full[st]);
+        if (lane == 0) FA_TRACE_AT(seq, 9);
         ++seq;
       }
     }
@@ -255,11 +257,17 @@ __global__ void __launch_bounds__(384, 1)
         ok = mbar_wait(kv_full, nunit & 1, abort_flag, 23);
         if (!ok) break;
         tc_fence_after();
+        // The epilogue of the previous unit must have read dV/dK before this
+        // unit writes them, and before dkv_full is committed again (so that
+        // barrier never runs two phases ahead of its waiter, also for units
+        // with no query tiles).
+        bool dkv_free = nunit == 0;
         for (int idx = 0; idx < w.ni && ok; ++idx) {
           const int st = qseq & 1;
           ok = mbar_wait(&q_full[st], (qseq >> 1) & 1, abort_flag, 24);
           if (!ok) break;
           tc_fence_after();
+          FA_TRACE_AT(it, 0);
           const uint32_t q_s = aQ + st * Lay::kTileBytes;
           const uint32_t do_s = aDO + st * Lay::kTileBytes;
           // S^T = K_j Q_i^T
@@ -272,6 +280,7 @@ __global__ void __launch_bounds__(384, 1)
             if (!ok) break;
             tc_fence_after();
           }
+          FA_TRACE_AT(it, 1);
           // dP^T = V_j dO_i^T
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
@@ -280,10 +289,12 @@ __global__ void __launch_bounds__(384, 1)
           ok = mbar_wait(p_full, it & 1, abort_flag, 26);
           if (!ok) break;
           tc_fence_after();
-          if (idx == 0 && nunit > 0) {
+          FA_TRACE_AT(it, 2);
+          if (!dkv_free) {
             ok = mbar_wait(dkv_empty, (nunit - 1) & 1, abort_flag, 27);
             if (!ok) break;
             tc_fence_after();
+            dkv_free = true;
           }
           // dV_j += P^T dO_i   (A = P^T in TMEM, 16 queries = 8 columns)
 #pragma unroll
@@ -300,12 +311,17 @@ __global__ void __launch_bounds__(384, 1)
           for (int kk = 0; kk < 8; ++kk)
             umma_ss(tmem + Lay::kColDQ, mnmaj(aDS, kk), mnmaj(aK, kk), kIdDQ, kk > 0);
           umma_commit(dq_full);
+          FA_TRACE_AT(it, 3);
           umma_commit(&q_empty[st]);
           umma_commit(ds_empty);
           ++qseq;
           ++it;
         }
         if (!ok) break;
+        if (!dkv_free) {
+          ok = mbar_wait(dkv_empty, (nunit - 1) & 1, abort_flag, 34);
+          if (!ok) break;
+        }
         umma_commit(dkv_full);
         umma_commit(kv_empty);
         ++nunit;
@@ -336,6 +352,7 @@ __global__ void __launch_bounds__(384, 1)
         if (ok && it > 0) ok = mbar_wait_warp(ds_empty, (it - 1) & 1, abort_flag, 31);
         if (!ok) break;
         tc_fence_after();
+        if (threadIdx.x == 0) FA_TRACE_AT(it, 4);
         const bool diag = p.causal && i == w.j;
         const float* lse2 = sLSE + st * 128;
         const float* dsm = sDSUM + st * 128;
@@ -373,6 +390,7 @@ __global__ void __launch_bounds__(384, 1)
         tc_fence_before();
         mbar_arrive(p_full);
         mbar_arrive(&ld_empty[st]);
+        if (threadIdx.x == 0) FA_TRACE_AT(it, 5);
         ++it;
       }
     }
@@ -390,6 +408,7 @@ __global__ void __launch_bounds__(384, 1)
         ok = mbar_wait_warp(dq_full, it & 1, abort_flag, 32);
         if (!ok) break;
         tc_fence_after();
+        if (threadIdx.x == 128) FA_TRACE_AT(it, 6);
         const int row = i * kBlockM + r;
         float* dst = p.dq_acc + (base + (row < p.N ? row : 0)) * D;
 #pragma unroll
@@ -406,6 +425,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         tc_fence_before();
         mbar_arrive(dq_empty);
+        if (threadIdx.x == 128) FA_TRACE_AT(it, 7);
         ++it;
       }
       if (!ok) break;

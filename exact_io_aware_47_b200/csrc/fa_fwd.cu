@@ -259,6 +259,7 @@ __global__ void __launch_bounds__(384, 1)
             if (j < je[t]) {
               ok = mbar_wait(&p_full[t], pcnt[t] & 1, abort_flag, 6);
               if (!ok) break;
+              FA_TRACE_AT(pcnt[t], t);
               ++pcnt[t];
               tc_fence_after();
               issue_pv(t, vslot, j > 0);
@@ -314,6 +315,7 @@ __global__ void __launch_bounds__(384, 1)
       for (int j = 0; j < jend; ++j) {
         ok = mbar_wait_warp(&s_full[t], scnt & 1, abort_flag, 8);
         if (!ok) break;
+        if (r == 0) FA_TRACE_AT(scnt, 2 + 2 * t);
         ++scnt;
         tc_fence_after();
         float x[128];
@@ -374,6 +376,7 @@ __global__ void __launch_bounds__(384, 1)
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&p_full[t]);
+        if (r == 0) FA_TRACE_AT(scnt - 1, 3 + 2 * t);
       }
       if (!ok) break;
       // epilogue: O / l -> 16-bit, LSE

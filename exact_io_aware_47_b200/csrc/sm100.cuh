@@ -26,6 +26,23 @@ __device__ __forceinline__ void record_error(unsigned code, unsigned site) {
   atomicCAS(&g_error_word, 0u, w);
 }
 
+// Optional device timeline (build with -DFA_TRACE): SM clock stamps of
+// pipeline events of CTA 0, slot = iteration * 16 + event.  Compiled out by
+// default.
+#ifdef FA_TRACE
+constexpr int kTraceSlots = 1 << 16;
+__device__ unsigned long long g_trace[kTraceSlots];
+#define FA_TRACE_AT(it, ev)                                                        \
+  do {                                                                            \
+    if (blockIdx.x == 0 && (it) < (kTraceSlots / 16))                             \
+      g_trace[(it) * 16 + (ev)] = static_cast<unsigned long long>(clock64());     \
+  } while (0)
+#else
+#define FA_TRACE_AT(it, ev) \
+  do {                      \
+  } while (0)
+#endif
+
 // A wait gives up after this long and reports kErrDeviceTimeout.  No wait in
 // a correct pipeline lasts more than microseconds.
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s
