@@ -91,6 +91,22 @@ int make_map(CUtensorMap* map, const void* ptr, int BH, int N, int d, int dtype)
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
+// [B*H, N, d] fp32 view of the dQ accumulator for TMA reduce-adds of 64 rows
+// x d columns, no swizzle; rows past N inside a head are skipped.
+int make_map_acc(CUtensorMap* map, void* ptr, int BH, int N, int d) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4,
+                                 static_cast<cuuint64_t>(N) * d * 4};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(d), 64, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 }  // namespace
@@ -201,10 +217,11 @@ extern "C" int fa_bwd_main(const void* q, const void* k, const void* v, const vo
   DeviceInfo di;
   int st = bwd_common(workspace, workspace_bytes, B, H, N, d, scale, dtype, seqlens, &p, &di);
   if (st != FA_OK) return st;
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tdq;
   const int BH = B * H;
   if (make_map(&tq, q, BH, N, d, dtype) != FA_OK || make_map(&tk, k, BH, N, d, dtype) != FA_OK ||
-      make_map(&tv, v, BH, N, d, dtype) != FA_OK || make_map(&tdo, dout, BH, N, d, dtype) != FA_OK)
+      make_map(&tv, v, BH, N, d, dtype) != FA_OK || make_map(&tdo, dout, BH, N, d, dtype) != FA_OK ||
+      make_map_acc(&tdq, p.dq_acc, BH, N, d) != FA_OK)
     return FA_ERR_CUDA;
   p.q = q;
   p.k = k;
@@ -214,7 +231,7 @@ extern "C" int fa_bwd_main(const void* q, const void* k, const void* v, const vo
   p.dk = dk;
   p.dv = dv;
   p.causal = causal ? 1 : 0;
-  const cudaError_t e = launch_bwd_main(d, dtype == FA_BF16, tq, tk, tv, tdo, p, di.num_sms,
+  const cudaError_t e = launch_bwd_main(d, dtype == FA_BF16, tq, tk, tv, tdo, tdq, p, di.num_sms,
                                         static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }

@@ -12,24 +12,27 @@
 // Three kernels:
 //  1. fa_bwd_pre: D_i = sum_c dO_ic O_ic (fp32) and zero the fp32 dQ
 //     accumulator;
-//  2. fa_bwd_kernel (persistent, one CTA per SM, 384 threads): a work unit is
+//  2. fa_bwd_kernel (persistent, one CTA per SM, 512 threads): a work unit is
 //     (batch*head, 128-key tile j).  K_j and V_j stay in shared memory while
 //     the query tiles i (i >= j when causal) stream past:
 //       S^T  = K_j Q_i^T      (tcgen05, TMEM, keys on lanes)
 //       dP^T = V_j dO_i^T     (tcgen05, TMEM)
 //       P^T  = exp2(c S^T - LSE_i log2 e), dS^T = P^T * (dP^T - D_i)
-//                              (warps 0-3, one key row per thread; P^T goes
-//                              back to TMEM over S^T as 16-bit, dS^T to a
-//                              swizzled shared-memory tile)
-//       dV_j += P^T dO_i,  dK_j += dS^T Q_i   (TMEM accumulators)
-//       dQ_i  = dS K_j     (TMEM; warps 4-7 reduce-add it into the fp32
+//                              (warps 0-7, one key row and half the queries
+//                              per thread; P^T goes back to TMEM over S^T as
+//                              16-bit, dS^T to a swizzled shared-memory tile)
+//       dQ_i  = dS K_j     (issued first; d = 128 computes dQ_i^T = K_j^T dS^T
+//                           so each warp's reduce-add is one contiguous row
+//                           segment; warps 8-11 add it into the fp32
 //                           accumulator in global memory)
-//     warp 8 issues the MMAs, warp 9 the TMA loads, warp 10 stages LSE_i and
-//     D_i in shared memory; warps 4-7 also write dK_j (times scale) and dV_j
-//     at the end of the unit;
+//       dV_j += P^T dO_i,  dK_j += dS^T Q_i   (TMEM accumulators)
+//     warp 12 issues the MMAs, warp 13 the TMA loads, warp 14 stages LSE_i
+//     and D_i in shared memory; warps 8-11 also write dK_j (times scale) and
+//     dV_j at the end of the unit;
 //  3. fa_bwd_post: dQ = scale * accumulator, rounded to 16-bit.
 //
-// TMEM columns: S^T/P^T [0,128), dP^T [128,256), dV [256,256+d),
+// TMEM columns: S^T [0,128) with P^T (16-bit) over [0,32) and [64,96),
+// dP^T [128,256), dV [256,256+d),
 // dK [256+d,256+2d); dQ_i reuses the dP^T columns when d = 128 (the 512
 // columns are all taken) and [384,448) when d = 64.
 #include <algorithm>
@@ -88,10 +91,10 @@ __device__ __forceinline__ BwdUnit bwd_decode(int u, const BwdParams& p) {
 }
 
 template <int D, bool BF16>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(512, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdo,
-                  const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tmdq, const BwdParams p) {
   using Lay = BwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -137,11 +140,11 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
       mbar_init(&ld_full[s], 32);
-      mbar_init(&ld_empty[s], 128);
+      mbar_init(&ld_empty[s], 256);
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
-    mbar_init(p_full, 128);
+    mbar_init(p_full, 256);
     mbar_init(ds_empty, 1);
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, 128);
@@ -151,7 +154,7 @@ __global__ void __launch_bounds__(384, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 8) {
+  if (warp == 12) {
     tmem_alloc(tmem_slot, Lay::kTmemCols);
     tmem_relinquish();
   }
@@ -160,7 +163,7 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 9) {
+  if (warp == 13) {
     // ------------------------------------------------------------- TMA loads
     if (lane == 0) {
       tma_prefetch_desc(&tmq);
@@ -205,7 +208,7 @@ __global__ void __launch_bounds__(384, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 10) {
+  } else if (warp == 14) {
     // ------------------------------------------------ LSE_i, D_i -> shared memory
     int seq = 0;
     bool ok = true;
@@ -232,12 +235,16 @@ __global__ void __launch_bounds__(384, 1)
         ++seq;
       }
     }
-  } else if (warp == 8) {
+  } else if (warp == 12) {
     // ------------------------------------------------------------- MMA issue
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_f16(BF16, 128, 128, false, false);  // S^T, dP^T
       constexpr uint32_t kIdTS = idesc_f16(BF16, 128, D, false, true);    // dV, dK (B MN-major)
-      constexpr uint32_t kIdDQ = idesc_f16(BF16, 128, D, true, true);     // dQ (A, B MN-major)
+      // dQ: d = 128 computes dQ^T = K^T dS^T (M = d, N = queries), so the
+      // reduce-adds of a warp cover one contiguous row segment; d = 64 keeps
+      // dQ = dS K (M = queries, N = d).
+      constexpr uint32_t kIdDQ =
+          D == 128 ? idesc_f16(BF16, 128, 128, true, true) : idesc_f16(BF16, 128, D, true, true);
       const uint32_t aK = smem_addr(sK), aV = smem_addr(sV), aQ = smem_addr(sQ),
                      aDO = smem_addr(sDO), aDS = smem_addr(sDS);
       int nunit = 0, qseq = 0, it = 0;
@@ -275,7 +282,8 @@ __global__ void __launch_bounds__(384, 1)
           for (int kk = 0; kk < D / 16; ++kk)
             umma_ss(tmem + Lay::kColS, kmaj(aK, kk), kmaj(q_s, kk), kIdS, kk > 0);
           umma_commit(s_full);
-          if (it > 0) {
+          // d = 128: dQ^T of the previous tile lives in the dP^T columns
+          if (D == 128 && it > 0) {
             ok = mbar_wait(dq_empty, (it - 1) & 1, abort_flag, 25);
             if (!ok) break;
             tc_fence_after();
@@ -290,30 +298,51 @@ __global__ void __launch_bounds__(384, 1)
           if (!ok) break;
           tc_fence_after();
           FA_TRACE_AT(it, 2);
+          if (D == 64 && it > 0) {
+            ok = mbar_wait(dq_empty, (it - 1) & 1, abort_flag, 25);
+            if (!ok) break;
+            tc_fence_after();
+          }
+          // dQ first, so its read-out overlaps the dV and dK MMAs
+          if constexpr (D == 128) {
+            // dQ^T = K_j^T dS^T: A = K_j read MN-major (d contiguous), B = dS^T
+            // read MN-major (queries contiguous)
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              umma_ss(tmem + Lay::kColDQ, mnmaj(aK, kk), mnmaj(aDS, kk), kIdDQ, kk > 0);
+          } else {
+            // dQ = dS K_j: A = dS^T read MN-major, B = K_j MN-major
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              umma_ss(tmem + Lay::kColDQ, mnmaj(aDS, kk), mnmaj(aK, kk), kIdDQ, kk > 0);
+          }
+          if (D == 64) umma_commit(dq_full);
+          FA_TRACE_AT(it, 3);
           if (!dkv_free) {
             ok = mbar_wait(dkv_empty, (nunit - 1) & 1, abort_flag, 27);
             if (!ok) break;
             tc_fence_after();
             dkv_free = true;
           }
-          // dV_j += P^T dO_i   (A = P^T in TMEM, 16 queries = 8 columns)
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            umma_ts(tmem + Lay::kColDV, tmem + Lay::kColS + kk * 8, mnmaj(do_s, kk), kIdTS,
-                    (idx > 0 || kk > 0) ? 1u : 0u);
           // dK_j += dS^T Q_i   (A = dS^T in shared memory, K-major)
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             umma_ss(tmem + Lay::kColDK, kmaj(aDS, kk), mnmaj(q_s, kk), kIdTS,
                     (idx > 0 || kk > 0) ? 1u : 0u);
-          // dQ_i = dS K_j      (A = the same dS^T tile read MN-major)
+          if constexpr (D == 128) {
+            // dQ^T and dK done = the dS^T tile has no MMA reader left: the dQ
+            // warps may stage dQ^T in it
+            umma_commit(dq_full);
+          } else {
+            umma_commit(ds_empty);
+          }
+          // dV_j += P^T dO_i   (A = P^T in TMEM, 16 queries = 8 columns; queries
+          // 64..127 sit 64 columns further, in the second half's S^T columns)
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            umma_ss(tmem + Lay::kColDQ, mnmaj(aDS, kk), mnmaj(aK, kk), kIdDQ, kk > 0);
-          umma_commit(dq_full);
-          FA_TRACE_AT(it, 3);
+            umma_ts(tmem + Lay::kColDV, tmem + Lay::kColS + (kk >> 2) * 64 + (kk & 3) * 8,
+                    mnmaj(do_s, kk), kIdTS, (idx > 0 || kk > 0) ? 1u : 0u);
           umma_commit(&q_empty[st]);
-          umma_commit(ds_empty);
           ++qseq;
           ++it;
         }
@@ -330,13 +359,15 @@ __global__ void __launch_bounds__(384, 1)
       mbar_wait_drain(drain, 0, 200000000ull);
     }
     __syncwarp();
-  } else if (warp < 4) {
-    // ----------------------------------------------- P^T and dS^T (key rows)
-    const int r = (warp << 5) | lane;  // key row in the tile = TMEM lane
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+  } else if (warp < 8) {
+    // ------------------------- P^T and dS^T: key row per thread, half the queries
+    const int half = warp >> 2;              // queries [64 half, 64 half + 64)
+    const int r = ((warp & 3) << 5) | lane;  // key row in the tile = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_off + Lay::kColS;
     const uint32_t tDP = tmem + lane_off + Lay::kColDP;
-    const uint32_t ds_row = smem_addr(sDS) + r * 128;
+    // dS^T row r, queries of this half: panel `half` of the swizzled tile
+    const uint32_t ds_row = smem_addr(sDS) + half * 16384 + r * 128;
     const float cl = p.scale_log2;
     int it = 0;
     bool ok = true;
@@ -353,35 +384,47 @@ __global__ void __launch_bounds__(384, 1)
         if (!ok) break;
         tc_fence_after();
         if (threadIdx.x == 0) FA_TRACE_AT(it, 4);
-        const bool diag = p.causal && i == w.j;
+        // a query tile on the causal diagonal hides keys above the query
+        const int diag_lim = (p.causal && i == w.j) ? r : -1;  // visible iff q_local >= r
         const float* lse2 = sLSE + st * 128;
         const float* dsm = sDSUM + st * 128;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = half * 2 + cc;  // 32-query chunk
           uint32_t sr[32], dr[32];
           tmem_ld32(tS + c * 32, sr);
           tmem_ld32(tDP + c * 32, dr);
           uint32_t pp[16], dd[16];
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
+          for (int e = 0; e < 32; e += 4) {
             const int q0 = c * 32 + e;
-            const bool v0 = key_ok && (!diag || r <= q0);
-            const bool v1 = key_ok && (!diag || r <= q0 + 1);
-            const float p0 = v0 ? ex2_approx(__uint_as_float(sr[e]) * cl - lse2[q0]) : 0.f;
-            const float p1 = v1 ? ex2_approx(__uint_as_float(sr[e + 1]) * cl - lse2[q0 + 1]) : 0.f;
-            const float g0 = p0 * (__uint_as_float(dr[e]) - dsm[q0]);
-            const float g1 = p1 * (__uint_as_float(dr[e + 1]) - dsm[q0 + 1]);
-            pp[e >> 1] = pack2<BF16>(p0, p1);
-            dd[e >> 1] = pack2<BF16>(g0, g1);
+            const float4 l4 = *reinterpret_cast<const float4*>(lse2 + q0);
+            const float4 d4 = *reinterpret_cast<const float4*>(dsm + q0);
+            const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+            const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+            float pv[4], gv[4];
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) {
+              const bool vis = key_ok && (q0 + k4 >= diag_lim);
+              const float x = fmaf(__uint_as_float(sr[e + k4]), cl, -lv[k4]);
+              pv[k4] = vis ? ex2_approx(x) : 0.f;
+              gv[k4] = pv[k4] * (__uint_as_float(dr[e + k4]) - dv4[k4]);
+            }
+            pp[(e >> 1)] = pack2<BF16>(pv[0], pv[1]);
+            pp[(e >> 1) + 1] = pack2<BF16>(pv[2], pv[3]);
+            dd[(e >> 1)] = pack2<BF16>(gv[0], gv[1]);
+            dd[(e >> 1) + 1] = pack2<BF16>(gv[2], gv[3]);
           }
-          tmem_st16(tS + c * 16, pp);  // P^T over the already-read S^T columns
-          // dS^T row r, queries [32c, 32c+32): four 16-byte units of a 128-byte
-          // swizzled row in panel c/2
-          const uint32_t prow = ds_row + (c >> 1) * 16384;
+          // P^T of queries [32c, 32c+32) goes to columns 64 half + 16 (c & 1): only
+          // over S^T columns this thread has already read, never the other
+          // half's
+          tmem_st16(tS + half * 64 + (c & 1) * 16, pp);
+          // four 16-byte units of the 128-byte swizzled row (chunk c = units
+          // 4 (c & 1) .. 4 (c & 1) + 3 of panel `half`)
 #pragma unroll
           for (int w4 = 0; w4 < 4; ++w4) {
             const uint32_t unit = ((c & 1) * 4 + w4) ^ (r & 7);
-            st_shared_v4(prow + unit * 16, dd[4 * w4], dd[4 * w4 + 1], dd[4 * w4 + 2],
+            st_shared_v4(ds_row + unit * 16, dd[4 * w4], dd[4 * w4 + 1], dd[4 * w4 + 2],
                          dd[4 * w4 + 3]);
           }
         }
@@ -394,9 +437,9 @@ __global__ void __launch_bounds__(384, 1)
         ++it;
       }
     }
-  } else if (warp < 8) {
-    // ------------------------------- dQ_i reduce-add; dK_j, dV_j at unit end
-    const int r = ((warp & 3) << 5) | lane;
+  } else if (warp < 12) {
+    // --------------------------- dQ read-out and reduce-add; dK_j, dV_j epilogue
+    const int r = ((warp & 3) << 5) | lane;  // TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     int it = 0, nunit = 0;
     bool ok = true;
@@ -408,24 +451,58 @@ __global__ void __launch_bounds__(384, 1)
         ok = mbar_wait_warp(dq_full, it & 1, abort_flag, 32);
         if (!ok) break;
         tc_fence_after();
-        if (threadIdx.x == 128) FA_TRACE_AT(it, 6);
-        const int row = i * kBlockM + r;
-        float* dst = p.dq_acc + (base + (row < p.N ? row : 0)) * D;
+        if (threadIdx.x == 256) FA_TRACE_AT(it, 6);
+        if constexpr (D == 128) {
+          // Lane r holds column r of dQ_i for the 128 query rows (dQ^T).  Two
+          // rounds of 64 rows: TMEM -> the dS^T tile reused as a [64][128]
+          // fp32 staging buffer -> one TMA reduce-add into the accumulator.
+          float* stg = reinterpret_cast<float*>(sDS);
+          const bool leader = warp == 8 && lane == 0;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tmem + lane_off + Lay::kColDQ + c * 32, v);
-          if (row < p.N) {
+          for (int half = 0; half < 2; ++half) {
+            uint32_t v[64];
+            tmem_ld64(tmem + lane_off + Lay::kColDQ + half * 64, v);
+            if (half == 1) {
+              // all of dQ^T is in registers: the MMA may overwrite its columns
+              tc_fence_before();
+              mbar_arrive(dq_empty);
+              if (leader) bulk_wait_read_all();  // round 0 has left the buffer
+              named_bar_sync(1, 128);
+            }
 #pragma unroll
-            for (int q4 = 0; q4 < 8; ++q4)
-              red_add_v4(dst + c * 32 + q4 * 4, __uint_as_float(v[4 * q4]),
-                         __uint_as_float(v[4 * q4 + 1]), __uint_as_float(v[4 * q4 + 2]),
-                         __uint_as_float(v[4 * q4 + 3]));
+            for (int e = 0; e < 64; ++e) stg[e * D + r] = __uint_as_float(v[e]);
+            fence_proxy_async_smem();
+            named_bar_sync(1, 128);
+            if (leader) {
+              tma_reduce_add_3d(&tmdq, stg, 0, i * kBlockM + half * 64, w.bh);
+              bulk_commit_group();
+            }
+          }
+          if (leader) {
+            bulk_wait_read_all();
+            mbar_arrive(ds_empty);  // the softmax warps may write dS^T again
+          }
+        } else {
+          const int row = i * kBlockM + r;
+          float* dst = p.dq_acc + (base + (row < p.N ? row : 0)) * D;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tmem + lane_off + Lay::kColDQ + c * 32, v);
+            if (row < p.N) {
+#pragma unroll
+              for (int q4 = 0; q4 < 8; ++q4)
+                red_add_v4(dst + c * 32 + q4 * 4, __uint_as_float(v[4 * q4]),
+                           __uint_as_float(v[4 * q4 + 1]), __uint_as_float(v[4 * q4 + 2]),
+                           __uint_as_float(v[4 * q4 + 3]));
+            }
           }
         }
-        tc_fence_before();
-        mbar_arrive(dq_empty);
-        if (threadIdx.x == 128) FA_TRACE_AT(it, 7);
+        if (D == 64) {
+          tc_fence_before();
+          mbar_arrive(dq_empty);
+        }
+        if (threadIdx.x == 256) FA_TRACE_AT(it, 7);
         ++it;
       }
       if (!ok) break;
@@ -471,12 +548,14 @@ __global__ void __launch_bounds__(384, 1)
       mbar_arrive(dkv_empty);
       ++nunit;
     }
+    // every reduce-add issued must have completed before the kernel ends
+    if (D == 128 && warp == 8 && lane == 0) bulk_wait_all();
   }
-  // warp 11 has no role
+  // warp 15 has no role
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == 12) {
     tc_fence_after();
     tmem_dealloc(tmem, Lay::kTmemCols);
   }
@@ -568,26 +647,28 @@ cudaError_t launch_bwd_pre(int d, bool bf16, const BwdParams& p, int num_sms,
 template <int D, bool BF16>
 static cudaError_t launch_bwd_main_t(const CUtensorMap& tmq, const CUtensorMap& tmk,
                                      const CUtensorMap& tmv, const CUtensorMap& tmdo,
-                                     const BwdParams& p, int num_sms, cudaStream_t stream) {
+                                     const CUtensorMap& tmdq, const BwdParams& p, int num_sms,
+                                     cudaStream_t stream) {
   using Lay = BwdLayout<D>;
   auto kern = fa_bwd_kernel<D, BF16>;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kSmemBytes);
   if (e != cudaSuccess) return e;
   const int grid = p.n_units < num_sms ? p.n_units : num_sms;
-  kern<<<grid, 384, Lay::kSmemBytes, stream>>>(tmq, tmk, tmv, tmdo, p);
+  kern<<<grid, 512, Lay::kSmemBytes, stream>>>(tmq, tmk, tmv, tmdo, tmdq, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_bwd_main(int d, bool bf16, const CUtensorMap& tmq, const CUtensorMap& tmk,
-                            const CUtensorMap& tmv, const CUtensorMap& tmdo, const BwdParams& p,
-                            int num_sms, cudaStream_t stream) {
+                            const CUtensorMap& tmv, const CUtensorMap& tmdo,
+                            const CUtensorMap& tmdq, const BwdParams& p, int num_sms,
+                            cudaStream_t stream) {
   if (d == 128) {
-    return bf16 ? launch_bwd_main_t<128, true>(tmq, tmk, tmv, tmdo, p, num_sms, stream)
-                : launch_bwd_main_t<128, false>(tmq, tmk, tmv, tmdo, p, num_sms, stream);
+    return bf16 ? launch_bwd_main_t<128, true>(tmq, tmk, tmv, tmdo, tmdq, p, num_sms, stream)
+                : launch_bwd_main_t<128, false>(tmq, tmk, tmv, tmdo, tmdq, p, num_sms, stream);
   }
-  return bf16 ? launch_bwd_main_t<64, true>(tmq, tmk, tmv, tmdo, p, num_sms, stream)
-              : launch_bwd_main_t<64, false>(tmq, tmk, tmv, tmdo, p, num_sms, stream);
+  return bf16 ? launch_bwd_main_t<64, true>(tmq, tmk, tmv, tmdo, tmdq, p, num_sms, stream)
+              : launch_bwd_main_t<64, false>(tmq, tmk, tmv, tmdo, tmdq, p, num_sms, stream);
 }
 
 cudaError_t launch_bwd_post(int d, bool bf16, const BwdParams& p, int num_sms,

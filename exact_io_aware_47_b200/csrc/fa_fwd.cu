@@ -48,6 +48,14 @@ struct FwdLayout {
   static constexpr uint32_t kColO = 256;
 };
 
+// Register split: 384 threads launched at 168 registers (launch bounds 384,1);
+// the two softmax warpgroups take 184, the MMA/TMA warpgroup keeps 136:
+// 2 * 184 + 136 = 3 * 168 (no spills at this split).
+constexpr int kFwdLaunchRegs = 168;
+constexpr int kFwdSoftmaxRegs = 184;
+constexpr int kFwdOtherRegs = 136;
+static_assert(2 * kFwdSoftmaxRegs + kFwdOtherRegs <= 3 * kFwdLaunchRegs, "register split");
+
 struct FwdUnit {
   int bh, qt0, L, jend0, jend1;
 };
@@ -131,6 +139,8 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  if (warp >= 8) {
+  regs_decrease<kFwdOtherRegs>();
   if (warp == 9) {
     // ------------------------------------------------------------- TMA loads
     if (lane == 0) {
@@ -290,7 +300,10 @@ __global__ void __launch_bounds__(384, 1)
       mbar_wait_drain(drain, 0, 200000000ull);
     }
     __syncwarp();
-  } else if (warp < 8) {
+  }
+  // warps 10 and 11 have no role
+  } else {
+    regs_increase<kFwdSoftmaxRegs>();
     // ------------------------------------------------------------- softmax
     const int t = warp >> 2;                 // query tile of the pair
     const int r = ((warp & 3) << 5) | lane;  // row inside the tile = TMEM lane
@@ -318,34 +331,57 @@ __global__ void __launch_bounds__(384, 1)
         if (r == 0) FA_TRACE_AT(scnt, 2 + 2 * t);
         ++scnt;
         tc_fence_after();
-        float x[128];
-        {
-          uint32_t rr[32];
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            tmem_ld32(tS + cc * 32, rr);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) x[cc * 32 + i] = __uint_as_float(rr[i]) * c;
-          }
-        }
+        uint32_t sr[128];  // raw scores q.k of this row, one TMEM load
+        tmem_ld128(tS, sr);
         const int kbase = j * kBlockN;
         const bool need_mask = (p.causal && j == qt) || (kbase + kBlockN > w.L);
         if (need_mask) {
           const int lim = p.causal ? min(w.L, row + 1) : w.L;  // keys < lim are visible
 #pragma unroll
           for (int i = 0; i < 128; ++i)
-            if (kbase + i >= lim) x[i] = -INFINITY;
+            if (kbase + i >= lim) sr[i] = __float_as_uint(-INFINITY);
         }
-        float mx = x[0];
+        // row max of the raw scores: four independent 3-input max chains,
+        // chain q4 takes elements 8k + 2 q4 and 8k + 2 q4 + 1
+        float mc[4];
 #pragma unroll
-        for (int i = 1; i < 128; ++i) mx = fmaxf(mx, x[i]);
+        for (int q4 = 0; q4 < 4; ++q4)
+          mc[q4] = fmaxf(__uint_as_float(sr[2 * q4]), __uint_as_float(sr[2 * q4 + 1]));
+#pragma unroll
+        for (int i = 8; i < 128; i += 8) {
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            mc[q4] = fmax3(mc[q4], __uint_as_float(sr[i + 2 * q4]), __uint_as_float(sr[i + 2 * q4 + 1]));
+        }
+        const float mx = fmax3(mc[0], mc[1], fmaxf(mc[2], mc[3])) * c;  // log2 units (c > 0)
         const float m_new = (mx > m + kRescaleThreshold) ? mx : m;
         const bool moved = m_new != m;
         const float alpha = moved ? ex2_approx(m - m_new) : 1.f;  // 0 when m was -inf
         l *= alpha;
+        m = m_new;
+        // p = 2^(c s - m): packed FMA on pairs, then ex2; row sum in fp32 over
+        // four independent accumulators
+        const float mu = (m == -INFINITY) ? 0.f : m;
+        const unsigned long long c2 = f2pack(c, c);
+        const unsigned long long nm2 = f2pack(-mu, -mu);
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t pk[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          float x0, x1;
+          f2unpack(ffma2(f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), c2, nm2),
+                   x0, x1);
+          const float p0 = ex2_approx(x0);
+          const float p1 = ex2_approx(x1);
+          acc[i & 3] += p0 + p1;
+          pk[i] = pack2<BF16>(p0, p1);
+        }
+        l += (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        tmem_st64(tS, pk);
         if (j > 0 && __any_sync(0xffffffffu, moved)) {
           // O_t holds the sum up to tile j-1 (its MMA completed before S_t(j)
-          // was committed); rows that did not move multiply by 1.
+          // was committed) and PV_t(j) waits for p_full: rescale it now; rows
+          // that did not move multiply by 1.
           uint32_t ro[32];
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc) {
@@ -354,24 +390,6 @@ __global__ void __launch_bounds__(384, 1)
             for (int i = 0; i < 32; ++i) ro[i] = __float_as_uint(__uint_as_float(ro[i]) * alpha);
             tmem_st32(tO + cc * 32, ro);
           }
-        }
-        m = m_new;
-        const float mu = (m == -INFINITY) ? 0.f : m;
-        float sum = 0.f;
-        uint32_t pk[64];
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float p0 = ex2_approx(x[2 * i] - mu);
-          const float p1 = ex2_approx(x[2 * i + 1] - mu);
-          sum += p0 + p1;
-          pk[i] = pack2<BF16>(p0, p1);
-        }
-        l += sum;
-        {
-          uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
-          uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
-          tmem_st32(tS, lo);
-          tmem_st32(tS + 32, hi);
         }
         tmem_st_wait();
         tc_fence_before();
@@ -406,7 +424,6 @@ __global__ void __launch_bounds__(384, 1)
       if (store) p.lse[static_cast<size_t>(w.bh) * p.N + row] = (m + log2f(l)) * 0.69314718055994531f;
     }
   }
-  // warps 10 and 11 have no role
 
   tc_fence_before();
   __syncthreads();
@@ -422,8 +439,12 @@ static cudaError_t launch_fwd_t(const CUtensorMap& tmq, const CUtensorMap& tmk,
                                 cudaStream_t stream) {
   using Lay = FwdLayout<D>;
   auto kern = fa_fwd_kernel<D, BF16>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       Lay::kSmemBytes);
+  cudaFuncAttributes attr;
+  cudaError_t e = cudaFuncGetAttributes(&attr, kern);
+  if (e != cudaSuccess) return e;
+  // the register split in the kernel assumes exactly this launch allocation
+  if (attr.numRegs != kFwdLaunchRegs) return cudaErrorInvalidConfiguration;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kSmemBytes);
   if (e != cudaSuccess) return e;
   const int grid = p.n_units < num_sms ? p.n_units : num_sms;
   kern<<<grid, 384, Lay::kSmemBytes, stream>>>(tmq, tmk, tmv, p);

@@ -59,8 +59,9 @@ cudaError_t launch_fwd(int d, bool bf16, const CUtensorMap& tmq, const CUtensorM
 cudaError_t launch_bwd_pre(int d, bool bf16, const BwdParams& p, int num_sms,
                            cudaStream_t stream);
 cudaError_t launch_bwd_main(int d, bool bf16, const CUtensorMap& tmq, const CUtensorMap& tmk,
-                            const CUtensorMap& tmv, const CUtensorMap& tmdo, const BwdParams& p,
-                            int num_sms, cudaStream_t stream);
+                            const CUtensorMap& tmv, const CUtensorMap& tmdo,
+                            const CUtensorMap& tmdq, const BwdParams& p, int num_sms,
+                            cudaStream_t stream);
 cudaError_t launch_bwd_post(int d, bool bf16, const BwdParams& p, int num_sms,
                             cudaStream_t stream);
 

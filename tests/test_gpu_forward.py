@@ -187,3 +187,52 @@ def test_host_side_rejections(fa):
     assert call(dtype=5) == _lib.FA_ERR_INVALID_ARG
     assert call() == _lib.FA_OK
     torch.cuda.synchronize()
+
+
+# --- closed forms on the GPU: cases where rounding cannot hide an error ------------
+
+def _bf16_ulp(x):
+    """Spacing of bf16 numbers at |x| (float64 array)."""
+    e = np.floor(np.log2(np.maximum(np.abs(x), 2.0 ** -126)))
+    return 2.0 ** (e - 7)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_single_visible_key_returns_its_value_exactly(fa, d, causal):
+    # one visible key: P = 1 exactly after the max is subtracted, so O = v_0
+    # with no rounding at all, and LSE = scale * q_i . k_0
+    from exact_io_aware_47_b200.inputs import make_inputs_shape
+    N = 300
+    inp = make_inputs_shape(2, 3, N, d, torch.bfloat16, seed=31 + d, seqlens=[1, 1])
+    q, k, v = (inp[n].cuda() for n in ("q", "k", "v"))
+    o, lse = fa.forward(q, k, v, causal=causal, seqlens=inp["seqlens"])
+    assert torch.equal(o, v[:, :, :1, :].expand_as(o))
+    s0 = (f64(q) * f64(k)[:, :, :1, :]).sum(-1) * d ** -0.5
+    assert np.abs(f64(lse) - s0).max() <= 1e-4
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_causal_row_zero_is_first_value_exactly(fa, d):
+    from exact_io_aware_47_b200.inputs import make_inputs_shape
+    inp = make_inputs_shape(2, 2, 777, d, torch.bfloat16, seed=41 + d)
+    q, k, v = (inp[n].cuda() for n in ("q", "k", "v"))
+    o, lse = fa.forward(q, k, v, causal=True)
+    assert torch.equal(o[:, :, 0], v[:, :, 0])
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("L", [3, 128, 129, 1000])
+def test_zero_query_gives_mean_within_one_ulp(fa, d, L):
+    # uniform scores: every p = 1 exactly, O = fp32 mean of the valid V rows,
+    # rounded once to bf16; LSE = ln L
+    from exact_io_aware_47_b200.inputs import make_inputs_shape
+    N = 1000
+    inp = make_inputs_shape(1, 2, N, d, torch.bfloat16, seed=L + d, seqlens=[L])
+    k, v = inp["k"].cuda(), inp["v"].cuda()
+    q = torch.zeros_like(k)
+    o, lse = fa.forward(q, k, v, seqlens=inp["seqlens"])
+    mean = f64(v)[:, :, :L].mean(axis=2, keepdims=True)
+    err = np.abs(f64(o) - mean)
+    assert (err <= _bf16_ulp(mean) * 0.5 + 1e-5 * np.abs(mean) + 1e-6).all(), err.max()
+    assert np.abs(f64(lse) - np.log(L)).max() <= 1e-5 * max(1.0, np.log(L))
