@@ -20,6 +20,7 @@ FA_ERR_DEVICE_TIMEOUT = 6
 FA_ERR_DEVICE_SEQLEN = 7
 FA_ERR_WORKSPACE = 8
 FA_ERR_DEVICE_LAYOUT = 9
+FA_ERR_SCRATCH_LIMIT = 10
 
 FA_BF16 = 0
 FA_FP16 = 1
@@ -35,6 +36,9 @@ SIGNATURES = {
     "fa_bwd_main": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _I, _I, _I, _I, _F, _I, _VP,
                          _I, _VP]),
     "fa_bwd_postprocess": (_I, [_VP, _SZ, _VP, _I, _I, _I, _I, _F, _I, _VP]),
+    "fa_bwd_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
+                            _I, _I, _I, _I, _F, _I, _VP, _I, _VP]),
+    "fa_bwd_noalloc_max_bytes": (_SZ, []),
     "fa_device_status": (_I, [_VP, ctypes.POINTER(ctypes.c_uint32)]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_version": (_I, []),
@@ -105,6 +109,16 @@ def fa_bwd_main(q, k, v, dout, lse, dk, dv, workspace, workspace_bytes, B, H, N,
 def fa_bwd_postprocess(workspace, workspace_bytes, dq, B, H, N, d, scale, dtype, stream):
     return load().fa_bwd_postprocess(workspace, workspace_bytes, dq, B, H, N, d, scale, dtype,
                                      stream)
+
+
+def fa_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal, seqlens, dtype,
+                   stream):
+    return load().fa_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal,
+                                 seqlens, dtype, stream)
+
+
+def fa_bwd_noalloc_max_bytes():
+    return load().fa_bwd_noalloc_max_bytes()
 
 
 def fa_device_status(stream):

@@ -273,6 +273,66 @@ extern "C" int fa_bwd(const void* q, const void* k, const void* v, const void* o
   return fa_bwd_postprocess(workspace, workspace_bytes, dq, B, H, N, d, scale, dtype, stream);
 }
 
+// ---------------------------------------------------------------------------
+// Backward pass without any allocation: the workspace is a static device
+// array of the library.
+//
+// Some callers cannot hand the library a workspace: plugin hosts that give an
+// operator only its input and output buffers and own every other byte of
+// device memory, and latency-critical paths that must not call cudaMalloc
+// (which may synchronise the device).  fa_bwd_noalloc serves them with a
+// fixed scratch array that every GPU loading the library holds until the
+// process exits.
+// ---------------------------------------------------------------------------
+namespace fa {
+namespace {
+
+constexpr size_t kStaticScratchBytes = 32ull << 20;  // 32 MiB per device
+static __device__ __align__(256) uint8_t g_bwd_scratch[kStaticScratchBytes];
+
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_bwd_scratch on the current device (host code cannot use
+// the symbol itself: on the host it names a stand-in, not device memory).
+// Looked up once per device, with that device current.
+int static_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_bwd_scratch) != cudaSuccess || ptr == nullptr)
+      return FA_ERR_CUDA;
+    g_scratch_ptr[dev] = ptr;
+  }
+  *out = g_scratch_ptr[dev];
+  return FA_OK;
+}
+
+}  // namespace
+}  // namespace fa
+
+extern "C" size_t fa_bwd_noalloc_max_bytes(void) { return kStaticScratchBytes; }
+
+extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                              const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                              int B, int H, int N, int d, float scale, int causal,
+                              const int32_t* seqlens, int dtype, void* stream) {
+  const size_t need = fa_bwd_workspace_size(B, H, N, d);
+  if (need == 0) {
+    const int st = check_common(B, H, N, d, scale, dtype);
+    return st != FA_OK ? st : FA_ERR_INVALID_ARG;
+  }
+  if (need > kStaticScratchBytes) return FA_ERR_SCRATCH_LIMIT;
+  void* scratch = nullptr;
+  const int st = static_scratch(&scratch);
+  if (st != FA_OK) return st;
+  // fa_bwd's preprocess rewrites the row dots and zeroes the dQ accumulator,
+  // so whatever an earlier call left in the array does not matter.
+  return fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, scratch, kStaticScratchBytes, B, H, N, d,
+                scale, causal, seqlens, dtype, stream);
+}
+
 extern "C" int fa_device_status(void* stream, uint32_t* detail) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
   unsigned int word = 0;
@@ -300,6 +360,8 @@ extern "C" const char* fa_status_string(int status) {
     case FA_ERR_DEVICE_SEQLEN: return "seqlens value outside [1, N] (clamped on device)";
     case FA_ERR_WORKSPACE: return "backward workspace missing or too small";
     case FA_ERR_DEVICE_LAYOUT: return "kernel refused: shared-memory window misaligned";
+    case FA_ERR_SCRATCH_LIMIT:
+      return "problem needs more backward scratch than fa_bwd_noalloc's static array holds";
     default: return "unknown status";
   }
 }

@@ -66,7 +66,8 @@ typedef enum {
   FA_ERR_DEVICE_TIMEOUT = 6,  /* device: a pipeline wait gave up (fa_device_status) */
   FA_ERR_DEVICE_SEQLEN = 7,   /* device: seqlens[b] outside [1, N] (fa_device_status) */
   FA_ERR_WORKSPACE = 8,       /* backward workspace missing or too small        */
-  FA_ERR_DEVICE_LAYOUT = 9    /* device: shared-memory window misaligned, kernel refused (fa_device_status) */
+  FA_ERR_DEVICE_LAYOUT = 9,   /* device: shared-memory window misaligned, kernel refused (fa_device_status) */
+  FA_ERR_SCRATCH_LIMIT = 10   /* fa_bwd_noalloc: workspace would exceed its static array */
 } fa_status;
 
 typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
@@ -125,6 +126,34 @@ int fa_bwd_main(const void* q, const void* k, const void* v, const void* dout,
 int fa_bwd_postprocess(void* workspace, size_t workspace_bytes, void* dq,
                        int B, int H, int N, int d, float scale, int dtype,
                        void* stream);
+
+/*
+ * Backward pass that allocates nothing and takes no workspace.  The pages
+ * have no counterpart: it exists for callers that cannot allocate device
+ * memory for a workspace, such as plugin hosts that hand an operator only its
+ * input and output buffers, or latency-critical paths that must not call
+ * cudaMalloc (which may synchronise the device).
+ *   Same arguments, results and checks as fa_bwd, minus the workspace.  The
+ *   workspace is a static device array of fa_bwd_noalloc_max_bytes()
+ *   (32 MiB) bytes inside the library, which every GPU that loads the
+ *   library holds until the process exits.  Problems with
+ *   fa_bwd_workspace_size(B, H, N, d) above that return FA_ERR_SCRATCH_LIMIT
+ *   before anything is launched (for d = 128 that is about 64K rows B*H*N).
+ *   All calls share the array: calls whose kernels overlap on the GPU (other
+ *   streams, other host threads) race and give wrong results; serialise them.
+ *   The array keeps the last call's contents; the preprocess stage rewrites
+ *   everything the call reads, so no clearing is needed between calls.
+ *   The first call on a device looks up the array's device address (once per
+ *   device, with that device current); make that first call before any
+ *   stream capture.
+ */
+int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                   const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                   int B, int H, int N, int d, float scale, int causal,
+                   const int32_t* seqlens, int dtype, void* stream);
+
+/* Size in bytes of the static workspace fa_bwd_noalloc uses. */
+size_t fa_bwd_noalloc_max_bytes(void);
 
 /*
  * Synchronises `stream`, then returns and clears the device status word of

@@ -93,6 +93,16 @@ def test_rejections_before_any_cuda_call(lib):
     assert bwd(H=0) == _lib.FA_ERR_INVALID_ARG
 
 
+def test_noalloc_size_limit_checked_on_the_host(lib):
+    from exact_io_aware_47_b200 import _lib
+    P = 1 << 20
+    assert lib.fa_bwd_noalloc_max_bytes() == 32 << 20
+    st = lib.fa_bwd_noalloc(P, P, P, P, P, P, P, P, P, 4, 32, 8192, 128, 0.088, 1, None, 0, None)
+    assert st == _lib.FA_ERR_SCRATCH_LIMIT
+    st = lib.fa_bwd_noalloc(P, P, P, P, P, P, P, P, P, 1, 1, 128, 96, 0.088, 1, None, 0, None)
+    assert st == _lib.FA_ERR_UNSUPPORTED
+
+
 def test_missing_library_fails_loudly(tmp_path):
     from exact_io_aware_47_b200 import _lib
     with pytest.raises(RuntimeError, match="missing"):
