@@ -380,7 +380,6 @@ __global__ void __launch_bounds__(512, 1)
         ok = mbar_wait_warp(&ld_full[st], (it >> 1) & 1, abort_flag, 28) &&
              mbar_wait_warp(s_full, it & 1, abort_flag, 29) &&
              mbar_wait_warp(dp_full, it & 1, abort_flag, 30);
-        if (ok && it > 0) ok = mbar_wait_warp(ds_empty, (it - 1) & 1, abort_flag, 31);
         if (!ok) break;
         tc_fence_after();
         if (threadIdx.x == 0) FA_TRACE_AT(it, 4);
@@ -419,6 +418,13 @@ __global__ void __launch_bounds__(512, 1)
           // over S^T columns this thread has already read, never the other
           // half's
           tmem_st16(tS + half * 64 + (c & 1) * 16, pp);
+          if (cc == 0 && it > 0) {
+            // the dS^T tile is free once the previous tile's MMAs and dQ
+            // staging are done with it; waiting only now overlaps that with
+            // the first chunk's arithmetic
+            ok = mbar_wait_warp(ds_empty, (it - 1) & 1, abort_flag, 31);
+            if (!ok) break;
+          }
           // four 16-byte units of the 128-byte swizzled row (chunk c = units
           // 4 (c & 1) .. 4 (c & 1) + 3 of panel `half`)
 #pragma unroll
@@ -428,6 +434,7 @@ __global__ void __launch_bounds__(512, 1)
                          dd[4 * w4 + 3]);
           }
         }
+        if (!ok) break;
         tmem_st_wait();
         fence_proxy_async_smem();
         tc_fence_before();
@@ -453,10 +460,12 @@ __global__ void __launch_bounds__(512, 1)
         tc_fence_after();
         if (threadIdx.x == 256) FA_TRACE_AT(it, 6);
         if constexpr (D == 128) {
-          // Lane r holds column r of dQ_i for the 128 query rows (dQ^T).  Two
-          // rounds of 64 rows: TMEM -> the dS^T tile reused as a [64][128]
-          // fp32 staging buffer -> one TMA reduce-add into the accumulator.
-          float* stg = reinterpret_cast<float*>(sDS);
+          // Lane r holds column r of dQ_i for the 128 query rows (dQ^T).  The
+          // dS^T tile (free: dQ^T and dK are done with it) becomes two 16 KB
+          // [32][128] fp32 staging buffers; four rounds of 32 rows alternate
+          // between them, each followed by one TMA reduce-add into the
+          // accumulator, so staging a round overlaps the previous round's
+          // transfer.
           const bool leader = warp == 8 && lane == 0;
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
@@ -466,16 +475,25 @@ __global__ void __launch_bounds__(512, 1)
               // all of dQ^T is in registers: the MMA may overwrite its columns
               tc_fence_before();
               mbar_arrive(dq_empty);
-              if (leader) bulk_wait_read_all();  // round 0 has left the buffer
-              named_bar_sync(1, 128);
             }
 #pragma unroll
-            for (int e = 0; e < 64; ++e) stg[e * D + r] = __uint_as_float(v[e]);
-            fence_proxy_async_smem();
-            named_bar_sync(1, 128);
-            if (leader) {
-              tma_reduce_add_3d(&tmdq, stg, 0, i * kBlockM + half * 64, w.bh);
-              bulk_commit_group();
+            for (int qr = 0; qr < 2; ++qr) {
+              const int round = half * 2 + qr;
+              float* stg = reinterpret_cast<float*>(sDS + (round & 1) * 16384);
+              if (round >= 2) {
+                // the transfer that used this buffer two rounds ago must have
+                // read it
+                if (leader) bulk_wait_read_one();
+                named_bar_sync(1, 128);
+              }
+#pragma unroll
+              for (int e = 0; e < 32; ++e) stg[e * D + r] = __uint_as_float(v[qr * 32 + e]);
+              fence_proxy_async_smem();
+              named_bar_sync(1, 128);
+              if (leader) {
+                tma_reduce_add_3d(&tmdq, stg, 0, i * kBlockM + round * 32, w.bh);
+                bulk_commit_group();
+              }
             }
           }
           if (leader) {
