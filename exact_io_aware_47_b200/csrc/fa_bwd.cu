@@ -52,10 +52,11 @@ struct BwdLayout {
   static constexpr int kPanels = D / 64;
   static constexpr int kK = 0;
   static constexpr int kV = kTileBytes;
-  static constexpr int kQ = 2 * kTileBytes;            // 2 stages
-  static constexpr int kDO = kQ + 2 * kTileBytes;      // 2 stages
-  static constexpr int kDS = kDO + 2 * kTileBytes;     // dS^T, 128 x 128 16-bit
-  static constexpr int kLSE = kDS + 128 * 128 * 2;     // 2 stages x 128 fp32
+  static constexpr int kSlot = 2 * kTileBytes;         // Q_i in slots 0/1 (alternating), dO_i in 2
+  static constexpr int kSlots = 3;
+  static constexpr int kDS = kSlot + kSlots * kTileBytes;  // dS^T, 128 x 128 16-bit
+  static constexpr int kSTG = kDS + 128 * 128 * 2;     // dQ staging: two [32][128] fp32
+  static constexpr int kLSE = kSTG + 2 * 32 * 128 * 4; // 2 stages x 128 fp32
   static constexpr int kDSUM = kLSE + 2 * 128 * 4;     // 2 stages x 128 fp32
   static constexpr int kBar = kDSUM + 2 * 128 * 4;
   static constexpr int kBarBytes = 256;
@@ -73,6 +74,18 @@ struct BwdLayout {
 struct BwdUnit {
   int bh, j, L, i0, ni;
 };
+
+// Register split: 512 threads launched at 128 registers (launch bounds 512,1);
+// the softmax warpgroups keep their P^T values between the two phases and the
+// dQ warpgroup holds a whole dQ^T row (128 fp32) before staging it, so they
+// take 144 each; the MMA/TMA/LSE warpgroup keeps 80: 2 * 144 + 144 + 80 =
+// 4 * 128.
+constexpr int kBwdLaunchRegs = 128;
+constexpr int kBwdSoftmaxRegs = 144;
+constexpr int kBwdDqRegs = 144;
+constexpr int kBwdOtherRegs = 80;
+static_assert(2 * kBwdSoftmaxRegs + kBwdDqRegs + kBwdOtherRegs <= 4 * kBwdLaunchRegs,
+              "register split");
 
 __device__ __forceinline__ BwdUnit bwd_decode(int u, const BwdParams& p) {
   BwdUnit w;
@@ -106,28 +119,29 @@ __global__ void __launch_bounds__(512, 1)
   }
   uint8_t* sK = smem + Lay::kK;
   uint8_t* sV = smem + Lay::kV;
-  uint8_t* sQ = smem + Lay::kQ;
-  uint8_t* sDO = smem + Lay::kDO;
+  uint8_t* sSlot = smem + Lay::kSlot;
   uint8_t* sDS = smem + Lay::kDS;
+  uint8_t* sSTG = smem + Lay::kSTG;
   float* sLSE = reinterpret_cast<float*>(smem + Lay::kLSE);
   float* sDSUM = reinterpret_cast<float*>(smem + Lay::kDSUM);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
   uint64_t* kv_full = bars + 0;
   uint64_t* kv_empty = bars + 1;
-  uint64_t* q_full = bars + 2;     // [2]
-  uint64_t* q_empty = bars + 4;    // [2]
-  uint64_t* ld_full = bars + 6;    // [2]
-  uint64_t* ld_empty = bars + 8;   // [2]
-  uint64_t* s_full = bars + 10;
-  uint64_t* dp_full = bars + 11;
-  uint64_t* p_full = bars + 12;
-  uint64_t* ds_empty = bars + 13;
-  uint64_t* dq_full = bars + 14;
-  uint64_t* dq_empty = bars + 15;
-  uint64_t* dkv_full = bars + 16;
-  uint64_t* dkv_empty = bars + 17;
-  uint64_t* drain = bars + 18;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 19);
+  uint64_t* slot_full = bars + 2;   // [3]
+  uint64_t* slot_empty = bars + 5;  // [3]
+  uint64_t* ld_full = bars + 8;     // [2]
+  uint64_t* ld_empty = bars + 10;   // [2]
+  uint64_t* s_full = bars + 12;
+  uint64_t* dp_full = bars + 13;
+  uint64_t* p_full = bars + 14;
+  uint64_t* ds_empty = bars + 15;
+  uint64_t* dq_full = bars + 16;
+  uint64_t* dq_empty = bars + 17;
+  uint64_t* dkv_full = bars + 18;
+  uint64_t* dkv_empty = bars + 19;
+  uint64_t* drain = bars + 20;
+  uint64_t* ds_full = bars + 21;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -136,15 +150,18 @@ __global__ void __launch_bounds__(512, 1)
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
     mbar_init(kv_empty, 1);
+    for (int s = 0; s < Lay::kSlots; ++s) {
+      mbar_init(&slot_full[s], 1);
+      mbar_init(&slot_empty[s], 1);
+    }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&q_full[s], 1);
-      mbar_init(&q_empty[s], 1);
       mbar_init(&ld_full[s], 32);
       mbar_init(&ld_empty[s], 256);
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
     mbar_init(p_full, 256);
+    mbar_init(ds_full, 256);
     mbar_init(ds_empty, 1);
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, 128);
@@ -163,6 +180,8 @@ __global__ void __launch_bounds__(512, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  if (warp >= 12) {
+  regs_decrease<kBwdOtherRegs>();
   if (warp == 13) {
     // ------------------------------------------------------------- TMA loads
     if (lane == 0) {
@@ -170,7 +189,7 @@ __global__ void __launch_bounds__(512, 1)
       tma_prefetch_desc(&tmk);
       tma_prefetch_desc(&tmv);
       tma_prefetch_desc(&tmdo);
-      int nunit = 0, qseq = 0;
+      int nunit = 0, lt = 0;  // lt: query tiles loaded (Q_lt -> slot lt & 1, dO_lt -> slot 2)
       bool ok = true;
       for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
         const BwdUnit w = bwd_decode(u, p);
@@ -185,27 +204,29 @@ __global__ void __launch_bounds__(512, 1)
         ++nunit;
         for (int idx = 0; idx < w.ni && ok; ++idx) {
           const int i = w.i0 + idx;
-          const int st = qseq & 1;
-          ok = mbar_wait(&q_empty[st], ((qseq >> 1) & 1) ^ 1, abort_flag, 21);
-          if (!ok) break;
-          mbar_arrive_expect_tx(&q_full[st], 2 * Lay::kTileBytes);
+          for (int t = 0; t < 2 && ok; ++t) {  // Q_i, then dO_i
+            const int slot = t == 0 ? (lt & 1) : 2;
+            const int use = t == 0 ? (lt >> 1) : lt;  // earlier loads into this slot
+            ok = mbar_wait(&slot_empty[slot], (use & 1) ^ 1, abort_flag, 21);
+            if (!ok) break;
+            FA_TRACE_AT(lt, 11 + t);
+            mbar_arrive_expect_tx(&slot_full[slot], Lay::kTileBytes);
 #pragma unroll
-          for (int pn = 0; pn < Lay::kPanels; ++pn) {
-            tma_load_3d(sQ + st * Lay::kTileBytes + pn * Lay::kPanelBytes, &tmq, &q_full[st],
-                        pn * 64, i * kBlockM, w.bh);
-            tma_load_3d(sDO + st * Lay::kTileBytes + pn * Lay::kPanelBytes, &tmdo, &q_full[st],
-                        pn * 64, i * kBlockM, w.bh);
+            for (int pn = 0; pn < Lay::kPanels; ++pn)
+              tma_load_3d(sSlot + slot * Lay::kTileBytes + pn * Lay::kPanelBytes,
+                          t == 0 ? &tmq : &tmdo, &slot_full[slot], pn * 64, i * kBlockM, w.bh);
           }
-          ++qseq;
+          ++lt;
         }
       }
       if (nunit > 0) mbar_wait_drain(kv_full, (nunit - 1) & 1, 200000000ull);
       for (int s = 0; s < 2; ++s) {
-        if (qseq > s) {
-          const int last = qseq - 1 - ((qseq - 1 - s) & 1);
-          mbar_wait_drain(&q_full[s], (last >> 1) & 1, 200000000ull);
+        if (lt > s) {
+          const int last = lt - 1 - ((lt - 1 - s) & 1);
+          mbar_wait_drain(&slot_full[s], (last >> 1) & 1, 200000000ull);
         }
       }
+      if (lt > 0) mbar_wait_drain(&slot_full[2], (lt - 1) & 1, 200000000ull);
     }
     __syncwarp();
   } else if (warp == 14) {
@@ -245,9 +266,9 @@ __global__ void __launch_bounds__(512, 1)
       // dQ = dS K (M = queries, N = d).
       constexpr uint32_t kIdDQ =
           D == 128 ? idesc_f16(BF16, 128, 128, true, true) : idesc_f16(BF16, 128, D, true, true);
-      const uint32_t aK = smem_addr(sK), aV = smem_addr(sV), aQ = smem_addr(sQ),
-                     aDO = smem_addr(sDO), aDS = smem_addr(sDS);
-      int nunit = 0, qseq = 0, it = 0;
+      const uint32_t aK = smem_addr(sK), aV = smem_addr(sV), aSlot = smem_addr(sSlot),
+                     aDS = smem_addr(sDS);
+      int nunit = 0, it = 0;
       bool ok = true;
       // K-major operands (A and B): 16-element steps walk 32 bytes inside a
       // 64-column panel, panels are 16 KB apart.
@@ -269,41 +290,83 @@ __global__ void __launch_bounds__(512, 1)
         // barrier never runs two phases ahead of its waiter, also for units
         // with no query tiles).
         bool dkv_free = nunit == 0;
-        for (int idx = 0; idx < w.ni && ok; ++idx) {
-          const int st = qseq & 1;
-          ok = mbar_wait(&q_full[st], (qseq >> 1) & 1, abort_flag, 24);
-          if (!ok) break;
-          tc_fence_after();
-          FA_TRACE_AT(it, 0);
-          const uint32_t q_s = aQ + st * Lay::kTileBytes;
-          const uint32_t do_s = aDO + st * Lay::kTileBytes;
-          // S^T = K_j Q_i^T
+        // Software pipeline over the query tiles of the unit:
+        //   S(0) | dP(i), dV(i), S(i+1), dK(i), dQ(i) | ...
+        // so the softmax of tile i+1 (first phase, from S) runs while the
+        // tensor core does dK(i) and dQ(i), and its second phase (from dP)
+        // while it does dV(i+1).
+        auto issue_s = [&](int t) {  // S^T(t) = K_j Q_t^T, Q_t in slot t & 1
+          const uint32_t q_s = aSlot + (t & 1) * Lay::kTileBytes;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
             umma_ss(tmem + Lay::kColS, kmaj(aK, kk), kmaj(q_s, kk), kIdS, kk > 0);
           umma_commit(s_full);
+        };
+        if (w.ni > 0) {
+          ok = mbar_wait(&slot_full[it & 1], (it >> 1) & 1, abort_flag, 24);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(it);
+        }
+        for (int idx = 0; idx < w.ni && ok; ++idx) {
+          FA_TRACE_AT(it, 0);
+          const uint32_t q_s = aSlot + (it & 1) * Lay::kTileBytes;
+          const uint32_t do_s = aSlot + 2 * Lay::kTileBytes;
           // d = 128: dQ^T of the previous tile lives in the dP^T columns
           if (D == 128 && it > 0) {
             ok = mbar_wait(dq_empty, (it - 1) & 1, abort_flag, 25);
             if (!ok) break;
-            tc_fence_after();
           }
+          FA_TRACE_AT(it, 10);
+          ok = mbar_wait(&slot_full[2], it & 1, abort_flag, 35);
+          if (!ok) break;
+          tc_fence_after();
           FA_TRACE_AT(it, 1);
           // dP^T = V_j dO_i^T
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk)
             umma_ss(tmem + Lay::kColDP, kmaj(aV, kk), kmaj(do_s, kk), kIdS, kk > 0);
           umma_commit(dp_full);
+          // dV_j += P^T dO_i once the first softmax phase wrote P^T
           ok = mbar_wait(p_full, it & 1, abort_flag, 26);
           if (!ok) break;
           tc_fence_after();
           FA_TRACE_AT(it, 2);
+          if (!dkv_free) {
+            ok = mbar_wait(dkv_empty, (nunit - 1) & 1, abort_flag, 27);
+            if (!ok) break;
+            tc_fence_after();
+            dkv_free = true;
+          }
+          // (A = P^T in TMEM, 16 queries = 8 columns; queries 64..127 sit 64
+          // columns further, in the second half's S^T columns)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_ts(tmem + Lay::kColDV, tmem + Lay::kColS + (kk >> 2) * 64 + (kk & 3) * 8,
+                    mnmaj(do_s, kk), kIdTS, (idx > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&slot_empty[2]);  // dO_i: dP and dV done
+          // S^T of the next tile: its MMA runs after dV (in order), which has
+          // read P^T out of these columns
+          if (idx + 1 < w.ni) {
+            ok = mbar_wait(&slot_full[(it + 1) & 1], ((it + 1) >> 1) & 1, abort_flag, 24);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(it + 1);
+          }
+          // dK_j += dS^T Q_i once the second phase wrote dS^T
+          ok = mbar_wait(ds_full, it & 1, abort_flag, 36);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_ss(tmem + Lay::kColDK, kmaj(aDS, kk), mnmaj(q_s, kk), kIdTS,
+                    (idx > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&slot_empty[it & 1]);  // Q_i: S and dK done
           if (D == 64 && it > 0) {
             ok = mbar_wait(dq_empty, (it - 1) & 1, abort_flag, 25);
             if (!ok) break;
             tc_fence_after();
           }
-          // dQ first, so its read-out overlaps the dV and dK MMAs
           if constexpr (D == 128) {
             // dQ^T = K_j^T dS^T: A = K_j read MN-major (d contiguous), B = dS^T
             // read MN-major (queries contiguous)
@@ -316,34 +379,9 @@ __global__ void __launch_bounds__(512, 1)
             for (int kk = 0; kk < 8; ++kk)
               umma_ss(tmem + Lay::kColDQ, mnmaj(aDS, kk), mnmaj(aK, kk), kIdDQ, kk > 0);
           }
-          if (D == 64) umma_commit(dq_full);
+          umma_commit(dq_full);
+          umma_commit(ds_empty);  // dK and dQ have read dS^T
           FA_TRACE_AT(it, 3);
-          if (!dkv_free) {
-            ok = mbar_wait(dkv_empty, (nunit - 1) & 1, abort_flag, 27);
-            if (!ok) break;
-            tc_fence_after();
-            dkv_free = true;
-          }
-          // dK_j += dS^T Q_i   (A = dS^T in shared memory, K-major)
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            umma_ss(tmem + Lay::kColDK, kmaj(aDS, kk), mnmaj(q_s, kk), kIdTS,
-                    (idx > 0 || kk > 0) ? 1u : 0u);
-          if constexpr (D == 128) {
-            // dQ^T and dK done = the dS^T tile has no MMA reader left: the dQ
-            // warps may stage dQ^T in it
-            umma_commit(dq_full);
-          } else {
-            umma_commit(ds_empty);
-          }
-          // dV_j += P^T dO_i   (A = P^T in TMEM, 16 queries = 8 columns; queries
-          // 64..127 sit 64 columns further, in the second half's S^T columns)
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            umma_ts(tmem + Lay::kColDV, tmem + Lay::kColS + (kk >> 2) * 64 + (kk & 3) * 8,
-                    mnmaj(do_s, kk), kIdTS, (idx > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(&q_empty[st]);
-          ++qseq;
           ++it;
         }
         if (!ok) break;
@@ -359,7 +397,10 @@ __global__ void __launch_bounds__(512, 1)
       mbar_wait_drain(drain, 0, 200000000ull);
     }
     __syncwarp();
+  }
+  // warp 15 has no role
   } else if (warp < 8) {
+    regs_increase<kBwdSoftmaxRegs>();
     // ------------------------- P^T and dS^T: key row per thread, half the queries
     const int half = warp >> 2;              // queries [64 half, 64 half + 64)
     const int r = ((warp & 3) << 5) | lane;  // key row in the tile = TMEM lane
@@ -377,9 +418,9 @@ __global__ void __launch_bounds__(512, 1)
       for (int idx = 0; idx < w.ni && ok; ++idx) {
         const int i = w.i0 + idx;
         const int st = it & 1;  // LSE/D staging advances with the iteration count
+        // ---- phase 1: P^T = 2^(c S^T - LSE_i log2 e) from S^T, back to TMEM
         ok = mbar_wait_warp(&ld_full[st], (it >> 1) & 1, abort_flag, 28) &&
-             mbar_wait_warp(s_full, it & 1, abort_flag, 29) &&
-             mbar_wait_warp(dp_full, it & 1, abort_flag, 30);
+             mbar_wait_warp(s_full, it & 1, abort_flag, 29);
         if (!ok) break;
         tc_fence_after();
         if (threadIdx.x == 0) FA_TRACE_AT(it, 4);
@@ -387,43 +428,58 @@ __global__ void __launch_bounds__(512, 1)
         const int diag_lim = (p.causal && i == w.j) ? r : -1;  // visible iff q_local >= r
         const float* lse2 = sLSE + st * 128;
         const float* dsm = sDSUM + st * 128;
+        float pv[64];  // this thread's P^T values, kept for the second phase
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           const int c = half * 2 + cc;  // 32-query chunk
-          uint32_t sr[32], dr[32];
+          uint32_t sr[32];
           tmem_ld32(tS + c * 32, sr);
-          tmem_ld32(tDP + c * 32, dr);
-          uint32_t pp[16], dd[16];
+          uint32_t pp[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 4) {
             const int q0 = c * 32 + e;
             const float4 l4 = *reinterpret_cast<const float4*>(lse2 + q0);
-            const float4 d4 = *reinterpret_cast<const float4*>(dsm + q0);
             const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-            const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
-            float pv[4], gv[4];
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
               const bool vis = key_ok && (q0 + k4 >= diag_lim);
               const float x = fmaf(__uint_as_float(sr[e + k4]), cl, -lv[k4]);
-              pv[k4] = vis ? ex2_approx(x) : 0.f;
-              gv[k4] = pv[k4] * (__uint_as_float(dr[e + k4]) - dv4[k4]);
+              pv[cc * 32 + e + k4] = vis ? ex2_approx(x) : 0.f;
             }
-            pp[(e >> 1)] = pack2<BF16>(pv[0], pv[1]);
-            pp[(e >> 1) + 1] = pack2<BF16>(pv[2], pv[3]);
-            dd[(e >> 1)] = pack2<BF16>(gv[0], gv[1]);
-            dd[(e >> 1) + 1] = pack2<BF16>(gv[2], gv[3]);
+            pp[(e >> 1)] = pack2<BF16>(pv[cc * 32 + e], pv[cc * 32 + e + 1]);
+            pp[(e >> 1) + 1] = pack2<BF16>(pv[cc * 32 + e + 2], pv[cc * 32 + e + 3]);
           }
           // P^T of queries [32c, 32c+32) goes to columns 64 half + 16 (c & 1): only
           // over S^T columns this thread has already read, never the other
           // half's
           tmem_st16(tS + half * 64 + (c & 1) * 16, pp);
-          if (cc == 0 && it > 0) {
-            // the dS^T tile is free once the previous tile's MMAs and dQ
-            // staging are done with it; waiting only now overlaps that with
-            // the first chunk's arithmetic
-            ok = mbar_wait_warp(ds_empty, (it - 1) & 1, abort_flag, 31);
-            if (!ok) break;
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(p_full);
+        if (threadIdx.x == 0) FA_TRACE_AT(it, 15);
+        // ---- phase 2: dS^T = P^T * (dP^T - D_i) from dP^T, to shared memory
+        ok = mbar_wait_warp(dp_full, it & 1, abort_flag, 30);
+        if (ok && it > 0) ok = mbar_wait_warp(ds_empty, (it - 1) & 1, abort_flag, 31);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = half * 2 + cc;
+          uint32_t dr[32];
+          tmem_ld32(tDP + c * 32, dr);
+          uint32_t dd[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            const int q0 = c * 32 + e;
+            const float4 d4 = *reinterpret_cast<const float4*>(dsm + q0);
+            const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+            float gv[4];
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4)
+              gv[k4] = pv[cc * 32 + e + k4] * (__uint_as_float(dr[e + k4]) - dv4[k4]);
+            dd[(e >> 1)] = pack2<BF16>(gv[0], gv[1]);
+            dd[(e >> 1) + 1] = pack2<BF16>(gv[2], gv[3]);
           }
           // four 16-byte units of the 128-byte swizzled row (chunk c = units
           // 4 (c & 1) .. 4 (c & 1) + 3 of panel `half`)
@@ -434,21 +490,20 @@ __global__ void __launch_bounds__(512, 1)
                          dd[4 * w4 + 3]);
           }
         }
-        if (!ok) break;
-        tmem_st_wait();
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(p_full);
+        mbar_arrive(ds_full);
         mbar_arrive(&ld_empty[st]);
         if (threadIdx.x == 0) FA_TRACE_AT(it, 5);
         ++it;
       }
     }
-  } else if (warp < 12) {
+  } else {
+    regs_increase<kBwdDqRegs>();
     // --------------------------- dQ read-out and reduce-add; dK_j, dV_j epilogue
     const int r = ((warp & 3) << 5) | lane;  // TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    int it = 0, nunit = 0;
+    int it = 0, nunit = 0, stage_round = 0;
     bool ok = true;
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
       const BwdUnit w = bwd_decode(u, p);
@@ -460,45 +515,35 @@ __global__ void __launch_bounds__(512, 1)
         tc_fence_after();
         if (threadIdx.x == 256) FA_TRACE_AT(it, 6);
         if constexpr (D == 128) {
-          // Lane r holds column r of dQ_i for the 128 query rows (dQ^T).  The
-          // dS^T tile (free: dQ^T and dK are done with it) becomes two 16 KB
-          // [32][128] fp32 staging buffers; four rounds of 32 rows alternate
-          // between them, each followed by one TMA reduce-add into the
-          // accumulator, so staging a round overlaps the previous round's
-          // transfer.
+          // Lane r holds column r of dQ_i for the 128 query rows (dQ^T).  Read
+          // it all, release the TMEM columns, then four rounds of 32 rows
+          // alternate between two 16 KB [32][128] fp32 staging buffers, each
+          // followed by one TMA reduce-add into the accumulator (the TMA path
+          // sustains more reduce bandwidth per SM than per-thread reds);
+          // staging a round overlaps the previous transfer.
           const bool leader = warp == 8 && lane == 0;
+          uint32_t v[128];
+          tmem_ld64x2(tmem + lane_off + Lay::kColDQ, v);
+          tc_fence_before();
+          mbar_arrive(dq_empty);
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            uint32_t v[64];
-            tmem_ld64(tmem + lane_off + Lay::kColDQ + half * 64, v);
-            if (half == 1) {
-              // all of dQ^T is in registers: the MMA may overwrite its columns
-              tc_fence_before();
-              mbar_arrive(dq_empty);
-            }
-#pragma unroll
-            for (int qr = 0; qr < 2; ++qr) {
-              const int round = half * 2 + qr;
-              float* stg = reinterpret_cast<float*>(sDS + (round & 1) * 16384);
-              if (round >= 2) {
-                // the transfer that used this buffer two rounds ago must have
-                // read it
-                if (leader) bulk_wait_read_one();
-                named_bar_sync(1, 128);
-              }
-#pragma unroll
-              for (int e = 0; e < 32; ++e) stg[e * D + r] = __uint_as_float(v[qr * 32 + e]);
-              fence_proxy_async_smem();
+          for (int rd = 0; rd < 4; ++rd) {
+            float* stg = reinterpret_cast<float*>(sSTG + (stage_round & 1) * 16384);
+            if (stage_round >= 2) {
+              // the transfer that used this buffer two rounds ago must have
+              // read it
+              if (leader) bulk_wait_read_one();
               named_bar_sync(1, 128);
-              if (leader) {
-                tma_reduce_add_3d(&tmdq, stg, 0, i * kBlockM + round * 32, w.bh);
-                bulk_commit_group();
-              }
             }
-          }
-          if (leader) {
-            bulk_wait_read_all();
-            mbar_arrive(ds_empty);  // the softmax warps may write dS^T again
+#pragma unroll
+            for (int e = 0; e < 32; ++e) stg[e * D + r] = __uint_as_float(v[rd * 32 + e]);
+            fence_proxy_async_smem();
+            named_bar_sync(1, 128);
+            if (leader) {
+              tma_reduce_add_3d(&tmdq, stg, 0, i * kBlockM + rd * 32, w.bh);
+              bulk_commit_group();
+            }
+            ++stage_round;
           }
         } else {
           const int row = i * kBlockM + r;
@@ -569,7 +614,6 @@ __global__ void __launch_bounds__(512, 1)
     // every reduce-add issued must have completed before the kernel ends
     if (D == 128 && warp == 8 && lane == 0) bulk_wait_all();
   }
-  // warp 15 has no role
 
   tc_fence_before();
   __syncthreads();
@@ -669,8 +713,12 @@ static cudaError_t launch_bwd_main_t(const CUtensorMap& tmq, const CUtensorMap& 
                                      cudaStream_t stream) {
   using Lay = BwdLayout<D>;
   auto kern = fa_bwd_kernel<D, BF16>;
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kSmemBytes);
+  cudaFuncAttributes attr;
+  cudaError_t e = cudaFuncGetAttributes(&attr, kern);
+  if (e != cudaSuccess) return e;
+  // the register split in the kernel assumes exactly this launch allocation
+  if (attr.numRegs != kBwdLaunchRegs) return cudaErrorInvalidConfiguration;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kSmemBytes);
   if (e != cudaSuccess) return e;
   const int grid = p.n_units < num_sms ? p.n_units : num_sms;
   kern<<<grid, 512, Lay::kSmemBytes, stream>>>(tmq, tmk, tmv, tmdo, tmdq, p);
