@@ -144,7 +144,7 @@ extern "C" int fa_fwd(const void* q, const void* k, const void* v, void* o, floa
   p.causal = causal ? 1 : 0;
   p.n_qtiles = (N + kBlockM - 1) / kBlockM;
   p.n_pairs = (p.n_qtiles + 1) / 2;
-  p.n_units = BH * p.n_pairs;
+  p.n_units = BH * ((p.n_pairs + 1) / 2);
   const cudaError_t e =
       launch_fwd(d, dtype == FA_BF16, tq, tk, tv, p, di.num_sms, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -182,7 +182,7 @@ int bwd_common(void* workspace, size_t workspace_bytes, int B, int H, int N, int
   p->scale = scale;
   p->scale_log2 = scale * 1.4426950408889634f;
   p->n_ktiles = (N + kBlockN - 1) / kBlockN;
-  p->n_units = B * H * p->n_ktiles;
+  p->n_units = B * H * ((p->n_ktiles + 1) / 2);
   return FA_OK;
 }
 

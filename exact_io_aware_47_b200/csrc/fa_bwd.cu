@@ -87,10 +87,12 @@ constexpr int kBwdOtherRegs = 80;
 static_assert(2 * kBwdSoftmaxRegs + kBwdDqRegs + kBwdOtherRegs <= 4 * kBwdLaunchRegs,
               "register split");
 
-__device__ __forceinline__ BwdUnit bwd_decode(int u, const BwdParams& p) {
+// Unit (bh, key tile j).  The work order hands out key tiles mirrored
+// (j = n-1-idx), so the long tile of a causal super-unit (small j) runs first.
+__device__ __forceinline__ BwdUnit bwd_decode(int bh, int idx, const BwdParams& p) {
   BwdUnit w;
-  w.bh = u / p.n_ktiles;
-  w.j = u % p.n_ktiles;  // causal: small j has the most query tiles, so runs first
+  w.bh = bh;
+  w.j = p.n_ktiles - 1 - idx;
   const int b = w.bh / p.H;
   int L = p.N;
   if (p.seqlens != nullptr) {
@@ -191,8 +193,11 @@ __global__ void __launch_bounds__(512, 1)
       tma_prefetch_desc(&tmdo);
       int nunit = 0, lt = 0;  // lt: query tiles loaded (Q_lt -> slot lt & 1, dO_lt -> slot 2)
       bool ok = true;
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-        const BwdUnit w = bwd_decode(u, p);
+      for (int k = 0; ok; ++k) {
+        WorkItem wi;
+        if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
+        if (wi.idx < 0) continue;
+        const BwdUnit w = bwd_decode(wi.bh, wi.idx, p);
         ok = mbar_wait(kv_empty, (nunit & 1) ^ 1, abort_flag, 20);
         if (!ok) break;
         mbar_arrive_expect_tx(kv_full, 2 * Lay::kTileBytes);
@@ -234,8 +239,11 @@ __global__ void __launch_bounds__(512, 1)
     int seq = 0;
     bool ok = true;
     const float log2e = 1.4426950408889634f;
-    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-      const BwdUnit w = bwd_decode(u, p);
+    for (int k = 0; ok; ++k) {
+      WorkItem wi;
+      if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
+      if (wi.idx < 0) continue;
+      const BwdUnit w = bwd_decode(wi.bh, wi.idx, p);
       const size_t base = static_cast<size_t>(w.bh) * p.N;
       for (int idx = 0; idx < w.ni && ok; ++idx) {
         const int i = w.i0 + idx;
@@ -280,8 +288,11 @@ __global__ void __launch_bounds__(512, 1)
       auto mnmaj = [](uint32_t base, int kk) {
         return sdesc_sw128(base + kk * 2048, 16384, 1024);
       };
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-        const BwdUnit w = bwd_decode(u, p);
+      for (int k = 0; ok; ++k) {
+        WorkItem wi;
+        if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
+        if (wi.idx < 0) continue;
+        const BwdUnit w = bwd_decode(wi.bh, wi.idx, p);
         ok = mbar_wait(kv_full, nunit & 1, abort_flag, 23);
         if (!ok) break;
         tc_fence_after();
@@ -412,8 +423,11 @@ __global__ void __launch_bounds__(512, 1)
     const float cl = p.scale_log2;
     int it = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-      const BwdUnit w = bwd_decode(u, p);
+    for (int k = 0; ok; ++k) {
+      WorkItem wi;
+      if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
+      if (wi.idx < 0) continue;
+      const BwdUnit w = bwd_decode(wi.bh, wi.idx, p);
       const bool key_ok = w.j * kBlockN + r < w.L;
       for (int idx = 0; idx < w.ni && ok; ++idx) {
         const int i = w.i0 + idx;
@@ -505,8 +519,11 @@ __global__ void __launch_bounds__(512, 1)
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     int it = 0, nunit = 0, stage_round = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-      const BwdUnit w = bwd_decode(u, p);
+    for (int k = 0; ok; ++k) {
+      WorkItem wi;
+      if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
+      if (wi.idx < 0) continue;
+      const BwdUnit w = bwd_decode(wi.bh, wi.idx, p);
       const size_t base = static_cast<size_t>(w.bh) * p.N;
       for (int idx = 0; idx < w.ni && ok; ++idx) {
         const int i = w.i0 + idx;

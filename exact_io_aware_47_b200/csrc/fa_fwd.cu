@@ -60,13 +60,10 @@ struct FwdUnit {
   int bh, qt0, L, jend0, jend1;
 };
 
-__device__ __forceinline__ FwdUnit fwd_decode(int u, const FwdParams& p) {
+// Unit (bh, pair): query tiles 2 pair and 2 pair + 1 of head bh.
+__device__ __forceinline__ FwdUnit fwd_decode(int bh, int pair, const FwdParams& p) {
   FwdUnit w;
-  const int r = u % p.n_pairs;
-  w.bh = u / p.n_pairs;
-  // causal units of one head run longest-first; heads stay contiguous so the
-  // CTAs running at the same time share K/V in L2
-  const int pair = p.causal ? (p.n_pairs - 1 - r) : r;
+  w.bh = bh;
   const int b = w.bh / p.H;
   int L = p.N;
   if (p.seqlens != nullptr) {
@@ -150,8 +147,11 @@ __global__ void __launch_bounds__(384, 1)
       int qload[2] = {0, 0};
       int kv_seq = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-        const FwdUnit w = fwd_decode(u, p);
+      for (int k = 0; ok; ++k) {
+        WorkItem wi;
+        if (!work_item(k, p.n_pairs, p.B * p.H, wi)) break;
+        if (wi.idx < 0) continue;
+        const FwdUnit w = fwd_decode(wi.bh, wi.idx, p);
         const int je[2] = {w.jend0, w.jend1};
         for (int t = 0; t < 2 && ok; ++t) {
           if (je[t] == 0) continue;
@@ -231,8 +231,11 @@ __global__ void __launch_bounds__(384, 1)
         }
       };
 
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-        const FwdUnit w = fwd_decode(u, p);
+      for (int k = 0; ok; ++k) {
+        WorkItem wi;
+        if (!work_item(k, p.n_pairs, p.B * p.H, wi)) break;
+        if (wi.idx < 0) continue;
+        const FwdUnit w = fwd_decode(wi.bh, wi.idx, p);
         const int je[2] = {w.jend0, w.jend1};
         const int jmax = max(je[0], je[1]);
         for (int t = 0; t < 2 && ok; ++t) {
@@ -313,8 +316,11 @@ __global__ void __launch_bounds__(384, 1)
     const float c = p.scale_log2;
     int scnt = 0, ocnt = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-      const FwdUnit w = fwd_decode(u, p);
+    for (int k = 0; ok; ++k) {
+      WorkItem wi;
+      if (!work_item(k, p.n_pairs, p.B * p.H, wi)) break;
+      if (wi.idx < 0) continue;
+      const FwdUnit w = fwd_decode(wi.bh, wi.idx, p);
       const int jend = t == 0 ? w.jend0 : w.jend1;
       if (jend == 0) continue;
       const int qt = w.qt0 + t;

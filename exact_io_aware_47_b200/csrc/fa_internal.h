@@ -25,8 +25,8 @@ struct FwdParams {
   float scale_log2;         // scale * log2(e)
   int causal;
   int n_qtiles;             // ceil(N / 128)
-  int n_pairs;              // ceil(n_qtiles / 2): a CTA work unit is two query tiles
-  int n_units;              // B * H * n_pairs
+  int n_pairs;              // ceil(n_qtiles / 2): a work unit is two query tiles
+  int n_units;              // B * H * ceil(n_pairs / 2) super-units (see work_item)
 };
 
 struct BwdParams {
@@ -47,8 +47,32 @@ struct BwdParams {
   float scale_log2;
   int causal;
   int n_ktiles;             // ceil(N / 128)
-  int n_units;              // B * H * n_ktiles
+  int n_units;              // B * H * ceil(n_ktiles / 2) super-units (see work_item)
 };
+
+// Work order of the persistent kernels.  A head's units (query-tile pairs in
+// the forward, key tiles in the backward) are paired with their mirror: unit
+// m and unit n-1-m form one super-unit, which costs the same for every m
+// under a causal mask (long + short).  CTA c takes super-units c, c + grid,
+// ... (head-major, so CTAs running together share K/V and dQ rows in L2) and
+// runs the two halves back to back.  k counts the work items of this CTA;
+// returns false past the end; idx < 0 marks the missing mirror of an odd
+// middle unit.
+struct WorkItem {
+  int bh;   // batch * head
+  int idx;  // unit index inside the head: n-1-m for the first half, m for the second
+};
+
+__device__ __forceinline__ bool work_item(int k, int per_head, int heads, WorkItem& wi) {
+  const int half = (per_head + 1) >> 1;
+  const int su = blockIdx.x + (k >> 1) * gridDim.x;
+  if (su >= heads * half) return false;
+  wi.bh = su / half;
+  const int m = su - wi.bh * half;
+  const int a = per_head - 1 - m;
+  wi.idx = (k & 1) == 0 ? a : (m != a ? m : -1);
+  return true;
+}
 
 // Host launchers (defined in the .cu files).  They assume validated
 // arguments and return a cudaError_t from the launch.
