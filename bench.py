@@ -143,11 +143,13 @@ def dist_setup():
 
 
 def dist_max(x, world):
+    """Max of x over the ranks (the device-timed region of the slowest rank)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -184,7 +186,7 @@ def run_reference(args, w):
     # host-only program: rank 0 runs it, other ranks exit without work
     if int(os.environ.get("RANK", "0")) != 0:
         return 0
-    n_rows = 4096
+    n_rows = min(4096, w.N)
     for _ in range(args.warmup):
         oracle_sample(w, n_rows)
     tot_t, tot_f, thr = 0.0, 0.0, 1
