@@ -368,6 +368,7 @@ extern "C" const char* fa_status_string(int status) {
 
 extern "C" int fa_version(void) { return 100; }
 
+
 #ifdef FA_TRACE
 // Trace builds only: copy the device timeline (see FA_TRACE_AT) to the host.
 extern "C" int fa_trace_read(unsigned long long* host, int n) {

@@ -205,17 +205,21 @@ __global__ void __launch_bounds__(384, 1)
       int kv_seq = 0;
       bool ok = true;
 
+      // Shared-memory descriptors of the fixed buffers, built once; an MMA
+      // moves them with one add.
+      const uint64_t dQ0 = sdesc_sw128(sq_addr, 16, 1024);                  // K-major
+      const uint64_t dK0 = sdesc_sw128(skv_addr, 16, 1024);                 // K-major
+      const uint64_t dV0 = sdesc_sw128(skv_addr, Lay::kPanelBytes, 1024);   // MN-major
       // S_t = Q_t K^T: A = Q tile (K-major), B = K tile (K-major); the
       // 16-element K steps walk 32 bytes inside a 128-byte swizzle panel.
       auto issue_s = [&](int t, int kslot) {
         const uint32_t d_tmem = tmem + t * 128;
-        const uint32_t qa = sq_addr + t * Lay::kTileBytes;
-        const uint32_t kb = skv_addr + kslot * Lay::kTileBytes;
+        const uint64_t qa = sdesc_add(dQ0, t * Lay::kTileBytes);
+        const uint64_t kb = sdesc_add(dK0, kslot * Lay::kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * Lay::kPanelBytes + (kk & 3) * 32;
-          umma_ss(d_tmem, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024),
-                  kIdescQK, kk > 0 ? 1u : 0u);
+          umma_ss(d_tmem, sdesc_add(qa, off), sdesc_add(kb, off), kIdescQK, kk > 0 ? 1u : 0u);
         }
       };
       // O_t += P_t V: A = P (16-bit, TMEM, over S_t), B = V tile read
@@ -223,11 +227,11 @@ __global__ void __launch_bounds__(384, 1)
       // 16 KB apart.
       auto issue_pv = [&](int t, int vslot, bool acc) {
         const uint32_t d_tmem = tmem + Lay::kColO + t * D;
-        const uint32_t vb = skv_addr + vslot * Lay::kTileBytes;
+        const uint64_t vb = sdesc_add(dV0, vslot * Lay::kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < kBlockN / 16; ++kk) {
-          umma_ts(d_tmem, tmem + t * 128 + kk * 8, sdesc_sw128(vb + kk * 2048, Lay::kPanelBytes, 1024),
-                  kIdescPV, (acc || kk > 0) ? 1u : 0u);
+          umma_ts(d_tmem, tmem + t * 128 + kk * 8, sdesc_add(vb, kk * 2048), kIdescPV,
+                  (acc || kk > 0) ? 1u : 0u);
         }
       };
 
@@ -366,23 +370,32 @@ __global__ void __launch_bounds__(384, 1)
         l *= alpha;
         m = m_new;
         // p = 2^(c s - m): packed FMA on pairs, then ex2; row sum in fp32 over
-        // four independent accumulators
+        // four packed accumulators
         const float mu = (m == -INFINITY) ? 0.f : m;
         const unsigned long long c2 = f2pack(c, c);
         const unsigned long long nm2 = f2pack(-mu, -mu);
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        unsigned long long acc[4] = {0ull, 0ull, 0ull, 0ull};
         uint32_t pk[64];
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
+          const unsigned long long x2 =
+              ffma2(f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), c2, nm2);
           float x0, x1;
-          f2unpack(ffma2(f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), c2, nm2),
-                   x0, x1);
-          const float p0 = ex2_approx(x0);
-          const float p1 = ex2_approx(x1);
-          acc[i & 3] += p0 + p1;
+          f2unpack(x2, x0, x1);
+          const unsigned long long p2 = f2pack(ex2_approx(x0), ex2_approx(x1));
+          acc[i & 3] = fadd2(acc[i & 3], p2);
+          float p0, p1;
+          f2unpack(p2, p0, p1);
           pk[i] = pack2<BF16>(p0, p1);
         }
-        l += (acc[0] + acc[1]) + (acc[2] + acc[3]);
+        {
+          float a0, a1, b0, b1, c0, c1, d0, d1;
+          f2unpack(acc[0], a0, a1);
+          f2unpack(acc[1], b0, b1);
+          f2unpack(acc[2], c0, c1);
+          f2unpack(acc[3], d0, d1);
+          l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
+        }
         tmem_st64(tS, pk);
         if (j > 0 && __any_sync(0xffffffffu, moved)) {
           // O_t holds the sum up to tile j-1 (its MMA completed before S_t(j)

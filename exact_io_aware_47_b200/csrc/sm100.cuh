@@ -259,6 +259,13 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   return d;
 }
 
+// The same descriptor moved by `bytes` (a multiple of 16): only the 14-bit
+// start-address field changes, and with shared memory below 256 KB it cannot
+// carry into the next field.
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t bytes) {
+  return desc + static_cast<uint64_t>(bytes >> 4);
+}
+
 // Instruction descriptor, kind::f16 with fp32 accumulation.
 __host__ __device__ constexpr uint32_t idesc_f16(bool bf16, int M, int N, bool a_mn_major,
                                                  bool b_mn_major) {
