@@ -91,17 +91,19 @@ int make_map(CUtensorMap* map, const void* ptr, int BH, int N, int d, int dtype)
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
-// [B*H, N, d] fp32 view of the dQ accumulator for TMA reduce-adds of 32 rows
-// x d columns, no swizzle; rows past N inside a head are skipped.
+// [B*H, N, d] fp32 view of the dQ accumulator for TMA reduce-adds of 128 rows
+// x 32 columns; rows past N inside a head are skipped.
 int make_map_acc(CUtensorMap* map, void* ptr, int BH, int N, int d) {
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                               static_cast<cuuint64_t>(BH)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4,
                                  static_cast<cuuint64_t>(N) * d * 4};
-  const cuuint32_t box[3] = {static_cast<cuuint32_t>(d), 32, 1};
+  // box: 32 columns (128 bytes) x 128 rows, read from a 128-byte-swizzled
+  // shared tile
+  const cuuint32_t box[3] = {32, 128, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box,
-                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;

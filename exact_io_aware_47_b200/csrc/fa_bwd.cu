@@ -55,7 +55,7 @@ struct BwdLayout {
   static constexpr int kSlot = 2 * kTileBytes;         // Q_i in slots 0/1 (alternating), dO_i in 2
   static constexpr int kSlots = 3;
   static constexpr int kDS = kSlot + kSlots * kTileBytes;  // dS^T, 128 x 128 16-bit
-  static constexpr int kSTG = kDS + 128 * 128 * 2;     // dQ staging: two [32][128] fp32
+  static constexpr int kSTG = kDS + 128 * 128 * 2;     // dQ staging: two [128][32] fp32
   static constexpr int kLSE = kSTG + 2 * 32 * 128 * 4; // 2 stages x 128 fp32
   static constexpr int kDSUM = kLSE + 2 * 128 * 4;     // 2 stages x 128 fp32
   static constexpr int kBar = kDSUM + 2 * 128 * 4;
@@ -214,7 +214,6 @@ __global__ void __launch_bounds__(512, 1)
             const int use = t == 0 ? (lt >> 1) : lt;  // earlier loads into this slot
             ok = mbar_wait(&slot_empty[slot], (use & 1) ^ 1, abort_flag, 21);
             if (!ok) break;
-            FA_TRACE_AT(lt, 11 + t);
             mbar_arrive_expect_tx(&slot_full[slot], Lay::kTileBytes);
 #pragma unroll
             for (int pn = 0; pn < Lay::kPanels; ++pn)
@@ -250,14 +249,14 @@ __global__ void __launch_bounds__(512, 1)
         const int st = seq & 1;
         ok = mbar_wait_warp(&ld_empty[st], ((seq >> 1) & 1) ^ 1, abort_flag, 22);
         if (!ok) break;
-        if (lane == 0) FA_TRACE_AT(seq, 8);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int ql = lane * 4 + e;
           const int q = i * kBlockM + ql;
-          // rows past N: LSE = +inf makes P = 0 there, D = 0
+          // rows past N: LSE = +inf makes P = 0 there, D = 0.  D is kept
+          // negated so the second softmax phase forms dP - D with one add.
           sLSE[st * 128 + ql] = q < p.N ? p.lse[base + q] * log2e : INFINITY;
-          sDSUM[st * 128 + ql] = q < p.N ? p.dsum[base + q] : 0.f;
+          sDSUM[st * 128 + ql] = q < p.N ? -p.dsum[base + q] : 0.f;
         }
         mbar_arrive(&ld_full[st]);
         if (lane == 0) FA_TRACE_AT(seq, 9);
@@ -269,11 +268,8 @@ __global__ void __launch_bounds__(512, 1)
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_f16(BF16, 128, 128, false, false);  // S^T, dP^T
       constexpr uint32_t kIdTS = idesc_f16(BF16, 128, D, false, true);    // dV, dK (B MN-major)
-      // dQ: d = 128 computes dQ^T = K^T dS^T (M = d, N = queries), so the
-      // reduce-adds of a warp cover one contiguous row segment; d = 64 keeps
-      // dQ = dS K (M = queries, N = d).
-      constexpr uint32_t kIdDQ =
-          D == 128 ? idesc_f16(BF16, 128, 128, true, true) : idesc_f16(BF16, 128, D, true, true);
+      // dQ = dS K_j (M = queries, N = d): a TMEM lane holds one query row
+      constexpr uint32_t kIdDQ = idesc_f16(BF16, 128, D, true, true);
       const uint32_t aK = smem_addr(sK), aV = smem_addr(sV), aSlot = smem_addr(sSlot),
                      aDS = smem_addr(sDS);
       int nunit = 0, it = 0;
@@ -328,7 +324,6 @@ __global__ void __launch_bounds__(512, 1)
             ok = mbar_wait(dq_empty, (it - 1) & 1, abort_flag, 25);
             if (!ok) break;
           }
-          FA_TRACE_AT(it, 10);
           ok = mbar_wait(&slot_full[2], it & 1, abort_flag, 35);
           if (!ok) break;
           tc_fence_after();
@@ -356,6 +351,7 @@ __global__ void __launch_bounds__(512, 1)
             umma_ts(tmem + Lay::kColDV, tmem + Lay::kColS + (kk >> 2) * 64 + (kk & 3) * 8,
                     mnmaj(do_s, kk), kIdTS, (idx > 0 || kk > 0) ? 1u : 0u);
           umma_commit(&slot_empty[2]);  // dO_i: dP and dV done
+          FA_TRACE_AT(it, 13);
           // S^T of the next tile: its MMA runs after dV (in order), which has
           // read P^T out of these columns
           if (idx + 1 < w.ni) {
@@ -364,33 +360,41 @@ __global__ void __launch_bounds__(512, 1)
             tc_fence_after();
             issue_s(it + 1);
           }
-          // dK_j += dS^T Q_i once the second phase wrote dS^T
+          FA_TRACE_AT(it, 14);
+          // dQ and dK_j += dS^T Q_i once the second phase wrote dS^T
           ok = mbar_wait(ds_full, it & 1, abort_flag, 36);
           if (!ok) break;
           tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            umma_ss(tmem + Lay::kColDK, kmaj(aDS, kk), mnmaj(q_s, kk), kIdTS,
-                    (idx > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(&slot_empty[it & 1]);  // Q_i: S and dK done
-          if (D == 64 && it > 0) {
-            ok = mbar_wait(dq_empty, (it - 1) & 1, abort_flag, 25);
-            if (!ok) break;
-            tc_fence_after();
-          }
-          if constexpr (D == 128) {
-            // dQ^T = K_j^T dS^T: A = K_j read MN-major (d contiguous), B = dS^T
-            // read MN-major (queries contiguous)
+          FA_TRACE_AT(it, 8);
+          auto issue_dk = [&]() {
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
-              umma_ss(tmem + Lay::kColDQ, mnmaj(aK, kk), mnmaj(aDS, kk), kIdDQ, kk > 0);
-          } else {
-            // dQ = dS K_j: A = dS^T read MN-major, B = K_j MN-major
+              umma_ss(tmem + Lay::kColDK, kmaj(aDS, kk), mnmaj(q_s, kk), kIdTS,
+                      (idx > 0 || kk > 0) ? 1u : 0u);
+            umma_commit(&slot_empty[it & 1]);  // Q_i: S and dK done
+          };
+          // dQ = dS K_j: A = dS^T read MN-major (queries contiguous), B = K_j
+          // read MN-major (d contiguous)
+          auto issue_dq = [&]() {
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
               umma_ss(tmem + Lay::kColDQ, mnmaj(aDS, kk), mnmaj(aK, kk), kIdDQ, kk > 0);
+            umma_commit(dq_full);
+          };
+          if constexpr (D == 128) {
+            // dQ lives in the dP^T columns: issued before dK, so that the dQ
+            // warps release them for the next tile's dP^T while dK runs
+            issue_dq();
+            issue_dk();
+          } else {
+            issue_dk();
+            if (it > 0) {
+              ok = mbar_wait(dq_empty, (it - 1) & 1, abort_flag, 25);
+              if (!ok) break;
+              tc_fence_after();
+            }
+            issue_dq();
           }
-          umma_commit(dq_full);
           umma_commit(ds_empty);  // dK and dQ have read dS^T
           FA_TRACE_AT(it, 3);
           ++it;
@@ -409,7 +413,46 @@ __global__ void __launch_bounds__(512, 1)
     }
     __syncwarp();
   }
-  // warp 15 has no role
+#ifdef FA_TRACE
+  if (warp == 15 && lane == 0 && blockIdx.x == 0) {
+    // Trace builds only: observe when each tensor-core phase of CTA 0
+    // completes (waits only, never arrives; gives up quietly).
+    auto seen = [&](uint64_t* bar, uint32_t parity) {
+      const uint32_t a = smem_addr(bar);
+      const unsigned long long t0 = globaltimer_ns();
+      while (!mbar_try_wait(a, parity))
+        if (globaltimer_ns() - t0 > 20000000ull) return false;
+      return true;
+    };
+    int it = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      WorkItem wi;
+      if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
+      if (wi.idx < 0) continue;
+      const BwdUnit w = bwd_decode(wi.bh, wi.idx, p);
+      if (w.ni > 0) {
+        ok = seen(s_full, it & 1);
+        FA_TRACE_AT(it, 16);
+      }
+      for (int idx = 0; idx < w.ni && ok; ++idx) {
+        ok = ok && seen(dp_full, it & 1);
+        FA_TRACE_AT(it, 17);
+        ok = ok && seen(&slot_empty[2], it & 1);
+        FA_TRACE_AT(it, 18);
+        if (idx + 1 < w.ni) {
+          ok = ok && seen(s_full, (it + 1) & 1);
+          FA_TRACE_AT(it + 1, 16);
+        }
+        ok = ok && seen(&slot_empty[it & 1], (it >> 1) & 1);
+        FA_TRACE_AT(it, 19);
+        ok = ok && seen(dq_full, it & 1);
+        FA_TRACE_AT(it, 20);
+        ++it;
+      }
+    }
+  }
+#endif
   } else if (warp < 8) {
     regs_increase<kBwdSoftmaxRegs>();
     // ------------------------- P^T and dS^T: key row per thread, half the queries
@@ -447,7 +490,9 @@ __global__ void __launch_bounds__(512, 1)
         for (int cc = 0; cc < 2; ++cc) {
           const int c = half * 2 + cc;  // 32-query chunk
           uint32_t sr[32];
+          if (threadIdx.x == 0 && cc == 1) FA_TRACE_AT(it, 27);
           tmem_ld32(tS + c * 32, sr);
+          if (threadIdx.x == 0) FA_TRACE_AT(it, cc == 0 ? 10 : 24);
           uint32_t pp[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 4) {
@@ -468,7 +513,9 @@ __global__ void __launch_bounds__(512, 1)
           // half's
           tmem_st16(tS + half * 64 + (c & 1) * 16, pp);
         }
+        if (threadIdx.x == 0) FA_TRACE_AT(it, 25);
         tmem_st_wait();
+        if (threadIdx.x == 0) FA_TRACE_AT(it, 26);
         tc_fence_before();
         mbar_arrive(p_full);
         if (threadIdx.x == 0) FA_TRACE_AT(it, 15);
@@ -477,21 +524,28 @@ __global__ void __launch_bounds__(512, 1)
         if (ok && it > 0) ok = mbar_wait_warp(ds_empty, (it - 1) & 1, abort_flag, 31);
         if (!ok) break;
         tc_fence_after();
+        if (threadIdx.x == 0) FA_TRACE_AT(it, 11);
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           const int c = half * 2 + cc;
           uint32_t dr[32];
+          if (threadIdx.x == 0 && cc == 1) FA_TRACE_AT(it, 28);
           tmem_ld32(tDP + c * 32, dr);
+          if (threadIdx.x == 0) FA_TRACE_AT(it, cc == 0 ? 12 : 21);
           uint32_t dd[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 4) {
             const int q0 = c * 32 + e;
-            const float4 d4 = *reinterpret_cast<const float4*>(dsm + q0);
-            const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+            const float4 nd = *reinterpret_cast<const float4*>(dsm + q0);  // -D
+            // packed pairs: (dP - D) then P (dP - D)
+            const int b0 = cc * 32 + e;
+            const auto x01 = fadd2(f2pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])),
+                                   f2pack(nd.x, nd.y));
+            const auto x23 = fadd2(f2pack(__uint_as_float(dr[e + 2]), __uint_as_float(dr[e + 3])),
+                                   f2pack(nd.z, nd.w));
             float gv[4];
-#pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4)
-              gv[k4] = pv[cc * 32 + e + k4] * (__uint_as_float(dr[e + k4]) - dv4[k4]);
+            f2unpack(fmul2(f2pack(pv[b0], pv[b0 + 1]), x01), gv[0], gv[1]);
+            f2unpack(fmul2(f2pack(pv[b0 + 2], pv[b0 + 3]), x23), gv[2], gv[3]);
             dd[(e >> 1)] = pack2<BF16>(gv[0], gv[1]);
             dd[(e >> 1) + 1] = pack2<BF16>(gv[2], gv[3]);
           }
@@ -504,7 +558,9 @@ __global__ void __launch_bounds__(512, 1)
                          dd[4 * w4 + 3]);
           }
         }
+        if (threadIdx.x == 0) FA_TRACE_AT(it, 22);
         fence_proxy_async_smem();
+        if (threadIdx.x == 0) FA_TRACE_AT(it, 23);
         tc_fence_before();
         mbar_arrive(ds_full);
         mbar_arrive(&ld_empty[st]);
@@ -531,56 +587,44 @@ __global__ void __launch_bounds__(512, 1)
         if (!ok) break;
         tc_fence_after();
         if (threadIdx.x == 256) FA_TRACE_AT(it, 6);
-        if constexpr (D == 128) {
-          // Lane r holds column r of dQ_i for the 128 query rows (dQ^T).  Read
-          // it all, release the TMEM columns, then four rounds of 32 rows
-          // alternate between two 16 KB [32][128] fp32 staging buffers, each
-          // followed by one TMA reduce-add into the accumulator (the TMA path
-          // sustains more reduce bandwidth per SM than per-thread reds);
-          // staging a round overlaps the previous transfer.
+        // Lane r holds row r of dQ_i (one query, d contiguous).  Read it all,
+        // release the TMEM columns, then D / 32 rounds: each stages a
+        // [128][32] fp32 column block of the tile in one of two 16 KB buffers
+        // (128-byte rows whose 16-byte units are permuted by the row as the
+        // 128-byte TMA swizzle expects, so the vector stores of a warp hit
+        // distinct banks) and reduce-adds it into the accumulator with one TMA
+        // transfer (the TMA path sustains more reduce bandwidth per SM than
+        // per-thread reds); staging a round overlaps the previous transfer.
+        // Rows past N are clipped by the transfer.
+        {
           const bool leader = warp == 8 && lane == 0;
-          uint32_t v[128];
-          tmem_ld64x2(tmem + lane_off + Lay::kColDQ, v);
+          uint32_t v[D];
+          if constexpr (D == 128) tmem_ld64x2(tmem + lane_off + Lay::kColDQ, v);
+          else tmem_ld64(tmem + lane_off + Lay::kColDQ, v);
           tc_fence_before();
           mbar_arrive(dq_empty);
 #pragma unroll
-          for (int rd = 0; rd < 4; ++rd) {
-            float* stg = reinterpret_cast<float*>(sSTG + (stage_round & 1) * 16384);
+          for (int rd = 0; rd < D / 32; ++rd) {
+            uint8_t* stg = sSTG + (stage_round & 1) * 16384;
             if (stage_round >= 2) {
               // the transfer that used this buffer two rounds ago must have
               // read it
               if (leader) bulk_wait_read_one();
               named_bar_sync(1, 128);
             }
+            const uint32_t row = smem_addr(stg) + r * 128;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) stg[e * D + r] = __uint_as_float(v[rd * 32 + e]);
+            for (int u = 0; u < 8; ++u)
+              st_shared_v4(row + ((u ^ (r & 7)) << 4), v[rd * 32 + 4 * u], v[rd * 32 + 4 * u + 1],
+                           v[rd * 32 + 4 * u + 2], v[rd * 32 + 4 * u + 3]);
             fence_proxy_async_smem();
             named_bar_sync(1, 128);
             if (leader) {
-              tma_reduce_add_3d(&tmdq, stg, 0, i * kBlockM + rd * 32, w.bh);
+              tma_reduce_add_3d(&tmdq, stg, rd * 32, i * kBlockM, w.bh);
               bulk_commit_group();
             }
             ++stage_round;
           }
-        } else {
-          const int row = i * kBlockM + r;
-          float* dst = p.dq_acc + (base + (row < p.N ? row : 0)) * D;
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t v[32];
-            tmem_ld32(tmem + lane_off + Lay::kColDQ + c * 32, v);
-            if (row < p.N) {
-#pragma unroll
-              for (int q4 = 0; q4 < 8; ++q4)
-                red_add_v4(dst + c * 32 + q4 * 4, __uint_as_float(v[4 * q4]),
-                           __uint_as_float(v[4 * q4 + 1]), __uint_as_float(v[4 * q4 + 2]),
-                           __uint_as_float(v[4 * q4 + 3]));
-            }
-          }
-        }
-        if (D == 64) {
-          tc_fence_before();
-          mbar_arrive(dq_empty);
         }
         if (threadIdx.x == 256) FA_TRACE_AT(it, 7);
         ++it;
@@ -629,7 +673,7 @@ __global__ void __launch_bounds__(512, 1)
       ++nunit;
     }
     // every reduce-add issued must have completed before the kernel ends
-    if (D == 128 && warp == 8 && lane == 0) bulk_wait_all();
+    if (warp == 8 && lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();

@@ -27,15 +27,15 @@ __device__ __forceinline__ void record_error(unsigned code, unsigned site) {
 }
 
 // Optional device timeline (build with -DFA_TRACE): SM clock stamps of
-// pipeline events of CTA 0, slot = iteration * 16 + event.  Compiled out by
+// pipeline events of CTA 0, slot = iteration * 32 + event.  Compiled out by
 // default.
 #ifdef FA_TRACE
 constexpr int kTraceSlots = 1 << 16;
 __device__ unsigned long long g_trace[kTraceSlots];
 #define FA_TRACE_AT(it, ev)                                                        \
   do {                                                                            \
-    if (blockIdx.x == 0 && (it) < (kTraceSlots / 16))                             \
-      g_trace[(it) * 16 + (ev)] = static_cast<unsigned long long>(clock64());     \
+    if (blockIdx.x == 0 && (it) < (kTraceSlots / 32))                             \
+      g_trace[(it) * 32 + (ev)] = static_cast<unsigned long long>(clock64());     \
   } while (0)
 #else
 #define FA_TRACE_AT(it, ev) \
