@@ -270,20 +270,19 @@ __global__ void __launch_bounds__(512, 1)
       constexpr uint32_t kIdTS = idesc_f16(BF16, 128, D, false, true);    // dV, dK (B MN-major)
       // dQ = dS K_j (M = queries, N = d): a TMEM lane holds one query row
       constexpr uint32_t kIdDQ = idesc_f16(BF16, 128, D, true, true);
-      const uint32_t aK = smem_addr(sK), aV = smem_addr(sV), aSlot = smem_addr(sSlot),
-                     aDS = smem_addr(sDS);
+      // Low descriptor words of every operand tile, K-major (_k) or MN-major
+      // (_m) view; the grouped MMAs derive the K steps from them.
+      const uint32_t aSlot = smem_addr(sSlot);
+      const uint32_t lK_k = sdesc_lo(smem_addr(sK), false), lK_m = sdesc_lo(smem_addr(sK), true);
+      const uint32_t lV_k = sdesc_lo(smem_addr(sV), false);
+      const uint32_t lQ0_k = sdesc_lo(aSlot, false), lQ0_m = sdesc_lo(aSlot, true);
+      const uint32_t lQ1_k = sdesc_lo(aSlot + Lay::kTileBytes, false),
+                     lQ1_m = sdesc_lo(aSlot + Lay::kTileBytes, true);
+      const uint32_t lO_k = sdesc_lo(aSlot + 2 * Lay::kTileBytes, false),
+                     lO_m = sdesc_lo(aSlot + 2 * Lay::kTileBytes, true);
+      const uint32_t lS_k = sdesc_lo(smem_addr(sDS), false), lS_m = sdesc_lo(smem_addr(sDS), true);
       int nunit = 0, it = 0;
       bool ok = true;
-      // K-major operands (A and B): 16-element steps walk 32 bytes inside a
-      // 64-column panel, panels are 16 KB apart.
-      auto kmaj = [](uint32_t base, int kk) {
-        return sdesc_sw128(base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-      };
-      // MN-major operands: 16 rows of K = 2048 bytes; 64-column MN panels
-      // 16 KB apart (leading byte offset).
-      auto mnmaj = [](uint32_t base, int kk) {
-        return sdesc_sw128(base + kk * 2048, 16384, 1024);
-      };
       for (int k = 0; ok; ++k) {
         WorkItem wi;
         if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
@@ -303,10 +302,8 @@ __global__ void __launch_bounds__(512, 1)
         // tensor core does dK(i) and dQ(i), and its second phase (from dP)
         // while it does dV(i+1).
         auto issue_s = [&](int t) {  // S^T(t) = K_j Q_t^T, Q_t in slot t & 1
-          const uint32_t q_s = aSlot + (t & 1) * Lay::kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            umma_ss(tmem + Lay::kColS, kmaj(aK, kk), kmaj(q_s, kk), kIdS, kk > 0);
+          umma_ss_group<D / 16, false, false>(tmem + Lay::kColS, lK_k, (t & 1) ? lQ1_k : lQ0_k,
+                                              kIdS, 0u);
           umma_commit(s_full);
         };
         if (w.ni > 0) {
@@ -317,8 +314,6 @@ __global__ void __launch_bounds__(512, 1)
         }
         for (int idx = 0; idx < w.ni && ok; ++idx) {
           FA_TRACE_AT(it, 0);
-          const uint32_t q_s = aSlot + (it & 1) * Lay::kTileBytes;
-          const uint32_t do_s = aSlot + 2 * Lay::kTileBytes;
           // d = 128: dQ^T of the previous tile lives in the dP^T columns
           if (D == 128 && it > 0) {
             ok = mbar_wait(dq_empty, (it - 1) & 1, abort_flag, 25);
@@ -329,9 +324,7 @@ __global__ void __launch_bounds__(512, 1)
           tc_fence_after();
           FA_TRACE_AT(it, 1);
           // dP^T = V_j dO_i^T
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            umma_ss(tmem + Lay::kColDP, kmaj(aV, kk), kmaj(do_s, kk), kIdS, kk > 0);
+          umma_ss_group<D / 16, false, false>(tmem + Lay::kColDP, lV_k, lO_k, kIdS, 0u);
           umma_commit(dp_full);
           // dV_j += P^T dO_i once the first softmax phase wrote P^T
           ok = mbar_wait(p_full, it & 1, abort_flag, 26);
@@ -346,10 +339,8 @@ __global__ void __launch_bounds__(512, 1)
           }
           // (A = P^T in TMEM, 16 queries = 8 columns; queries 64..127 sit 64
           // columns further, in the second half's S^T columns)
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            umma_ts(tmem + Lay::kColDV, tmem + Lay::kColS + (kk >> 2) * 64 + (kk & 3) * 8,
-                    mnmaj(do_s, kk), kIdTS, (idx > 0 || kk > 0) ? 1u : 0u);
+          umma_ts_group8<true, true>(tmem + Lay::kColDV, tmem + Lay::kColS, lO_m, kIdTS,
+                                     idx > 0 ? 1u : 0u);
           umma_commit(&slot_empty[2]);  // dO_i: dP and dV done
           FA_TRACE_AT(it, 13);
           // S^T of the next tile: its MMA runs after dV (in order), which has
@@ -366,19 +357,15 @@ __global__ void __launch_bounds__(512, 1)
           if (!ok) break;
           tc_fence_after();
           FA_TRACE_AT(it, 8);
-          auto issue_dk = [&]() {
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              umma_ss(tmem + Lay::kColDK, kmaj(aDS, kk), mnmaj(q_s, kk), kIdTS,
-                      (idx > 0 || kk > 0) ? 1u : 0u);
+          auto issue_dk = [&]() {  // A = dS^T K-major, B = Q_i MN-major
+            umma_ss_group<8, false, true>(tmem + Lay::kColDK, lS_k, (it & 1) ? lQ1_m : lQ0_m,
+                                          kIdTS, idx > 0 ? 1u : 0u);
             umma_commit(&slot_empty[it & 1]);  // Q_i: S and dK done
           };
           // dQ = dS K_j: A = dS^T read MN-major (queries contiguous), B = K_j
           // read MN-major (d contiguous)
           auto issue_dq = [&]() {
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              umma_ss(tmem + Lay::kColDQ, mnmaj(aDS, kk), mnmaj(aK, kk), kIdDQ, kk > 0);
+            umma_ss_group<8, true, true>(tmem + Lay::kColDQ, lS_m, lK_m, kIdDQ, 0u);
             umma_commit(dq_full);
           };
           if constexpr (D == 128) {

@@ -205,34 +205,21 @@ __global__ void __launch_bounds__(384, 1)
       int kv_seq = 0;
       bool ok = true;
 
-      // Shared-memory descriptors of the fixed buffers, built once; an MMA
-      // moves them with one add.
-      const uint64_t dQ0 = sdesc_sw128(sq_addr, 16, 1024);                  // K-major
-      const uint64_t dK0 = sdesc_sw128(skv_addr, 16, 1024);                 // K-major
-      const uint64_t dV0 = sdesc_sw128(skv_addr, Lay::kPanelBytes, 1024);   // MN-major
-      // S_t = Q_t K^T: A = Q tile (K-major), B = K tile (K-major); the
-      // 16-element K steps walk 32 bytes inside a 128-byte swizzle panel.
+      // Low descriptor words of the Q tiles and of the K/V ring, K-major and
+      // MN-major (V); the grouped MMAs derive the K steps from them.
+      constexpr uint32_t kTileLo = Lay::kTileBytes >> 4;
+      const uint32_t lQ_k = sdesc_lo(sq_addr, false);
+      const uint32_t lKV_k = sdesc_lo(skv_addr, false), lKV_m = sdesc_lo(skv_addr, true);
+      // S_t = Q_t K^T: A = Q tile (K-major), B = K tile (K-major).
       auto issue_s = [&](int t, int kslot) {
-        const uint32_t d_tmem = tmem + t * 128;
-        const uint64_t qa = sdesc_add(dQ0, t * Lay::kTileBytes);
-        const uint64_t kb = sdesc_add(dK0, kslot * Lay::kTileBytes);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * Lay::kPanelBytes + (kk & 3) * 32;
-          umma_ss(d_tmem, sdesc_add(qa, off), sdesc_add(kb, off), kIdescQK, kk > 0 ? 1u : 0u);
-        }
+        umma_ss_group<D / 16, false, false>(tmem + t * 128, lQ_k + t * kTileLo,
+                                            lKV_k + kslot * kTileLo, kIdescQK, 0u);
       };
-      // O_t += P_t V: A = P (16-bit, TMEM, over S_t), B = V tile read
-      // MN-major (d contiguous): 16 keys = 2048 bytes, 64-column panels
-      // 16 KB apart.
+      // O_t += P_t V: A = P (16-bit, TMEM, over S_t, 8 columns per 16 keys),
+      // B = V tile read MN-major (d contiguous).
       auto issue_pv = [&](int t, int vslot, bool acc) {
-        const uint32_t d_tmem = tmem + Lay::kColO + t * D;
-        const uint64_t vb = sdesc_add(dV0, vslot * Lay::kTileBytes);
-#pragma unroll
-        for (int kk = 0; kk < kBlockN / 16; ++kk) {
-          umma_ts(d_tmem, tmem + t * 128 + kk * 8, sdesc_add(vb, kk * 2048), kIdescPV,
-                  (acc || kk > 0) ? 1u : 0u);
-        }
+        umma_ts_group8<true, false>(tmem + Lay::kColO + t * D, tmem + t * 128,
+                                    lKV_m + vslot * kTileLo, kIdescPV, acc ? 1u : 0u);
       };
 
       for (int k = 0; ok; ++k) {

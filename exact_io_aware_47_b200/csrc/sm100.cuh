@@ -279,6 +279,108 @@ __host__ __device__ constexpr uint32_t idesc_f16(bool bf16, int M, int N, bool a
 }
 
 // ---------------------------------------------------------------------------
+// Grouped MMAs: a whole K = 64 or K = 128 contraction (4 or 8 tcgen05.mma of
+// K = 16) into one accumulator from one asm statement.  Every descriptor of
+// the group is the 128-byte-swizzled descriptor of its first step plus an
+// immediate offset on the start-address field, so a step costs one 32-bit add
+// per shared operand; the accumulate predicate is set once.  Operands are
+// given by the low descriptor word (start address >> 4 | leading byte offset
+// >> 4 << 16, see sdesc_lo); the high word (stride byte offset 1024, sm_100
+// version bit, 128-byte swizzle) is the same for every operand here.  The
+// start-address field never carries into the next field: shared addresses
+// stay below 256 KB.
+// ---------------------------------------------------------------------------
+constexpr uint32_t kSdescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+
+// K-major operand (rows of 128 bytes, 64-element panels 16 KB apart): LBO 16.
+// MN-major operand (64-element MN panels 16 KB apart): LBO 16384.
+__device__ __forceinline__ uint32_t sdesc_lo(uint32_t saddr, bool mn_major) {
+  return ((saddr >> 4) & 0x3FFFu) | ((mn_major ? (16384u >> 4) : 1u) << 16);
+}
+
+// Start-address step (16-byte units) of K-step kk (16 elements of 16 bits):
+// K-major walks 32 bytes inside a 64-element panel, then the next panel;
+// MN-major walks 16 rows of 128 bytes.
+__host__ __device__ constexpr uint32_t sw128_step(bool mn_major, int kk) {
+  return mn_major ? static_cast<uint32_t>(kk) * 128u
+                  : static_cast<uint32_t>(kk >> 2) * 1024u + static_cast<uint32_t>(kk & 3) * 2u;
+}
+
+#define FA_MMA_PROLOGUE                                                        \
+  "{\n\t.reg .pred p, t;\n\t.reg .b32 h, a, b;\n\t.reg .b64 da, db;\n\t"       \
+  "setp.ne.b32 p, %4, 0;\n\tsetp.eq.b32 t, %4, %4;\n\tmov.b32 h, %5;\n\t"
+#define FA_MMA_SS_FIRST                                                        \
+  "mov.b64 da, {%1, h};\n\tmov.b64 db, {%2, h};\n\t"                           \
+  "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p;\n\t"
+#define FA_MMA_SS_STEP(ao, bo)                                                 \
+  "add.u32 a, %1, %" #ao ";\n\tadd.u32 b, %2, %" #bo ";\n\t"                   \
+  "mov.b64 da, {a, h};\n\tmov.b64 db, {b, h};\n\t"                             \
+  "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, t;\n\t"
+#define FA_MMA_TS_FIRST                                                        \
+  "mov.b64 db, {%2, h};\n\t"                                                   \
+  "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %3, p;\n\t"
+#define FA_MMA_TS_STEP(ao, bo)                                                 \
+  "add.u32 a, %1, %" #ao ";\n\tadd.u32 b, %2, %" #bo ";\n\t"                   \
+  "mov.b64 db, {b, h};\n\t"                                                    \
+  "tcgen05.mma.cta_group::1.kind::f16 [%0], [a], db, %3, t;\n\t"
+
+// D (+)= A B over K = 16 * NK (NK = 4 or 8), A and B in shared memory.
+// accumulate = 0 overwrites D with the first step.
+template <int NK, bool A_MN, bool B_MN>
+__device__ __forceinline__ void umma_ss_group(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
+                                              uint32_t idesc, uint32_t accumulate) {
+  static_assert(NK == 4 || NK == 8, "group of 4 or 8 steps");
+  if constexpr (NK == 8) {
+    asm volatile(FA_MMA_PROLOGUE FA_MMA_SS_FIRST FA_MMA_SS_STEP(6, 13) FA_MMA_SS_STEP(7, 14)
+                     FA_MMA_SS_STEP(8, 15) FA_MMA_SS_STEP(9, 16) FA_MMA_SS_STEP(10, 17)
+                         FA_MMA_SS_STEP(11, 18) FA_MMA_SS_STEP(12, 19) "}" ::"r"(d_tmem),
+                 "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accumulate), "n"(kSdescHi),
+                 "n"(sw128_step(A_MN, 1)), "n"(sw128_step(A_MN, 2)), "n"(sw128_step(A_MN, 3)),
+                 "n"(sw128_step(A_MN, 4)), "n"(sw128_step(A_MN, 5)), "n"(sw128_step(A_MN, 6)),
+                 "n"(sw128_step(A_MN, 7)), "n"(sw128_step(B_MN, 1)), "n"(sw128_step(B_MN, 2)),
+                 "n"(sw128_step(B_MN, 3)), "n"(sw128_step(B_MN, 4)), "n"(sw128_step(B_MN, 5)),
+                 "n"(sw128_step(B_MN, 6)), "n"(sw128_step(B_MN, 7))
+                 : "memory");
+  } else {
+    asm volatile(FA_MMA_PROLOGUE FA_MMA_SS_FIRST FA_MMA_SS_STEP(6, 9) FA_MMA_SS_STEP(7, 10)
+                     FA_MMA_SS_STEP(8, 11) "}" ::"r"(d_tmem),
+                 "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accumulate), "n"(kSdescHi),
+                 "n"(sw128_step(A_MN, 1)), "n"(sw128_step(A_MN, 2)), "n"(sw128_step(A_MN, 3)),
+                 "n"(sw128_step(B_MN, 1)), "n"(sw128_step(B_MN, 2)), "n"(sw128_step(B_MN, 3))
+                 : "memory");
+  }
+}
+
+// TMEM column step of K-step kk (16 elements of 16 bits = 8 columns): either
+// contiguous, or split so that steps 4..7 sit 64 columns after steps 0..3.
+__host__ __device__ constexpr uint32_t tmem_step(bool split, int kk) {
+  return split ? static_cast<uint32_t>(kk >> 2) * 64u + static_cast<uint32_t>(kk & 3) * 8u
+               : static_cast<uint32_t>(kk) * 8u;
+}
+
+// D (+)= A B over K = 128, A in TMEM (16-bit elements packed in pairs, laid
+// out as tmem_step says), B in shared memory.
+template <bool B_MN, bool A_SPLIT>
+__device__ __forceinline__ void umma_ts_group8(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
+                                               uint32_t idesc, uint32_t accumulate) {
+  asm volatile(FA_MMA_PROLOGUE FA_MMA_TS_FIRST FA_MMA_TS_STEP(6, 13) FA_MMA_TS_STEP(7, 14)
+                   FA_MMA_TS_STEP(8, 15) FA_MMA_TS_STEP(9, 16) FA_MMA_TS_STEP(10, 17)
+                       FA_MMA_TS_STEP(11, 18) FA_MMA_TS_STEP(12, 19) "}" ::"r"(d_tmem),
+               "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(accumulate), "n"(kSdescHi),
+               "n"(tmem_step(A_SPLIT, 1)), "n"(tmem_step(A_SPLIT, 2)), "n"(tmem_step(A_SPLIT, 3)),
+               "n"(tmem_step(A_SPLIT, 4)), "n"(tmem_step(A_SPLIT, 5)), "n"(tmem_step(A_SPLIT, 6)),
+               "n"(tmem_step(A_SPLIT, 7)), "n"(sw128_step(B_MN, 1)), "n"(sw128_step(B_MN, 2)),
+               "n"(sw128_step(B_MN, 3)), "n"(sw128_step(B_MN, 4)), "n"(sw128_step(B_MN, 5)),
+               "n"(sw128_step(B_MN, 6)), "n"(sw128_step(B_MN, 7))
+               : "memory");
+}
+#undef FA_MMA_PROLOGUE
+#undef FA_MMA_SS_FIRST
+#undef FA_MMA_SS_STEP
+#undef FA_MMA_TS_FIRST
+#undef FA_MMA_TS_STEP
+
+// ---------------------------------------------------------------------------
 // TMEM <-> registers, 32 data-path lanes x 32 bit, 32 consecutive columns.
 // The warp's lane quarter is fixed by (warp id % 4); taddr carries it.
 // tmem_ld32 waits for its own load inside the same asm statement, so the
