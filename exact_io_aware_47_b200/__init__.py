@@ -5,10 +5,16 @@
     o, lse = forward(q, k, v, causal=True)
     dq, dk, dv = backward(q, k, v, o, lse, do, causal=True)
 
+Packed variable-length batches ([H, T, d], sequence b in rows
+cu_seqlens[b] .. cu_seqlens[b + 1] - 1): ``forward_varlen`` /
+``backward_varlen``.
+
 The CUDA library is loaded on first use; a missing library raises instead of
 falling back to anything else.
 """
 
-from .attention import backward, device_status, forward, workspace_bytes
+from .attention import (backward, backward_varlen, device_status, forward, forward_varlen,
+                        workspace_bytes)
 
-__all__ = ["forward", "backward", "workspace_bytes", "device_status"]
+__all__ = ["forward", "backward", "forward_varlen", "backward_varlen", "workspace_bytes",
+           "device_status"]

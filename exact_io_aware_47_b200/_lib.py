@@ -39,6 +39,9 @@ SIGNATURES = {
     "fa_bwd_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
                             _I, _I, _I, _I, _F, _I, _VP, _I, _VP]),
     "fa_bwd_noalloc_max_bytes": (_SZ, []),
+    "fa_fwd_varlen": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _I, _VP]),
+    "fa_bwd_varlen": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP,
+                           _I, _I, _I, _I, _I, _F, _I, _I, _VP]),
     "fa_device_status": (_I, [_VP, ctypes.POINTER(ctypes.c_uint32)]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_version": (_I, []),
@@ -115,6 +118,18 @@ def fa_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal,
                    stream):
     return load().fa_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal,
                                  seqlens, dtype, stream)
+
+
+def fa_fwd_varlen(q, k, v, o, lse, cu_seqlens, B, H, T, max_seqlen, d, scale, causal, dtype,
+                  stream):
+    return load().fa_fwd_varlen(q, k, v, o, lse, cu_seqlens, B, H, T, max_seqlen, d, scale, causal,
+                                dtype, stream)
+
+
+def fa_bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, cu_seqlens, B, H,
+                  T, max_seqlen, d, scale, causal, dtype, stream):
+    return load().fa_bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes,
+                                cu_seqlens, B, H, T, max_seqlen, d, scale, causal, dtype, stream)
 
 
 def fa_bwd_noalloc_max_bytes():

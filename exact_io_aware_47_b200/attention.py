@@ -1,9 +1,11 @@
 """torch-facing calls of the CUDA library: allocate outputs, pass pointers.
 
-``forward`` and ``backward`` validate tensor properties that ctypes cannot
-see (device, dtype, contiguity, shapes), allocate the outputs and the
-backward workspace with torch, and call ``fa_fwd`` / ``fa_bwd`` on the
-current CUDA stream.  No arithmetic of the method happens here.
+``forward`` and ``backward`` ([B, H, N, d]) and ``forward_varlen`` /
+``backward_varlen`` (packed [H, T, d] with cu_seqlens) validate tensor
+properties that ctypes cannot see (device, dtype, contiguity, shapes),
+allocate the outputs and the backward workspace with torch, and call the
+library on the current CUDA stream.  No arithmetic of the method happens
+here.
 """
 
 import math
@@ -100,6 +102,65 @@ def backward(q, k, v, o, lse, do, scale=None, causal=False, seqlens=None, worksp
                          B, H, N, d, scale, int(bool(causal)), sl_ptr, _DTYPES[q.dtype],
                          _stream_handle(dev))
     _lib.check("fa_bwd", st)
+    return dq, dk, dv
+
+
+def _cu_seqlens_arg(cu_seqlens, T, device):
+    cu = cu_seqlens
+    if not (torch.is_tensor(cu) and cu.is_cuda and cu.dtype == torch.int32 and cu.is_contiguous()):
+        cu = torch.as_tensor(cu_seqlens, dtype=torch.int32).to(device).contiguous()
+    if cu.dim() != 1 or cu.numel() < 2:
+        raise ValueError("cu_seqlens must be [B + 1] row offsets")
+    return cu, cu.numel() - 1
+
+
+def forward_varlen(q, k, v, cu_seqlens, max_seqlen, scale=None, causal=False, out=None, lse=None):
+    """O, LSE of packed sequences on the GPU: q, k, v [H, T, d] bf16/fp16,
+    sequence b in rows cu_seqlens[b] .. cu_seqlens[b + 1] - 1 of every head."""
+    if q.dim() != 3:
+        raise ValueError("q must be [H, T, d]")
+    H, T, d = q.shape
+    dev = q.device
+    if q.dtype not in _DTYPES:
+        raise ValueError("dtype must be bfloat16 or float16")
+    _check_inputs({"q": q, "k": k, "v": v}, (H, T, d), q.dtype, dev)
+    cu, B = _cu_seqlens_arg(cu_seqlens, T, dev)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((H, T), dtype=torch.float32, device=dev) if lse is None else lse
+    _check_inputs({"out": out}, (H, T, d), q.dtype, dev)
+    _check_inputs({"lse": lse}, (H, T), torch.float32, dev)
+    with torch.cuda.device(dev):
+        st = _lib.fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                lse.data_ptr(), cu.data_ptr(), B, H, T, int(max_seqlen), d, scale,
+                                int(bool(causal)), _DTYPES[q.dtype], _stream_handle(dev))
+    _lib.check("fa_fwd_varlen", st)
+    return out, lse
+
+
+def backward_varlen(q, k, v, o, lse, do, cu_seqlens, max_seqlen, scale=None, causal=False,
+                    workspace=None, dq=None, dk=None, dv=None):
+    """dQ, dK, dV of the loss <dO, O> for packed sequences ([H, T, d])."""
+    H, T, d = q.shape
+    dev = q.device
+    _check_inputs({"q": q, "k": k, "v": v, "o": o, "do": do}, (H, T, d), q.dtype, dev)
+    _check_inputs({"lse": lse}, (H, T), torch.float32, dev)
+    cu, B = _cu_seqlens_arg(cu_seqlens, T, dev)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check_inputs({"dq": dq, "dk": dk, "dv": dv}, (H, T, d), q.dtype, dev)
+    if workspace is None:
+        workspace = torch.empty(workspace_bytes(1, H, T, d), dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        st = _lib.fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                dv.data_ptr(), workspace.data_ptr(),
+                                workspace.numel() * workspace.element_size(), cu.data_ptr(), B, H,
+                                T, int(max_seqlen), d, scale, int(bool(causal)), _DTYPES[q.dtype],
+                                _stream_handle(dev))
+    _lib.check("fa_bwd_varlen", st)
     return dq, dk, dv
 
 

@@ -116,40 +116,81 @@ size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 using namespace fa;
 
-extern "C" int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                      int H, int N, int d, float scale, int causal, const int32_t* seqlens,
-                      int dtype, void* stream) {
-  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
-  int st = check_common(B, H, N, d, scale, dtype);
-  if (st != FA_OK) return st;
+namespace fa {
+namespace {
+
+// Forward for both layouts (cu_seqlens == nullptr: [B, H, N, d]; else packed
+// [H, T = N, d]); arguments already checked except the pointers' alignment.
+int fwd_core(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+             int N, int d, float scale, int causal, const int32_t* seqlens,
+             const int32_t* cu_seqlens, int max_seqlen, int dtype, void* stream) {
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
-      (seqlens && (reinterpret_cast<uintptr_t>(seqlens) & 3u)))
+      (seqlens && (reinterpret_cast<uintptr_t>(seqlens) & 3u)) ||
+      (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)))
     return FA_ERR_ALIGNMENT;
   DeviceInfo di;
-  st = current_device_info(&di);
+  const int st = current_device_info(&di);
   if (st != FA_OK) return st;
 
   CUtensorMap tq, tk, tv;
-  const int BH = B * H;
-  if (make_map(&tq, q, BH, N, d, dtype) != FA_OK || make_map(&tk, k, BH, N, d, dtype) != FA_OK ||
-      make_map(&tv, v, BH, N, d, dtype) != FA_OK)
+  const int blocks = cu_seqlens ? H : B * H;  // row blocks of N rows
+  if (make_map(&tq, q, blocks, N, d, dtype) != FA_OK ||
+      make_map(&tk, k, blocks, N, d, dtype) != FA_OK ||
+      make_map(&tv, v, blocks, N, d, dtype) != FA_OK)
     return FA_ERR_CUDA;
 
   FwdParams p;
   p.o = o;
   p.lse = lse;
   p.seqlens = seqlens;
+  p.cu_seqlens = cu_seqlens;
+  p.max_seqlen = cu_seqlens ? max_seqlen : N;
   p.B = B;
   p.H = H;
   p.N = N;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.causal = causal ? 1 : 0;
-  p.n_qtiles = (N + kBlockM - 1) / kBlockM;
+  p.n_qtiles = (p.max_seqlen + kBlockM - 1) / kBlockM;
   p.n_pairs = (p.n_qtiles + 1) / 2;
-  p.n_units = BH * ((p.n_pairs + 1) / 2);
+  p.n_units = B * H * ((p.n_pairs + 1) / 2);
   const cudaError_t e =
       launch_fwd(d, dtype == FA_BF16, tq, tk, tv, p, di.num_sms, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// Packed-layout argument checks shared by the forward and the backward: the
+// [H, T, d] tensors as in check_common (B = 1, N = T), B >= 1 sequences, and
+// the work-unit count B * H * ceil(max_seqlen / 128) within int range.
+int check_varlen(const int32_t* cu_seqlens, int B, int H, int T, int max_seqlen, int d,
+                 float scale, int dtype) {
+  if (!cu_seqlens || B < 1 || max_seqlen < 1) return FA_ERR_INVALID_ARG;
+  const int st = check_common(1, H, T, d, scale, dtype);
+  if (st != FA_OK) return st;
+  const long long tiles = (static_cast<long long>(max_seqlen < T ? max_seqlen : T) + 127) / 128;
+  if (static_cast<long long>(B) * H * tiles >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+}  // namespace
+}  // namespace fa
+
+extern "C" int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                      int H, int N, int d, float scale, int causal, const int32_t* seqlens,
+                      int dtype, void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  const int st = check_common(B, H, N, d, scale, dtype);
+  if (st != FA_OK) return st;
+  return fwd_core(q, k, v, o, lse, B, H, N, d, scale, causal, seqlens, nullptr, 0, dtype, stream);
+}
+
+extern "C" int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                             const int32_t* cu_seqlens, int B, int H, int T, int max_seqlen,
+                             int d, float scale, int causal, int dtype, void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  const int st = check_varlen(cu_seqlens, B, H, T, max_seqlen, d, scale, dtype);
+  if (st != FA_OK) return st;
+  return fwd_core(q, k, v, o, lse, B, H, T, d, scale, causal, nullptr, cu_seqlens,
+                  max_seqlen < T ? max_seqlen : T, dtype, stream);
 }
 
 extern "C" size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
@@ -161,29 +202,37 @@ extern "C" size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
 namespace fa {
 namespace {
 
-// Checks shared by the backward stages; fills the workspace carving.
+// Checks shared by the backward stages; fills the workspace carving.  With
+// cu_seqlens the tensors are packed [H, T = N, d] (max_seqlen already clamped
+// to T) and the workspace is that of fa_bwd_workspace_size(1, H, T, d).
 int bwd_common(void* workspace, size_t workspace_bytes, int B, int H, int N, int d, float scale,
-               int dtype, const int32_t* seqlens, BwdParams* p, DeviceInfo* di) {
-  int st = check_common(B, H, N, d, scale, dtype);
+               int dtype, const int32_t* seqlens, BwdParams* p, DeviceInfo* di,
+               const int32_t* cu_seqlens = nullptr, int max_seqlen = 0) {
+  int st = cu_seqlens ? check_varlen(cu_seqlens, B, H, N, max_seqlen, d, scale, dtype)
+                      : check_common(B, H, N, d, scale, dtype);
   if (st != FA_OK) return st;
-  if (seqlens && (reinterpret_cast<uintptr_t>(seqlens) & 3u)) return FA_ERR_ALIGNMENT;
-  const size_t need = fa_bwd_workspace_size(B, H, N, d);
+  if ((seqlens && (reinterpret_cast<uintptr_t>(seqlens) & 3u)) ||
+      (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)))
+    return FA_ERR_ALIGNMENT;
+  const size_t need = cu_seqlens ? fa_bwd_workspace_size(1, H, N, d) : fa_bwd_workspace_size(B, H, N, d);
   if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FA_ERR_ALIGNMENT;
   st = current_device_info(di);
   if (st != FA_OK) return st;
-  const size_t rows = static_cast<size_t>(B) * H * N;
+  const size_t rows = static_cast<size_t>(cu_seqlens ? 1 : B) * H * N;
   std::memset(p, 0, sizeof(*p));
   p->dsum = static_cast<float*>(workspace);
   p->dq_acc =
       reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round256(rows * sizeof(float)));
   p->seqlens = seqlens;
+  p->cu_seqlens = cu_seqlens;
+  p->max_seqlen = cu_seqlens ? max_seqlen : N;
   p->B = B;
   p->H = H;
   p->N = N;
   p->scale = scale;
   p->scale_log2 = scale * 1.4426950408889634f;
-  p->n_ktiles = (N + kBlockN - 1) / kBlockN;
+  p->n_ktiles = (p->max_seqlen + kBlockN - 1) / kBlockN;
   p->n_units = B * H * ((p->n_ktiles + 1) / 2);
   return FA_OK;
 }
@@ -273,6 +322,43 @@ extern "C" int fa_bwd(const void* q, const void* k, const void* v, const void* o
                    causal, seqlens, dtype, stream);
   if (st != FA_OK) return st;
   return fa_bwd_postprocess(workspace, workspace_bytes, dq, B, H, N, d, scale, dtype, stream);
+}
+
+extern "C" int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
+                             const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                             void* workspace, size_t workspace_bytes, const int32_t* cu_seqlens,
+                             int B, int H, int T, int max_seqlen, int d, float scale, int causal,
+                             int dtype, void* stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_ALIGNMENT;
+  BwdParams p;
+  DeviceInfo di;
+  int st = bwd_common(workspace, workspace_bytes, B, H, T, d, scale, dtype, nullptr, &p, &di,
+                      cu_seqlens, max_seqlen < T ? max_seqlen : T);
+  if (st != FA_OK) return st;
+  CUtensorMap tq, tk, tv, tdo, tdq;
+  if (make_map(&tq, q, H, T, d, dtype) != FA_OK || make_map(&tk, k, H, T, d, dtype) != FA_OK ||
+      make_map(&tv, v, H, T, d, dtype) != FA_OK || make_map(&tdo, dout, H, T, d, dtype) != FA_OK ||
+      make_map_acc(&tdq, p.dq_acc, H, T, d) != FA_OK)
+    return FA_ERR_CUDA;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.o = o;
+  p.dout = dout;
+  p.lse = lse;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.causal = causal ? 1 : 0;
+  const bool bf16 = dtype == FA_BF16;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (launch_bwd_pre(d, bf16, p, di.num_sms, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (launch_bwd_main(d, bf16, tq, tk, tv, tdo, tdq, p, di.num_sms, s) != cudaSuccess)
+    return FA_ERR_CUDA;
+  return launch_bwd_post(d, bf16, p, di.num_sms, s) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------------------

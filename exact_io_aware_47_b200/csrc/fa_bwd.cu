@@ -73,6 +73,8 @@ struct BwdLayout {
 
 struct BwdUnit {
   int bh, j, L, i0, ni;
+  int z, row0, rows;  // slice placement (SliceInfo)
+  bool skip;          // packed key tile past its sequence: no role does anything
 };
 
 // Register split: 512 threads launched at 128 registers (launch bounds 512,1);
@@ -93,15 +95,16 @@ __device__ __forceinline__ BwdUnit bwd_decode(int bh, int idx, const BwdParams& 
   BwdUnit w;
   w.bh = bh;
   w.j = p.n_ktiles - 1 - idx;
-  const int b = w.bh / p.H;
-  int L = p.N;
-  if (p.seqlens != nullptr) {
-    L = p.seqlens[b];
-    L = L < 1 ? 1 : (L > p.N ? p.N : L);
-  }
-  w.L = L;
+  const SliceInfo si = slice_info(bh, p, kErrDeviceSeqlen);
+  w.z = si.z;
+  w.row0 = si.row0;
+  w.rows = si.rows;
+  w.L = si.L;
+  const int nq = min((si.rows + kBlockM - 1) / kBlockM, p.n_ktiles);  // query tiles computed
   w.i0 = p.causal ? w.j : 0;
-  w.ni = (w.j * kBlockN < L) ? (p.n_ktiles - w.i0) : 0;  // a key tile past L only gets zeros
+  // a key tile past L only gets zeros (fixed length) or nothing (packed)
+  w.ni = (w.j * kBlockN < si.L) ? max(nq - w.i0, 0) : 0;
+  w.skip = p.cu_seqlens != nullptr && w.ni == 0;
   return w;
 }
 
@@ -198,13 +201,16 @@ __global__ void __launch_bounds__(512, 1)
         if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
         if (wi.idx < 0) continue;
         const BwdUnit w = bwd_decode(wi.bh, wi.idx, p);
+        if (w.skip) continue;
         ok = mbar_wait(kv_empty, (nunit & 1) ^ 1, abort_flag, 20);
         if (!ok) break;
         mbar_arrive_expect_tx(kv_full, 2 * Lay::kTileBytes);
 #pragma unroll
         for (int pn = 0; pn < Lay::kPanels; ++pn) {
-          tma_load_3d(sK + pn * Lay::kPanelBytes, &tmk, kv_full, pn * 64, w.j * kBlockN, w.bh);
-          tma_load_3d(sV + pn * Lay::kPanelBytes, &tmv, kv_full, pn * 64, w.j * kBlockN, w.bh);
+          tma_load_3d(sK + pn * Lay::kPanelBytes, &tmk, kv_full, pn * 64, w.row0 + w.j * kBlockN,
+                      w.z);
+          tma_load_3d(sV + pn * Lay::kPanelBytes, &tmv, kv_full, pn * 64, w.row0 + w.j * kBlockN,
+                      w.z);
         }
         ++nunit;
         for (int idx = 0; idx < w.ni && ok; ++idx) {
@@ -218,7 +224,8 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
             for (int pn = 0; pn < Lay::kPanels; ++pn)
               tma_load_3d(sSlot + slot * Lay::kTileBytes + pn * Lay::kPanelBytes,
-                          t == 0 ? &tmq : &tmdo, &slot_full[slot], pn * 64, i * kBlockM, w.bh);
+                          t == 0 ? &tmq : &tmdo, &slot_full[slot], pn * 64,
+                          w.row0 + i * kBlockM, w.z);
           }
           ++lt;
         }
@@ -243,7 +250,8 @@ __global__ void __launch_bounds__(512, 1)
       if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
       if (wi.idx < 0) continue;
       const BwdUnit w = bwd_decode(wi.bh, wi.idx, p);
-      const size_t base = static_cast<size_t>(w.bh) * p.N;
+      if (w.skip) continue;
+      const size_t base = static_cast<size_t>(w.z) * p.N + w.row0;
       for (int idx = 0; idx < w.ni && ok; ++idx) {
         const int i = w.i0 + idx;
         const int st = seq & 1;
@@ -253,10 +261,13 @@ __global__ void __launch_bounds__(512, 1)
         for (int e = 0; e < 4; ++e) {
           const int ql = lane * 4 + e;
           const int q = i * kBlockM + ql;
-          // rows past N: LSE = +inf makes P = 0 there, D = 0.  D is kept
-          // negated so the second softmax phase forms dP - D with one add.
-          sLSE[st * 128 + ql] = q < p.N ? p.lse[base + q] * log2e : INFINITY;
-          sDSUM[st * 128 + ql] = q < p.N ? -p.dsum[base + q] : 0.f;
+          // rows past the computed ones (past N, or past a packed sequence):
+          // LSE = +inf makes P = 0 there, D = 0, so they add exactly zero to
+          // dK, dV and dQ.  D is kept negated so the second softmax phase
+          // forms dP - D with one add.
+          const bool live = q < w.rows;
+          sLSE[st * 128 + ql] = live ? p.lse[base + q] * log2e : INFINITY;
+          sDSUM[st * 128 + ql] = live ? -p.dsum[base + q] : 0.f;
         }
         mbar_arrive(&ld_full[st]);
         if (lane == 0) FA_TRACE_AT(seq, 9);
@@ -288,6 +299,7 @@ __global__ void __launch_bounds__(512, 1)
         if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
         if (wi.idx < 0) continue;
         const BwdUnit w = bwd_decode(wi.bh, wi.idx, p);
+        if (w.skip) continue;
         ok = mbar_wait(kv_full, nunit & 1, abort_flag, 23);
         if (!ok) break;
         tc_fence_after();
@@ -418,6 +430,7 @@ __global__ void __launch_bounds__(512, 1)
       if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
       if (wi.idx < 0) continue;
       const BwdUnit w = bwd_decode(wi.bh, wi.idx, p);
+      if (w.skip) continue;
       if (w.ni > 0) {
         ok = seen(s_full, it & 1);
         FA_TRACE_AT(it, 16);
@@ -458,6 +471,7 @@ __global__ void __launch_bounds__(512, 1)
       if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
       if (wi.idx < 0) continue;
       const BwdUnit w = bwd_decode(wi.bh, wi.idx, p);
+      if (w.skip) continue;
       const bool key_ok = w.j * kBlockN + r < w.L;
       for (int idx = 0; idx < w.ni && ok; ++idx) {
         const int i = w.i0 + idx;
@@ -567,7 +581,8 @@ __global__ void __launch_bounds__(512, 1)
       if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
       if (wi.idx < 0) continue;
       const BwdUnit w = bwd_decode(wi.bh, wi.idx, p);
-      const size_t base = static_cast<size_t>(w.bh) * p.N;
+      if (w.skip) continue;
+      const size_t base = static_cast<size_t>(w.z) * p.N + w.row0;
       for (int idx = 0; idx < w.ni && ok; ++idx) {
         const int i = w.i0 + idx;
         ok = mbar_wait_warp(dq_full, it & 1, abort_flag, 32);
@@ -607,7 +622,7 @@ __global__ void __launch_bounds__(512, 1)
             fence_proxy_async_smem();
             named_bar_sync(1, 128);
             if (leader) {
-              tma_reduce_add_3d(&tmdq, stg, rd * 32, i * kBlockM, w.bh);
+              tma_reduce_add_3d(&tmdq, stg, rd * 32, w.row0 + i * kBlockM, w.z);
               bulk_commit_group();
             }
             ++stage_round;
@@ -622,7 +637,7 @@ __global__ void __launch_bounds__(512, 1)
       tc_fence_after();
       const int key = w.j * kBlockN + r;
       const bool keep = key < w.L;  // padded keys get exactly zero
-      const bool store = key < p.N;
+      const bool store = key < w.rows;
       const size_t off = (base + (store ? key : 0)) * (D * 2);
       uint8_t* dvrow = reinterpret_cast<uint8_t*>(p.dv) + off;
       uint8_t* dkrow = reinterpret_cast<uint8_t*>(p.dk) + off;
@@ -739,7 +754,7 @@ static int elementwise_grid(long long n8, int num_sms) {
 
 cudaError_t launch_bwd_pre(int d, bool bf16, const BwdParams& p, int num_sms,
                            cudaStream_t stream) {
-  const long long rows = static_cast<long long>(p.B) * p.H * p.N;
+  const long long rows = total_rows(p);
   const int grid = elementwise_grid(rows * d / 8, num_sms);
   const uint4* o = static_cast<const uint4*>(p.o);
   const uint4* dout = static_cast<const uint4*>(p.dout);
@@ -787,7 +802,7 @@ cudaError_t launch_bwd_main(int d, bool bf16, const CUtensorMap& tmq, const CUte
 
 cudaError_t launch_bwd_post(int d, bool bf16, const BwdParams& p, int num_sms,
                             cudaStream_t stream) {
-  const long long n8 = static_cast<long long>(p.B) * p.H * p.N * d / 8;
+  const long long n8 = total_rows(p) * d / 8;
   const int grid = elementwise_grid(n8, num_sms);
   const float4* acc = reinterpret_cast<const float4*>(p.dq_acc);
   uint4* dq = static_cast<uint4*>(p.dq);

@@ -58,26 +58,27 @@ static_assert(2 * kFwdSoftmaxRegs + kFwdOtherRegs <= 3 * kFwdLaunchRegs, "regist
 
 struct FwdUnit {
   int bh, qt0, L, jend0, jend1;
+  int z, row0, rows;  // slice placement (SliceInfo)
 };
 
-// Unit (bh, pair): query tiles 2 pair and 2 pair + 1 of head bh.
+// Unit (bh, pair): query tiles 2 pair and 2 pair + 1 of slice bh.  A query
+// tile that starts at or past the slice's computed rows has no work.
 __device__ __forceinline__ FwdUnit fwd_decode(int bh, int pair, const FwdParams& p) {
   FwdUnit w;
   w.bh = bh;
-  const int b = w.bh / p.H;
-  int L = p.N;
-  if (p.seqlens != nullptr) {
-    L = p.seqlens[b];
-    L = L < 1 ? 1 : (L > p.N ? p.N : L);
-  }
-  w.L = L;
-  const int nkb = (L + kBlockN - 1) / kBlockN;
+  const SliceInfo si = slice_info(bh, p, kErrDeviceSeqlen);
+  w.z = si.z;
+  w.row0 = si.row0;
+  w.rows = si.rows;
+  w.L = si.L;
+  const int nkb = (si.L + kBlockN - 1) / kBlockN;
+  const int nq = (si.rows + kBlockM - 1) / kBlockM;
   w.qt0 = 2 * pair;
   int je[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     const int qt = w.qt0 + t;
-    if (qt < p.n_qtiles) je[t] = p.causal ? min(nkb, qt + 1) : nkb;
+    if (qt < nq && qt < p.n_qtiles) je[t] = p.causal ? min(nkb, qt + 1) : nkb;
     else je[t] = 0;
   }
   w.jend0 = je[0];
@@ -161,7 +162,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int pn = 0; pn < Lay::kPanels; ++pn)
             tma_load_3d(sq + t * Lay::kTileBytes + pn * Lay::kPanelBytes, &tmq, &q_full[t],
-                        pn * 64, (w.qt0 + t) * kBlockM, w.bh);
+                        pn * 64, w.row0 + (w.qt0 + t) * kBlockM, w.z);
           ++qload[t];
         }
         const int jmax = max(je[0], je[1]);
@@ -176,7 +177,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
             for (int pn = 0; pn < Lay::kPanels; ++pn)
               tma_load_3d(dst + pn * Lay::kPanelBytes, kv ? &tmv : &tmk, &kv_full[slot], pn * 64,
-                          j * kBlockN, w.bh);
+                          w.row0 + j * kBlockN, w.z);
             ++kv_seq;
           }
         }
@@ -229,6 +230,7 @@ __global__ void __launch_bounds__(384, 1)
         const FwdUnit w = fwd_decode(wi.bh, wi.idx, p);
         const int je[2] = {w.jend0, w.jend1};
         const int jmax = max(je[0], je[1]);
+        if (jmax == 0) continue;  // both tiles past a packed sequence: nothing was loaded
         for (int t = 0; t < 2 && ok; ++t) {
           if (je[t] == 0) continue;
           ok = mbar_wait(&q_full[t], qload[t] & 1, abort_flag, 3);
@@ -409,9 +411,9 @@ __global__ void __launch_bounds__(384, 1)
       ++ocnt;
       tc_fence_after();
       const float inv_l = 1.f / l;
-      const bool store = row < p.N;
-      uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) +
-                      (static_cast<size_t>(w.bh) * p.N + (store ? row : 0)) * (D * 2);
+      const bool store = row < w.rows;
+      const size_t orow_idx = static_cast<size_t>(w.z) * p.N + w.row0 + (store ? row : 0);
+      uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) + orow_idx * (D * 2);
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t ro[32];
@@ -427,7 +429,7 @@ __global__ void __launch_bounds__(384, 1)
                          pk[4 * v4 + 3]);
         }
       }
-      if (store) p.lse[static_cast<size_t>(w.bh) * p.N + row] = (m + log2f(l)) * 0.69314718055994531f;
+      if (store) p.lse[orow_idx] = (m + log2f(l)) * 0.69314718055994531f;
     }
   }
 

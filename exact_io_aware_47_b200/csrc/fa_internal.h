@@ -6,6 +6,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "sm100.cuh"
+
 namespace fa {
 
 constexpr int kBlockM = 128;  // query rows per tile (TMEM lanes)
@@ -17,10 +19,17 @@ constexpr int kBlockN = 128;  // keys per tile
 // with the same max) still yields the exact softmax.
 constexpr float kRescaleThreshold = 8.0f;
 
+// Two layouts share the kernels.  Fixed length: tensors [B, H, N, d], a
+// (batch, head) slice is row block b * H + h of N rows.  Packed (cu_seqlens
+// given): tensors [H, T, d] with the B sequences of head h back to back,
+// sequence b in rows [cu_seqlens[b], cu_seqlens[b + 1]) of block h; N holds T
+// and the tile counts come from max_seqlen.
 struct FwdParams {
-  void* o;                  // [B, H, N, d] 16-bit
-  float* lse;               // [B, H, N] natural-log log-sum-exp
-  const int32_t* seqlens;   // [B] valid key lengths, or nullptr
+  void* o;                  // [B, H, N, d] or [H, T, d], 16-bit
+  float* lse;               // [B, H, N] or [H, T] natural-log log-sum-exp
+  const int32_t* seqlens;   // [B] valid key lengths (fixed length), or nullptr
+  const int32_t* cu_seqlens;  // [B + 1] sequence offsets (packed), or nullptr
+  int max_seqlen;           // packed: upper bound of every sequence length
   int B, H, N;
   float scale_log2;         // scale * log2(e)
   int causal;
@@ -42,6 +51,8 @@ struct BwdParams {
   float* dsum;              // workspace [B, H, N]: D_i = <dO_i, O_i>
   float* dq_acc;            // workspace [B, H, N, d] fp32 accumulator
   const int32_t* seqlens;
+  const int32_t* cu_seqlens;  // as in FwdParams
+  int max_seqlen;
   int B, H, N;
   float scale;
   float scale_log2;
@@ -58,6 +69,50 @@ struct BwdParams {
 // runs the two halves back to back.  k counts the work items of this CTA;
 // returns false past the end; idx < 0 marks the missing mirror of an odd
 // middle unit.
+// Where a (batch, head) slice lives and how long it is: rows [row0, row0 + L)
+// of row block z (z = b * H + h, row0 = 0, L = seqlens[b] or N for fixed
+// length; z = h, row0 = cu_seqlens[b] packed).  `rows` bounds the query rows
+// that are computed and stored: N for fixed length (padded query rows are
+// still computed), L packed (the rows after L belong to the next sequence).
+// Out-of-range sequence descriptions are clamped and reported.
+struct SliceInfo {
+  int z, row0, L, rows;
+};
+
+template <class P>
+__device__ __forceinline__ SliceInfo slice_info(int bh, const P& p, int err_code) {
+  SliceInfo s;
+  const int b = bh / p.H;
+  if (p.cu_seqlens != nullptr) {
+    int s0 = p.cu_seqlens[b], s1 = p.cu_seqlens[b + 1];
+    const int c0 = min(max(s0, 0), p.N);
+    const int c1 = min(max(s1, c0), min(p.N, c0 + p.max_seqlen));
+    if (c0 != s0 || c1 != s1) record_error(err_code, 1);
+    s.z = bh - b * p.H;
+    s.row0 = c0;
+    s.L = c1 - c0;
+    s.rows = s.L;
+  } else {
+    int L = p.N;
+    if (p.seqlens != nullptr) {
+      L = p.seqlens[b];
+      L = L < 1 ? 1 : (L > p.N ? p.N : L);
+    }
+    s.z = bh;
+    s.row0 = 0;
+    s.L = L;
+    s.rows = p.N;
+  }
+  return s;
+}
+
+// Rows of all (batch, head) slices together (the element-wise kernels).
+template <class P>
+__host__ __device__ inline long long total_rows(const P& p) {
+  return p.cu_seqlens != nullptr ? static_cast<long long>(p.H) * p.N
+                                 : static_cast<long long>(p.B) * p.H * p.N;
+}
+
 struct WorkItem {
   int bh;   // batch * head
   int idx;  // unit index inside the head: n-1-m for the first half, m for the second

@@ -16,6 +16,11 @@ always hands both the kernel and the oracle the same tensors):
    that the running row max keeps growing across K tiles;
 4. each tensor cast round-to-nearest-even to the workload's 16-bit dtype.
 
+Packed variable-length inputs (``make_inputs_varlen``): sequence lengths
+drawn uniformly from {1, ..., max_len} (``torch.randint``) unless given,
+``cu_seqlens`` their running sum from 0, then Q, K, V, dO each an iid N(0, 1)
+float32 draw of shape [H, T, d] (T = total length), cast as in step 4.
+
 The pages name no dataset or benchmark suite; these shapes stand in for the
 workloads they discuss (n = 8192 fp16 sizing, 32k context, short training
 shapes, padded batches).
@@ -26,7 +31,8 @@ from dataclasses import dataclass, field
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_inputs_shape"]
+__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_inputs_shape", "PackedWorkload",
+           "PACKED_WORKLOADS", "make_inputs_varlen", "make_inputs_packed"]
 
 
 @dataclass(frozen=True)
@@ -98,3 +104,60 @@ def make_inputs(name, dtype=None, seed=0, with_do=True, device="cpu"):
     dt = dtype if dtype is not None else w.dtypes[0]
     return make_inputs_shape(w.B, w.H, w.N, w.d, dt, seed=seed, ragged=w.ragged,
                              with_do=with_do, device=device)
+
+
+@dataclass(frozen=True)
+class PackedWorkload:
+    name: str
+    B: int          # sequences
+    H: int
+    max_len: int    # lengths ~ U{1, ..., max_len}
+    d: int
+    causal: bool
+    dtype: torch.dtype
+    description: str = field(default="", compare=False)
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+
+PACKED_WORKLOADS = {
+    "varlen": PackedWorkload("varlen", 8, 16, 4099, 128, False, torch.bfloat16,
+                             description="8 packed sequences, lengths ~ U{1..4099}, H16 d128 bf16, "
+                                         "non-causal (the padded batch without its padding)"),
+}
+
+
+def make_inputs_varlen(B, H, max_len, d, dtype, seed=0, lengths=None, with_do=True,
+                       device="cpu"):
+    """Draw a packed batch: q, k, v (and dO) [H, T, d], ``cu_seqlens`` int32
+    [B + 1] and the host list ``lengths``; ``max_seqlen`` is max(lengths, 1)."""
+    device = torch.device(device)
+    g = torch.Generator(device=device).manual_seed(seed)
+    if lengths is None:
+        ln = torch.randint(1, max_len + 1, (B,), generator=g, dtype=torch.int64, device=device)
+        lengths = [int(x) for x in ln.cpu()]
+    lengths = [int(x) for x in lengths]
+    if len(lengths) != B or min(lengths) < 0:
+        raise ValueError("lengths must be B non-negative integers")
+    cu = [0]
+    for n in lengths:
+        cu.append(cu[-1] + n)
+    T = cu[-1]
+    shape = (H, T, d)
+    q = torch.randn(shape, generator=g, dtype=torch.float32, device=device)
+    k = torch.randn(shape, generator=g, dtype=torch.float32, device=device)
+    v = torch.randn(shape, generator=g, dtype=torch.float32, device=device)
+    do = torch.randn(shape, generator=g, dtype=torch.float32, device=device) if with_do else None
+    return {"q": q.to(dtype), "k": k.to(dtype), "v": v.to(dtype),
+            "do": do.to(dtype) if do is not None else None,
+            "cu_seqlens": torch.tensor(cu, dtype=torch.int32, device=device),
+            "lengths": lengths, "max_seqlen": max(max(lengths), 1)}
+
+
+def make_inputs_packed(name, seed=0, with_do=True, device="cpu"):
+    """Inputs of a named packed workload (``PACKED_WORKLOADS``)."""
+    w = PACKED_WORKLOADS[name]
+    return make_inputs_varlen(w.B, w.H, w.max_len, w.d, w.dtype, seed=seed, with_do=with_do,
+                              device=device)

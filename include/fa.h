@@ -128,6 +128,43 @@ int fa_bwd_postprocess(void* workspace, size_t workspace_bytes, void* dq,
                        void* stream);
 
 /*
+ * Packed variable-length batches: B sequences of different lengths stored
+ * back to back, with no padding rows.  Same method, masks and numerics as
+ * fa_fwd / fa_bwd, with each sequence its own attention problem: queries of
+ * sequence b see only keys of sequence b ("How Flash Attention Works",
+ * section "Tiling Q, K, and V": the sequence is tiled and ragged edges are
+ * masked per tile; here the edges are the sequence boundaries).
+ *   Layout.  Q, K, V, O, dO, dQ, dK, dV are [H, T, d] 16-bit: head-major like
+ *     the fixed-length tensors, with the B sequences of every head
+ *     concatenated along the T rows.  LSE is [H, T] float32.  cu_seqlens is a
+ *     device int32 [B + 1] array of row offsets: sequence b occupies rows
+ *     cu_seqlens[b] .. cu_seqlens[b + 1] - 1 of every head, with
+ *     0 = cu_seqlens[0] <= ... <= cu_seqlens[B] = T.  Empty sequences are
+ *     allowed.  max_seqlen (host int) bounds every length; it sets the work
+ *     decomposition, so a tight bound wastes no work.
+ *   Masks.  causal != 0 hides key j from query i of the same sequence when
+ *     j > i (positions counted from the sequence start).  Rows of other
+ *     sequences never enter a sequence's result.  Rows outside
+ *     [cu_seqlens[0], cu_seqlens[B]) belong to no sequence: o, lse, dk and
+ *     dv leave them untouched, dq gets zeros there.
+ *   Sizes.  B, H, T, max_seqlen >= 1; d in {64, 128}; H*T*d < 2^31;
+ *     B*H*ceil(min(max_seqlen, T) / 128) < 2^31.  A cu_seqlens description
+ *     that is out of range (decreasing, past T, a sequence longer than
+ *     max_seqlen) is clamped on the device and reported by
+ *     fa_device_status() as FA_ERR_DEVICE_SEQLEN.
+ *   fa_bwd_varlen's workspace: fa_bwd_workspace_size(1, H, T, d) bytes,
+ *     256-byte aligned; it runs the three backward stages on `stream`.
+ */
+int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                  const int32_t* cu_seqlens, int B, int H, int T, int max_seqlen,
+                  int d, float scale, int causal, int dtype, void* stream);
+int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
+                  const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                  void* workspace, size_t workspace_bytes, const int32_t* cu_seqlens,
+                  int B, int H, int T, int max_seqlen, int d, float scale, int causal,
+                  int dtype, void* stream);
+
+/*
  * Backward pass that allocates nothing and takes no workspace.  The pages
  * have no counterpart: it exists for callers that cannot allocate device
  * memory for a workspace, such as plugin hosts that hand an operator only its

@@ -44,19 +44,19 @@ def assert_fwd_close(o_gpu, lse_gpu, o_ref, lse_ref, what=""):
     return do.max(), do.mean(), dl.max()
 
 
-def assert_grad_close(g_gpu, g_ref, what="", typical=None):
+def assert_grad_close(g_gpu, g_ref, what="", typical=None, floor_frac=1e-3):
     """max |g_gpu - g_ref| <= GRAD_REL_MAX * max|g_ref|.
 
     ``typical`` is the gradient magnitude of the whole tensor the slice comes
     from.  Rounding residuals scale with the magnitudes being combined, not
     with a slice's exact result, so a slice whose exact gradient vanishes (one
-    visible key) is held to GRAD_REL_MAX * 1e-3 * typical (and never less than
-    GRAD_REL_MAX * GRAD_ABS_FLOOR).
+    visible key) is held to GRAD_REL_MAX * floor_frac * typical (and never
+    less than GRAD_REL_MAX * GRAD_ABS_FLOOR).
     """
     assert np.isfinite(g_gpu).all(), f"{what}: non-finite gradient"
     err = np.abs(g_gpu - g_ref).max()
     scale = np.abs(g_ref).max()
-    floor = GRAD_ABS_FLOOR if typical is None else max(GRAD_ABS_FLOOR, 1e-3 * typical)
+    floor = GRAD_ABS_FLOOR if typical is None else max(GRAD_ABS_FLOOR, floor_frac * typical)
     assert err <= GRAD_REL_MAX * max(scale, floor), \
         f"{what}: max|d| {err:.3e} vs max|ref| {scale:.3e}"
     return err / max(scale, 1e-30)
