@@ -1,6 +1,7 @@
 """Throughput of exact tiled attention (forward + backward) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload mid|small|long|ragged|tiny|varlen]
 
 One step is the whole hot path over one batch: fa_fwd, then the three
 backward stages (row-dot preprocess, main kernel, dQ convert), on the
@@ -12,6 +13,9 @@ backward 2.5x that.
 With N > 1 (torchrun), every rank runs its own replica of the workload (the
 op has no cross-GPU exchange); the time is the max over ranks and the value
 counts the work of all ranks.
+
+``--workload varlen`` times the packed variable-length path (fa_fwd_varlen +
+fa_bwd_varlen) on 8 sequences of lengths ~ U{1..4099}, H16, d128, bf16.
 
 ``--impl reference`` times the float64 CPU oracle (test infrastructure, the
 only other place this script runs it) on bounded samples of the same
@@ -395,9 +399,180 @@ def run_ours(args, w):
     return 0
 
 
+# ------------------------------------------------------ packed (variable length)
+def flops_fwd_packed(lengths, H, d, causal):
+    return sum(flops_fwd(1, H, n, d, causal) for n in lengths)
+
+
+def run_ours_packed(args, w):
+    """``--workload varlen``: one step = fa_fwd_varlen + fa_bwd_varlen (its
+    three kernels in one call) on a packed batch; FLOPs summed per sequence."""
+    import torch
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from exact_io_aware_47_b200 import _lib, build
+    build.build()
+    import exact_io_aware_47_b200 as fa
+    from exact_io_aware_47_b200.inputs import make_inputs_packed
+
+    inp = make_inputs_packed(w.name, seed=rank, device=dev)
+    q, k, v, do = inp["q"], inp["k"], inp["v"], inp["do"]
+    cu, ms, lengths = inp["cu_seqlens"], inp["max_seqlen"], inp["lengths"]
+    H, T, d = q.shape
+    B, causal, scale = w.B, w.causal, w.scale
+    o, lse = torch.empty_like(q), torch.empty((H, T), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_bytes = fa.workspace_bytes(1, H, T, d)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    dt_code = _lib.FA_BF16 if w.dtype == torch.bfloat16 else _lib.FA_FP16
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        _lib.check("fa_fwd_varlen", _lib.fa_fwd_varlen(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), cu.data_ptr(),
+            B, H, T, ms, d, scale, int(causal), dt_code, sh))
+        if ev is not None:
+            ev[1].record(stream)
+        _lib.check("fa_bwd_varlen", _lib.fa_bwd_varlen(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
+            dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws_bytes, cu.data_ptr(),
+            B, H, T, ms, d, scale, int(causal), dt_code, sh))
+        if ev is not None:
+            ev[2].record(stream)
+
+    warmup = max(3, args.warmup)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    st, word = _lib.fa_device_status(sh)
+    if st != 0:
+        raise RuntimeError(f"device status {st} ({word:#x}) after warm-up")
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    if not args.no_clocks:
+        clocks.start()
+        time.sleep(0.3)
+    dist_barrier(world)
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(K):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    dist_barrier(world)
+    clk = None if args.no_clocks else clocks.stop()
+    st, word = _lib.fa_device_status(sh)
+    if st != 0:
+        raise RuntimeError(f"device status {st} ({word:#x}) after timing")
+    total_ms = dist_max(t0.elapsed_time(t1), world)
+    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
+    bwd_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / K
+    f_fwd = flops_fwd_packed(lengths, H, d, causal)
+    f_bwd = 2.5 * f_fwd
+    step_flops = f_fwd + f_bwd
+    value = world * step_flops * K / (total_ms / 1e3) / 1e12
+    peaks, peak_src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    fwd_tf = f_fwd / (fwd_ms / 1e3) / 1e12
+    bwd_tf = f_bwd / (bwd_ms / 1e3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "fa_bwd_varlen (preprocess + main + postprocess)",
+                "achieved": bwd_tf, "peak": peak, "unit": "TFLOP/s", "frac": bwd_tf / peak,
+                "traffic": None, "peak_source": f"{peak_src} bf16 dense (burst)",
+                "flops_per_launch": f_bwd}
+    roofline_fwd = {"bound": "tensor", "kernel": "fa_fwd_kernel (fa_fwd_varlen)",
+                    "achieved": fwd_tf, "peak": peak, "unit": "TFLOP/s", "frac": fwd_tf / peak,
+                    "traffic": None, "peak_source": f"{peak_src} bf16 dense (burst)",
+                    "flops_per_launch": f_fwd}
+
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
+        ho, hdq, hdk, hdv = (torch.empty(q.shape, dtype=w.dtype, pin_memory=True)
+                             for _ in range(4))
+        hlse = torch.empty((H, T), dtype=torch.float32, pin_memory=True)
+        hcu = cu.cpu().pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo, hcu))
+        d2h = sum(t.numel() * t.element_size() for t in (ho, hlse, hdq, hdk, hdv))
+
+        def e2e_step():
+            for src, dst in ((hq, q), (hk, k), (hv, v), (hdo, do), (hcu, cu)):
+                dst.copy_(src, non_blocking=True)
+            fa.forward_varlen(q, k, v, cu, ms, scale=scale, causal=causal, out=o, lse=lse)
+            fa.backward_varlen(q, k, v, o, lse, do, cu, ms, scale=scale, causal=causal,
+                               workspace=ws, dq=dq, dk=dk, dv=dv)
+            for src, dst in ((o, ho), (lse, hlse), (dq, hdq), (dk, hdk), (dv, hdv)):
+                dst.copy_(src, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        ke = max(3, min(K, 10))
+        dist_barrier(world)
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(ke):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        dist_barrier(world)
+        e_ms = dist_max(a.elapsed_time(b), world)
+        e2e = {"value": world * step_flops * ke / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / ke}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from threadpoolctl import threadpool_info
+        from oracle import ref_bwd_slice, ref_fwd_slice
+        s0, s1 = int(cu[0]), int(cu[1])
+        sl = slice(s0, s1)
+        qq, kk, vv, dd = (t[0, sl].double().cpu().numpy() for t in (q, k, v, do))
+        tc = time.perf_counter()
+        ref_fwd_slice(qq, kk, vv, scale, causal)
+        ref_bwd_slice(qq, kk, vv, dd, scale, causal)
+        dt = time.perf_counter() - tc
+        fl = 3.5 * flops_fwd(1, 1, s1 - s0, d, causal)
+        thr = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+               "sample": f"float64 oracle forward+backward of head 0 of the first packed "
+                         f"sequence ({s1 - s0} rows, {dt:.1f} s)"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == torch.bfloat16 else "f16", "data": "synthetic",
+        "config": {"workload": w.description, "B": B, "H": H, "T": T, "max_seqlen": ms, "d": d,
+                   "causal": causal, "lengths": lengths,
+                   "step": "fa_fwd_varlen + fa_bwd_varlen", "flops_per_step": step_flops,
+                   "parallelism": f"replicas x{world}",
+                   "l2": f"inputs {4 * q.numel() * q.element_size() / 2**20:.0f} MiB per step, "
+                         "no flush"},
+        "fwd": {"ms": fwd_ms, "tflops": fwd_tf, "frac": fwd_tf / peak},
+        "bwd": {"ms": bwd_ms, "tflops": bwd_tf, "frac": bwd_tf / peak},
+        "roofline": roofline, "roofline_fwd": roofline_fwd,
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 4 * K, "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse()
-    from exact_io_aware_47_b200.inputs import WORKLOADS
+    from exact_io_aware_47_b200.inputs import PACKED_WORKLOADS, WORKLOADS
+    if args.workload in PACKED_WORKLOADS:
+        if args.impl == "reference":
+            raise SystemExit("--impl reference times the fixed-length workloads")
+        return run_ours_packed(args, PACKED_WORKLOADS[args.workload])
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
