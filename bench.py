@@ -529,18 +529,26 @@ def run_ours_packed(args, w):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         from threadpoolctl import threadpool_info
         from oracle import ref_bwd_slice, ref_fwd_slice
-        s0, s1 = int(cu[0]), int(cu[1])
-        sl = slice(s0, s1)
-        qq, kk, vv, dd = (t[0, sl].double().cpu().numpy() for t in (q, k, v, do))
-        tc = time.perf_counter()
-        ref_fwd_slice(qq, kk, vv, scale, causal)
-        ref_bwd_slice(qq, kk, vv, dd, scale, causal)
-        dt = time.perf_counter() - tc
-        fl = 3.5 * flops_fwd(1, 1, s1 - s0, d, causal)
+        cuh = [int(x) for x in cu.cpu()]
+        dt, fl, n_done = 0.0, 0.0, 0
+        for h in range(H):  # whole (head, sequence) slices until ~10 s of CPU work
+            for b in range(B):
+                s0, s1 = cuh[b], cuh[b + 1]
+                if s1 == s0:
+                    continue
+                qq, kk, vv, dd = (t[h, s0:s1].double().cpu().numpy() for t in (q, k, v, do))
+                tc = time.perf_counter()
+                ref_fwd_slice(qq, kk, vv, scale, causal)
+                ref_bwd_slice(qq, kk, vv, dd, scale, causal)
+                dt += time.perf_counter() - tc
+                fl += 3.5 * flops_fwd(1, 1, s1 - s0, d, causal)
+                n_done += 1
+            if dt >= 10.0:
+                break
         thr = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
         cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
-               "sample": f"float64 oracle forward+backward of head 0 of the first packed "
-                         f"sequence ({s1 - s0} rows, {dt:.1f} s)"}
+               "sample": f"float64 oracle forward+backward of {n_done} whole (head, sequence) "
+                         f"slices, all sequences of the first heads ({dt:.1f} s)"}
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,

@@ -91,11 +91,12 @@ static_assert(2 * kBwdSoftmaxRegs + kBwdDqRegs + kBwdOtherRegs <= 4 * kBwdLaunch
 
 // Unit (bh, key tile j).  The work order hands out key tiles mirrored
 // (j = n-1-idx), so the long tile of a causal super-unit (small j) runs first.
+template <bool PACKED>
 __device__ __forceinline__ BwdUnit bwd_decode(int bh, int idx, const BwdParams& p) {
   BwdUnit w;
   w.bh = bh;
   w.j = p.n_ktiles - 1 - idx;
-  const SliceInfo si = slice_info(bh, p, kErrDeviceSeqlen);
+  const SliceInfo si = slice_info<PACKED>(bh, p, kErrDeviceSeqlen);
   w.z = si.z;
   w.row0 = si.row0;
   w.rows = si.rows;
@@ -104,11 +105,11 @@ __device__ __forceinline__ BwdUnit bwd_decode(int bh, int idx, const BwdParams& 
   w.i0 = p.causal ? w.j : 0;
   // a key tile past L only gets zeros (fixed length) or nothing (packed)
   w.ni = (w.j * kBlockN < si.L) ? max(nq - w.i0, 0) : 0;
-  w.skip = p.cu_seqlens != nullptr && w.ni == 0;
+  w.skip = PACKED && w.ni == 0;
   return w;
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool PACKED>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdo,
@@ -200,7 +201,7 @@ __global__ void __launch_bounds__(512, 1)
         WorkItem wi;
         if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
         if (wi.idx < 0) continue;
-        const BwdUnit w = bwd_decode(wi.bh, wi.idx, p);
+        const BwdUnit w = bwd_decode<PACKED>(wi.bh, wi.idx, p);
         if (w.skip) continue;
         ok = mbar_wait(kv_empty, (nunit & 1) ^ 1, abort_flag, 20);
         if (!ok) break;
@@ -249,7 +250,7 @@ __global__ void __launch_bounds__(512, 1)
       WorkItem wi;
       if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
       if (wi.idx < 0) continue;
-      const BwdUnit w = bwd_decode(wi.bh, wi.idx, p);
+      const BwdUnit w = bwd_decode<PACKED>(wi.bh, wi.idx, p);
       if (w.skip) continue;
       const size_t base = static_cast<size_t>(w.z) * p.N + w.row0;
       for (int idx = 0; idx < w.ni && ok; ++idx) {
@@ -298,7 +299,7 @@ __global__ void __launch_bounds__(512, 1)
         WorkItem wi;
         if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
         if (wi.idx < 0) continue;
-        const BwdUnit w = bwd_decode(wi.bh, wi.idx, p);
+        const BwdUnit w = bwd_decode<PACKED>(wi.bh, wi.idx, p);
         if (w.skip) continue;
         ok = mbar_wait(kv_full, nunit & 1, abort_flag, 23);
         if (!ok) break;
@@ -429,7 +430,7 @@ __global__ void __launch_bounds__(512, 1)
       WorkItem wi;
       if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
       if (wi.idx < 0) continue;
-      const BwdUnit w = bwd_decode(wi.bh, wi.idx, p);
+      const BwdUnit w = bwd_decode<PACKED>(wi.bh, wi.idx, p);
       if (w.skip) continue;
       if (w.ni > 0) {
         ok = seen(s_full, it & 1);
@@ -470,7 +471,7 @@ __global__ void __launch_bounds__(512, 1)
       WorkItem wi;
       if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
       if (wi.idx < 0) continue;
-      const BwdUnit w = bwd_decode(wi.bh, wi.idx, p);
+      const BwdUnit w = bwd_decode<PACKED>(wi.bh, wi.idx, p);
       if (w.skip) continue;
       const bool key_ok = w.j * kBlockN + r < w.L;
       for (int idx = 0; idx < w.ni && ok; ++idx) {
@@ -580,7 +581,7 @@ __global__ void __launch_bounds__(512, 1)
       WorkItem wi;
       if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
       if (wi.idx < 0) continue;
-      const BwdUnit w = bwd_decode(wi.bh, wi.idx, p);
+      const BwdUnit w = bwd_decode<PACKED>(wi.bh, wi.idx, p);
       if (w.skip) continue;
       const size_t base = static_cast<size_t>(w.z) * p.N + w.row0;
       for (int idx = 0; idx < w.ni && ok; ++idx) {
@@ -769,13 +770,13 @@ cudaError_t launch_bwd_pre(int d, bool bf16, const BwdParams& p, int num_sms,
   return cudaGetLastError();
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool PACKED>
 static cudaError_t launch_bwd_main_t(const CUtensorMap& tmq, const CUtensorMap& tmk,
                                      const CUtensorMap& tmv, const CUtensorMap& tmdo,
                                      const CUtensorMap& tmdq, const BwdParams& p, int num_sms,
                                      cudaStream_t stream) {
   using Lay = BwdLayout<D>;
-  auto kern = fa_bwd_kernel<D, BF16>;
+  auto kern = fa_bwd_kernel<D, BF16, PACKED>;
   cudaFuncAttributes attr;
   cudaError_t e = cudaFuncGetAttributes(&attr, kern);
   if (e != cudaSuccess) return e;
@@ -792,12 +793,16 @@ cudaError_t launch_bwd_main(int d, bool bf16, const CUtensorMap& tmq, const CUte
                             const CUtensorMap& tmv, const CUtensorMap& tmdo,
                             const CUtensorMap& tmdq, const BwdParams& p, int num_sms,
                             cudaStream_t stream) {
+  const bool packed = p.cu_seqlens != nullptr;
+#define FA_BWD_LAUNCH(DD, BB, PP) \
+  launch_bwd_main_t<DD, BB, PP>(tmq, tmk, tmv, tmdo, tmdq, p, num_sms, stream)
   if (d == 128) {
-    return bf16 ? launch_bwd_main_t<128, true>(tmq, tmk, tmv, tmdo, tmdq, p, num_sms, stream)
-                : launch_bwd_main_t<128, false>(tmq, tmk, tmv, tmdo, tmdq, p, num_sms, stream);
+    if (packed) return bf16 ? FA_BWD_LAUNCH(128, true, true) : FA_BWD_LAUNCH(128, false, true);
+    return bf16 ? FA_BWD_LAUNCH(128, true, false) : FA_BWD_LAUNCH(128, false, false);
   }
-  return bf16 ? launch_bwd_main_t<64, true>(tmq, tmk, tmv, tmdo, tmdq, p, num_sms, stream)
-              : launch_bwd_main_t<64, false>(tmq, tmk, tmv, tmdo, tmdq, p, num_sms, stream);
+  if (packed) return bf16 ? FA_BWD_LAUNCH(64, true, true) : FA_BWD_LAUNCH(64, false, true);
+  return bf16 ? FA_BWD_LAUNCH(64, true, false) : FA_BWD_LAUNCH(64, false, false);
+#undef FA_BWD_LAUNCH
 }
 
 cudaError_t launch_bwd_post(int d, bool bf16, const BwdParams& p, int num_sms,

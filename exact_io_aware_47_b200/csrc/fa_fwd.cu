@@ -63,10 +63,11 @@ struct FwdUnit {
 
 // Unit (bh, pair): query tiles 2 pair and 2 pair + 1 of slice bh.  A query
 // tile that starts at or past the slice's computed rows has no work.
+template <bool PACKED>
 __device__ __forceinline__ FwdUnit fwd_decode(int bh, int pair, const FwdParams& p) {
   FwdUnit w;
   w.bh = bh;
-  const SliceInfo si = slice_info(bh, p, kErrDeviceSeqlen);
+  const SliceInfo si = slice_info<PACKED>(bh, p, kErrDeviceSeqlen);
   w.z = si.z;
   w.row0 = si.row0;
   w.rows = si.rows;
@@ -86,7 +87,7 @@ __device__ __forceinline__ FwdUnit fwd_decode(int bh, int pair, const FwdParams&
   return w;
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool PACKED>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const FwdParams p) {
@@ -152,7 +153,7 @@ __global__ void __launch_bounds__(384, 1)
         WorkItem wi;
         if (!work_item(k, p.n_pairs, p.B * p.H, wi)) break;
         if (wi.idx < 0) continue;
-        const FwdUnit w = fwd_decode(wi.bh, wi.idx, p);
+        const FwdUnit w = fwd_decode<PACKED>(wi.bh, wi.idx, p);
         const int je[2] = {w.jend0, w.jend1};
         for (int t = 0; t < 2 && ok; ++t) {
           if (je[t] == 0) continue;
@@ -227,10 +228,10 @@ __global__ void __launch_bounds__(384, 1)
         WorkItem wi;
         if (!work_item(k, p.n_pairs, p.B * p.H, wi)) break;
         if (wi.idx < 0) continue;
-        const FwdUnit w = fwd_decode(wi.bh, wi.idx, p);
+        const FwdUnit w = fwd_decode<PACKED>(wi.bh, wi.idx, p);
         const int je[2] = {w.jend0, w.jend1};
         const int jmax = max(je[0], je[1]);
-        if (jmax == 0) continue;  // both tiles past a packed sequence: nothing was loaded
+        if (PACKED && jmax == 0) continue;  // both tiles past a packed sequence: nothing loaded
         for (int t = 0; t < 2 && ok; ++t) {
           if (je[t] == 0) continue;
           ok = mbar_wait(&q_full[t], qload[t] & 1, abort_flag, 3);
@@ -313,7 +314,7 @@ __global__ void __launch_bounds__(384, 1)
       WorkItem wi;
       if (!work_item(k, p.n_pairs, p.B * p.H, wi)) break;
       if (wi.idx < 0) continue;
-      const FwdUnit w = fwd_decode(wi.bh, wi.idx, p);
+      const FwdUnit w = fwd_decode<PACKED>(wi.bh, wi.idx, p);
       const int jend = t == 0 ? w.jend0 : w.jend1;
       if (jend == 0) continue;
       const int qt = w.qt0 + t;
@@ -441,12 +442,12 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool PACKED>
 static cudaError_t launch_fwd_t(const CUtensorMap& tmq, const CUtensorMap& tmk,
                                 const CUtensorMap& tmv, const FwdParams& p, int num_sms,
                                 cudaStream_t stream) {
   using Lay = FwdLayout<D>;
-  auto kern = fa_fwd_kernel<D, BF16>;
+  auto kern = fa_fwd_kernel<D, BF16, PACKED>;
   cudaFuncAttributes attr;
   cudaError_t e = cudaFuncGetAttributes(&attr, kern);
   if (e != cudaSuccess) return e;
@@ -462,12 +463,19 @@ static cudaError_t launch_fwd_t(const CUtensorMap& tmq, const CUtensorMap& tmk,
 cudaError_t launch_fwd(int d, bool bf16, const CUtensorMap& tmq, const CUtensorMap& tmk,
                        const CUtensorMap& tmv, const FwdParams& p, int num_sms,
                        cudaStream_t stream) {
+  const bool packed = p.cu_seqlens != nullptr;
   if (d == 128) {
-    return bf16 ? launch_fwd_t<128, true>(tmq, tmk, tmv, p, num_sms, stream)
-                : launch_fwd_t<128, false>(tmq, tmk, tmv, p, num_sms, stream);
+    if (packed)
+      return bf16 ? launch_fwd_t<128, true, true>(tmq, tmk, tmv, p, num_sms, stream)
+                  : launch_fwd_t<128, false, true>(tmq, tmk, tmv, p, num_sms, stream);
+    return bf16 ? launch_fwd_t<128, true, false>(tmq, tmk, tmv, p, num_sms, stream)
+                : launch_fwd_t<128, false, false>(tmq, tmk, tmv, p, num_sms, stream);
   }
-  return bf16 ? launch_fwd_t<64, true>(tmq, tmk, tmv, p, num_sms, stream)
-              : launch_fwd_t<64, false>(tmq, tmk, tmv, p, num_sms, stream);
+  if (packed)
+    return bf16 ? launch_fwd_t<64, true, true>(tmq, tmk, tmv, p, num_sms, stream)
+                : launch_fwd_t<64, false, true>(tmq, tmk, tmv, p, num_sms, stream);
+  return bf16 ? launch_fwd_t<64, true, false>(tmq, tmk, tmv, p, num_sms, stream)
+              : launch_fwd_t<64, false, false>(tmq, tmk, tmv, p, num_sms, stream);
 }
 
 }  // namespace fa

@@ -74,16 +74,18 @@ struct BwdParams {
 // length; z = h, row0 = cu_seqlens[b] packed).  `rows` bounds the query rows
 // that are computed and stored: N for fixed length (padded query rows are
 // still computed), L packed (the rows after L belong to the next sequence).
-// Out-of-range sequence descriptions are clamped and reported.
+// Out-of-range sequence descriptions are clamped and reported.  The kernels
+// are instantiated per layout (PACKED), so the fixed-length code carries no
+// trace of the packed one.
 struct SliceInfo {
   int z, row0, L, rows;
 };
 
-template <class P>
+template <bool PACKED, class P>
 __device__ __forceinline__ SliceInfo slice_info(int bh, const P& p, int err_code) {
   SliceInfo s;
   const int b = bh / p.H;
-  if (p.cu_seqlens != nullptr) {
+  if constexpr (PACKED) {
     int s0 = p.cu_seqlens[b], s1 = p.cu_seqlens[b + 1];
     const int c0 = min(max(s0, 0), p.N);
     const int c1 = min(max(s1, c0), min(p.N, c0 + p.max_seqlen));
