@@ -31,7 +31,14 @@ design notes of the repository):
   every query row; query rows i >= L are still computed against the L valid
   keys;
 * a row whose every key is masked yields O = 0 and LSE = -inf (cannot occur
-  for valid inputs: L >= 1 and key 0 is always visible);
+  for dense inputs: L >= 1 and key 0 is always visible; it does with a block
+  mask);
+* block-sparse attention ("sparse-attention-flashattention" glossary page,
+  definition: the original paper's block-sparse extension, a separate
+  configuration of the same exact attention): a boolean block mask over
+  (query block, key block) pairs of ``block`` x ``block`` scores hides every
+  score of a block whose entry is false, on top of the causal and padding
+  masks; the softmax runs over what remains;
 * the gradients are those of O with respect to Q, K, V by the chain rule:
   dV = P^T dO, dP = dO V^T, D_i = sum_j P_ij dP_ij, dS = P * (dP - D),
   dQ = scale * dS K, dK = scale * dS^T Q.
@@ -52,22 +59,27 @@ __all__ = [
 ]
 
 
-def allowed_mask(rows, n_keys, valid_len, causal):
+def allowed_mask(rows, n_keys, valid_len, causal, block_mask=None, block=128):
     """Boolean [len(rows), n_keys]: True where key j is visible to query row i.
 
     Key padding masks keys j >= valid_len ("Tiling Q, K, and V" section:
     padding applied per tile).  Causal masking hides keys j > i ("The
-    Exact-Attention Idea": causal masking for autoregressive decoding).
+    Exact-Attention Idea": causal masking for autoregressive decoding).  A
+    block mask (boolean [query blocks, key blocks]) hides the scores of every
+    block whose entry is false.
     """
     rows = np.asarray(rows)
     j = np.arange(n_keys)
     allowed = np.broadcast_to(j[None, :] < valid_len, (rows.shape[0], n_keys)).copy()
     if causal:
         allowed &= j[None, :] <= rows[:, None]
+    if block_mask is not None:
+        bm = np.asarray(block_mask, dtype=bool)
+        allowed &= bm[rows[:, None] // block, j[None, :] // block]
     return allowed
 
 
-def _scores_probs(q, k, scale, causal, valid_len, rows):
+def _scores_probs(q, k, scale, causal, valid_len, rows, block_mask=None, block=128):
     """S (masked with -inf) and P = softmax(S) for the given query rows.
 
     Follows the textbook schedule of the "Standard attention I/O is the
@@ -76,7 +88,7 @@ def _scores_probs(q, k, scale, causal, valid_len, rows):
     """
     n_keys = k.shape[0]
     s = scale * (q[rows] @ k.T)                       # [R, N] float64
-    allowed = allowed_mask(rows, n_keys, valid_len, causal)
+    allowed = allowed_mask(rows, n_keys, valid_len, causal, block_mask, block)
     s = np.where(allowed, s, -np.inf)
     m = s.max(axis=1)                                 # row max
     finite = np.isfinite(m)
@@ -89,13 +101,16 @@ def _scores_probs(q, k, scale, causal, valid_len, rows):
     return s, p, lse
 
 
-def ref_fwd_slice(q, k, v, scale, causal, valid_len=None, rows=None, row_block=2048):
+def ref_fwd_slice(q, k, v, scale, causal, valid_len=None, rows=None, row_block=2048,
+                  block_mask=None, block=128):
     """Forward attention of one (batch, head) slice.
 
     q, k, v: float64 [N, d].  Returns (O [R, d], LSE [R]) for the query rows
     ``rows`` (all rows when None), computed in blocks of ``row_block`` rows so
     that S and P for a block fit in host memory.  Blocking over query rows does
-    not change any value: each row is computed independently.
+    not change any value: each row is computed independently.  ``block_mask``
+    (boolean [ceil(N/block), ceil(N/block)] or None) restricts the scores as
+    in allowed_mask.
     """
     n = q.shape[0]
     if valid_len is None:
@@ -105,7 +120,7 @@ def ref_fwd_slice(q, k, v, scale, causal, valid_len=None, rows=None, row_block=2
     lse = np.zeros(rows.shape[0], dtype=np.float64)
     for r0 in range(0, rows.shape[0], row_block):
         rb = rows[r0:r0 + row_block]
-        _, p, lse_b = _scores_probs(q, k, scale, causal, valid_len, rb)
+        _, p, lse_b = _scores_probs(q, k, scale, causal, valid_len, rb, block_mask, block)
         out[r0:r0 + rb.shape[0]] = p @ v              # O = P V
         lse[r0:r0 + rb.shape[0]] = lse_b
     return out, lse
@@ -129,7 +144,7 @@ def ref_fwd(q, k, v, scale, causal, seqlens=None, row_block=2048):
 
 
 def ref_bwd_slice(q, k, v, do, scale, causal, valid_len=None, q_rows=None,
-                  k_rows=None, row_block=2048):
+                  k_rows=None, row_block=2048, block_mask=None, block=128):
     """Gradients of one (batch, head) slice for the loss <dO, O>.
 
     Returns (dQ [len(q_rows), d], dK [len(k_rows), d], dV [len(k_rows), dv]).
@@ -140,6 +155,7 @@ def ref_bwd_slice(q, k, v, do, scale, causal, valid_len=None, q_rows=None,
     Chain rule through the textbook schedule:
       dV = P^T dO,  dP = dO V^T,  D_i = sum_j P_ij dP_ij,
       dS = P * (dP - D),  dQ = scale dS K,  dK = scale dS^T Q.
+    Rows without a visible key have P = 0 and contribute nothing.
     """
     n = q.shape[0]
     if valid_len is None:
@@ -155,7 +171,7 @@ def ref_bwd_slice(q, k, v, do, scale, causal, valid_len=None, q_rows=None,
     all_rows = np.arange(n)
     for r0 in range(0, n, row_block):
         rb = all_rows[r0:r0 + row_block]
-        _, p, _ = _scores_probs(q, k, scale, causal, valid_len, rb)   # [R, N]
+        _, p, _ = _scores_probs(q, k, scale, causal, valid_len, rb, block_mask, block)
         dp = do[rb] @ v.T                                             # [R, N]
         dsum = (p * dp).sum(axis=1)                                   # D_i
         ds = p * (dp - dsum[:, None])                                 # dS

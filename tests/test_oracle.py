@@ -264,3 +264,96 @@ def test_online_model_growing_max_lazy_rescale():
         o2, lse2 = tiled_fwd_slice(q, k, v, 1.0, False, 50, 16, 8, tau)
         np.testing.assert_allclose(o2, o, rtol=0, atol=1e-11)
         np.testing.assert_allclose(lse2, lse, rtol=1e-13, atol=1e-11)
+
+
+# --- block-sparse masks ------------------------------------------------------------
+
+def _blocks(n, b):
+    return [slice(i, min(i + b, n)) for i in range(0, n, b)]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_block_diagonal_mask_is_independent_blocks(causal):
+    """Query block i may only see key block i: every block is then an attention
+    problem of its own, computed here by the dense oracle on the slices."""
+    n, d, b = 10, 3, 4
+    q, k, v, do = (_rand((n, d), s) for s in (60, 61, 62, 63))
+    nb = -(-n // b)
+    mask = np.eye(nb, dtype=bool)
+    o, lse = ref_fwd_slice(q, k, v, 0.6, causal, block_mask=mask, block=b)
+    dq, dk, dv = ref_bwd_slice(q, k, v, do, 0.6, causal, block_mask=mask, block=b)
+    for sl in _blocks(n, b):
+        ro, rl = ref_fwd_slice(q[sl], k[sl], v[sl], 0.6, causal)
+        gq, gk, gv = ref_bwd_slice(q[sl], k[sl], v[sl], do[sl], 0.6, causal)
+        np.testing.assert_allclose(o[sl], ro, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(lse[sl], rl, rtol=0, atol=1e-13)
+        for a, r in ((dq, gq), (dk, gk), (dv, gv)):
+            np.testing.assert_allclose(a[sl], r, rtol=0, atol=1e-12)
+
+
+def test_off_diagonal_mask_is_not_transposed():
+    """Mask [[0, 1], [1, 0]]: query block 0 sees only key block 1 and query
+    block 1 only key block 0 (a transposed mask would give the same here only
+    if it were symmetric; [[0, 1], [0, 0]] below is not)."""
+    n, d, b = 8, 3, 4
+    q, k, v = (_rand((n, d), s) for s in (64, 65, 66))
+    o, lse = ref_fwd_slice(q, k, v, 0.7, False, block_mask=np.array([[0, 1], [0, 0]], bool), block=b)
+    ro, rl = ref_fwd_slice(q[:4], k[4:], v[4:], 0.7, False)
+    np.testing.assert_allclose(o[:4], ro, atol=1e-13)
+    np.testing.assert_allclose(lse[:4], rl, atol=1e-13)
+    assert np.all(o[4:] == 0.0) and np.all(np.isneginf(lse[4:]))
+
+
+def test_fully_masked_rows_are_zero_and_drop_out_of_key_gradients():
+    """Query block 1 may see no key block: its rows give O = 0, LSE = -inf and
+    dQ = 0, and dK, dV equal those of the other query rows alone."""
+    n, d, b = 12, 4, 4
+    q, k, v, do = (_rand((n, d), s) for s in (67, 68, 69, 70))
+    mask = np.array([[1, 0, 1], [0, 0, 0], [1, 1, 1]], bool)
+    o, lse = ref_fwd_slice(q, k, v, 0.5, False, block_mask=mask, block=b)
+    dq, dk, dv = ref_bwd_slice(q, k, v, do, 0.5, False, block_mask=mask, block=b)
+    assert np.all(o[4:8] == 0.0) and np.all(np.isneginf(lse[4:8])) and np.all(dq[4:8] == 0.0)
+    keep = np.r_[0:4, 8:12]          # query blocks 0 and 2, in blocks of 4 rows
+    gq, gk, gv = ref_bwd_slice(q[keep], k, v, do[keep], 0.5, False, valid_len=n,
+                               block_mask=mask[[0, 2]], block=b, k_rows=np.arange(n))
+    np.testing.assert_allclose(dk, gk, atol=1e-12)
+    np.testing.assert_allclose(dv, gv, atol=1e-12)
+    np.testing.assert_allclose(dq[keep], gq, atol=1e-12)
+
+
+def test_key_block_permutation_invariance():
+    """Non-causal: permuting whole key blocks (K, V rows) together with the
+    mask's columns leaves the output unchanged."""
+    n, d, b = 12, 3, 4
+    q, k, v = (_rand((n, d), s) for s in (71, 72, 73))
+    mask = np.array([[1, 0, 1], [0, 1, 1], [1, 1, 0]], bool)
+    perm = [2, 0, 1]
+    rows = np.concatenate([np.arange(p * b, p * b + b) for p in perm])
+    o1, l1 = ref_fwd_slice(q, k, v, 0.8, False, block_mask=mask, block=b)
+    o2, l2 = ref_fwd_slice(q, k[rows], v[rows], 0.8, False, block_mask=mask[:, perm], block=b)
+    np.testing.assert_allclose(o1, o2, atol=1e-13)
+    np.testing.assert_allclose(l1, l2, atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_block_sparse_backward_matches_central_differences(causal):
+    n, d, b, sc = 9, 3, 3, 0.5
+    mask = np.array([[1, 0, 1], [1, 1, 0], [0, 1, 1]], bool)
+    q, k, v, do = (_rand((n, d), s) for s in (74, 75, 76, 77))
+    dq, dk, dv = ref_bwd_slice(q, k, v, do, sc, causal, block_mask=mask, block=b)
+
+    def loss(qq, kk, vv):
+        o, _ = ref_fwd_slice(qq, kk, vv, sc, causal, block_mask=mask, block=b)
+        return float((o * do).sum())
+
+    eps = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            args = {"q": q.copy(), "k": k.copy(), "v": v.copy()}
+            args[name][idx] += eps
+            lp = loss(args["q"], args["k"], args["v"])
+            args[name][idx] -= 2 * eps
+            lm = loss(args["q"], args["k"], args["v"])
+            num[idx] = (lp - lm) / (2 * eps)
+        assert np.abs(num - g).max() / max(np.abs(num).max(), 1e-30) < 1e-6, name
