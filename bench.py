@@ -1,7 +1,7 @@
 """Throughput of exact tiled attention (forward + backward) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload mid|small|long|ragged|tiny|varlen]
+                    [--workload mid|small|long|ragged|tiny|varlen|sparse]
 
 One step is the whole hot path over one batch: fa_fwd, then the three
 backward stages (row-dot preprocess, main kernel, dQ convert), on the
@@ -16,6 +16,10 @@ counts the work of all ranks.
 
 ``--workload varlen`` times the packed variable-length path (fa_fwd_varlen +
 fa_bwd_varlen) on 8 sequences of lengths ~ U{1..4099}, H16, d128, bf16.
+
+``--workload sparse`` times block-sparse attention (fa_fwd_blocksparse +
+fa_bwd_blocksparse) on the mid workload with an 8-tile sliding window plus
+the first key tile.
 
 ``--impl reference`` times the float64 CPU oracle (test infrastructure, the
 only other place this script runs it) on bounded samples of the same
@@ -574,9 +578,200 @@ def run_ours_packed(args, w):
     return 0
 
 
+# ----------------------------------------------------------------- block-sparse
+def flops_fwd_blocksparse(mask, B, H, d, causal):
+    """Scores actually computed: 128 x 128 per allowed tile below the diagonal,
+    half a tile on the diagonal when causal (the dense causal convention)."""
+    f = 0.0
+    nt = len(mask)
+    for i in range(nt):
+        for j in range(nt):
+            if not mask[i][j] or (causal and j > i):
+                continue
+            f += 0.5 if (causal and i == j) else 1.0
+    return 4.0 * B * H * d * 128 * 128 * f
+
+
+def run_ours_blocksparse(args, spec):
+    """``--workload sparse``: one step = fa_fwd_blocksparse + fa_bwd_blocksparse
+    (its three kernels in one call) on a dense workload's inputs and a tile mask."""
+    import torch
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from exact_io_aware_47_b200 import _lib, build
+    build.build()
+    import exact_io_aware_47_b200 as fa
+    from exact_io_aware_47_b200.inputs import WORKLOADS, make_inputs, window_block_mask
+
+    w = WORKLOADS[spec["base"]]
+    B, H, N, d = w.B, w.H, w.N, w.d
+    dtype, causal, scale = w.dtypes[0], w.causal, w.scale
+    nt = (N + 127) // 128
+    mask_b = window_block_mask(nt, spec["window"], spec["n_global"])
+    mask = mask_b.to(torch.uint8).to(dev).contiguous()
+    inp = make_inputs(w.name, dtype=dtype, seed=rank, device=dev)
+    q, k, v, do = inp["q"], inp["k"], inp["v"], inp["do"]
+    o, lse = torch.empty_like(q), torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_bytes = fa.workspace_bytes(B, H, N, d)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    dt_code = _lib.FA_BF16 if dtype == torch.bfloat16 else _lib.FA_FP16
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        _lib.check("fa_fwd_blocksparse", _lib.fa_fwd_blocksparse(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+            mask.data_ptr(), B, H, N, d, scale, int(causal), None, dt_code, sh))
+        if ev is not None:
+            ev[1].record(stream)
+        _lib.check("fa_bwd_blocksparse", _lib.fa_bwd_blocksparse(
+            q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
+            dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws_bytes, mask.data_ptr(),
+            B, H, N, d, scale, int(causal), None, dt_code, sh))
+        if ev is not None:
+            ev[2].record(stream)
+
+    warmup = max(3, args.warmup)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    st, word = _lib.fa_device_status(sh)
+    if st != 0:
+        raise RuntimeError(f"device status {st} ({word:#x}) after warm-up")
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    if not args.no_clocks:
+        clocks.start()
+        time.sleep(0.3)
+    dist_barrier(world)
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(K):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    dist_barrier(world)
+    clk = None if args.no_clocks else clocks.stop()
+    st, word = _lib.fa_device_status(sh)
+    if st != 0:
+        raise RuntimeError(f"device status {st} ({word:#x}) after timing")
+    total_ms = dist_max(t0.elapsed_time(t1), world)
+    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
+    bwd_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / K
+    mask_list = mask_b.tolist()
+    f_fwd = flops_fwd_blocksparse(mask_list, B, H, d, causal)
+    f_bwd = 2.5 * f_fwd
+    step_flops = f_fwd + f_bwd
+    value = world * step_flops * K / (total_ms / 1e3) / 1e12
+    peaks, peak_src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    fwd_tf = f_fwd / (fwd_ms / 1e3) / 1e12
+    bwd_tf = f_bwd / (bwd_ms / 1e3) / 1e12
+    allowed = sum(1 for i in range(nt) for j in range(nt) if mask_list[i][j] and not (causal and j > i))
+
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
+        ho, hdq, hdk, hdv = (torch.empty(q.shape, dtype=dtype, pin_memory=True) for _ in range(4))
+        hlse = torch.empty((B, H, N), dtype=torch.float32, pin_memory=True)
+        hmask = mask.cpu().pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo, hmask))
+        d2h = sum(t.numel() * t.element_size() for t in (ho, hlse, hdq, hdk, hdv))
+
+        def e2e_step():
+            for src, dst in ((hq, q), (hk, k), (hv, v), (hdo, do), (hmask, mask)):
+                dst.copy_(src, non_blocking=True)
+            fa.forward_blocksparse(q, k, v, mask, scale=scale, causal=causal, out=o, lse=lse)
+            fa.backward_blocksparse(q, k, v, o, lse, do, mask, scale=scale, causal=causal,
+                                    workspace=ws, dq=dq, dk=dk, dv=dv)
+            for src, dst in ((o, ho), (lse, hlse), (dq, hdq), (dk, hdk), (dv, hdv)):
+                dst.copy_(src, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        ke = max(3, min(K, 10))
+        dist_barrier(world)
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(ke):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        dist_barrier(world)
+        e_ms = dist_max(a.elapsed_time(b), world)
+        e2e = {"value": world * step_flops * ke / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / ke}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from threadpoolctl import threadpool_info
+        from oracle import ref_bwd_slice, ref_fwd_slice
+        import numpy as np
+        mnp = np.array(mask_list, dtype=bool)
+        dt, fl, n_done = 0.0, 0.0, 0
+        for b in range(B):  # whole (batch, head) slices until ~10 s of CPU work
+            for h in range(H):
+                qq, kk, vv, dd = (t[b, h].double().cpu().numpy() for t in (q, k, v, do))
+                tc = time.perf_counter()
+                ref_fwd_slice(qq, kk, vv, scale, causal, block_mask=mnp)
+                ref_bwd_slice(qq, kk, vv, dd, scale, causal, block_mask=mnp)
+                dt += time.perf_counter() - tc
+                fl += 3.5 * flops_fwd_blocksparse(mask_list, 1, 1, d, causal)
+                n_done += 1
+                if dt >= 10.0:
+                    break
+            if dt >= 10.0:
+                break
+        thr = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+               "sample": f"float64 oracle forward+backward (dense S, block mask applied) of "
+                         f"{n_done} whole (batch, head) slices ({dt:.1f} s); FLOPs counted "
+                         f"over the allowed tiles only"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if dtype == torch.bfloat16 else "f16", "data": "synthetic",
+        "config": {"workload": spec["description"], "B": B, "H": H, "N": N, "d": d,
+                   "causal": causal, "tiles_computed": allowed, "tiles_total": nt * nt,
+                   "step": "fa_fwd_blocksparse + fa_bwd_blocksparse",
+                   "flops_per_step": step_flops, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (4 x 128 MiB per step), no flush"},
+        "fwd": {"ms": fwd_ms, "tflops": fwd_tf, "frac": fwd_tf / peak},
+        "bwd": {"ms": bwd_ms, "tflops": bwd_tf, "frac": bwd_tf / peak},
+        "roofline": {"bound": "tensor", "kernel": "fa_bwd_blocksparse (preprocess + main + postprocess)",
+                     "achieved": bwd_tf, "peak": peak, "unit": "TFLOP/s", "frac": bwd_tf / peak,
+                     "traffic": None, "peak_source": f"{peak_src} bf16 dense (burst)",
+                     "flops_per_launch": f_bwd},
+        "roofline_fwd": {"bound": "tensor", "kernel": "fa_fwd_kernel (fa_fwd_blocksparse)",
+                         "achieved": fwd_tf, "peak": peak, "unit": "TFLOP/s",
+                         "frac": fwd_tf / peak, "traffic": None,
+                         "peak_source": f"{peak_src} bf16 dense (burst)", "flops_per_launch": f_fwd},
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 4 * K, "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse()
-    from exact_io_aware_47_b200.inputs import PACKED_WORKLOADS, WORKLOADS
+    from exact_io_aware_47_b200.inputs import BLOCKSPARSE_WORKLOADS, PACKED_WORKLOADS, WORKLOADS
+    if args.workload in BLOCKSPARSE_WORKLOADS:
+        if args.impl == "reference":
+            raise SystemExit("--impl reference times the dense workloads")
+        return run_ours_blocksparse(args, BLOCKSPARSE_WORKLOADS[args.workload])
     if args.workload in PACKED_WORKLOADS:
         if args.impl == "reference":
             raise SystemExit("--impl reference times the fixed-length workloads")

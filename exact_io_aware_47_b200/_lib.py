@@ -39,6 +39,10 @@ SIGNATURES = {
     "fa_bwd_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
                             _I, _I, _I, _I, _F, _I, _VP, _I, _VP]),
     "fa_bwd_noalloc_max_bytes": (_SZ, []),
+    "fa_fwd_blocksparse": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _VP, _I,
+                                _VP]),
+    "fa_bwd_blocksparse": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP,
+                                _I, _I, _I, _I, _F, _I, _VP, _I, _VP]),
     "fa_fwd_varlen": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _I, _VP]),
     "fa_bwd_varlen": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP,
                            _I, _I, _I, _I, _I, _F, _I, _I, _VP]),
@@ -118,6 +122,19 @@ def fa_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal,
                    stream):
     return load().fa_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal,
                                  seqlens, dtype, stream)
+
+
+def fa_fwd_blocksparse(q, k, v, o, lse, block_mask, B, H, N, d, scale, causal, seqlens, dtype,
+                       stream):
+    return load().fa_fwd_blocksparse(q, k, v, o, lse, block_mask, B, H, N, d, scale, causal,
+                                     seqlens, dtype, stream)
+
+
+def fa_bwd_blocksparse(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, block_mask,
+                       B, H, N, d, scale, causal, seqlens, dtype, stream):
+    return load().fa_bwd_blocksparse(q, k, v, o, dout, lse, dq, dk, dv, workspace,
+                                     workspace_bytes, block_mask, B, H, N, d, scale, causal,
+                                     seqlens, dtype, stream)
 
 
 def fa_fwd_varlen(q, k, v, o, lse, cu_seqlens, B, H, T, max_seqlen, d, scale, causal, dtype,

@@ -1,7 +1,9 @@
 """torch-facing calls of the CUDA library: allocate outputs, pass pointers.
 
-``forward`` and ``backward`` ([B, H, N, d]) and ``forward_varlen`` /
-``backward_varlen`` (packed [H, T, d] with cu_seqlens) validate tensor
+``forward`` and ``backward`` ([B, H, N, d]), ``forward_blocksparse`` /
+``backward_blocksparse`` (the same with a 128 x 128 tile mask) and
+``forward_varlen`` / ``backward_varlen`` (packed [H, T, d] with cu_seqlens)
+validate tensor
 properties that ctypes cannot see (device, dtype, contiguity, shapes),
 allocate the outputs and the backward workspace with torch, and call the
 library on the current CUDA stream.  No arithmetic of the method happens
@@ -102,6 +104,68 @@ def backward(q, k, v, o, lse, do, scale=None, causal=False, seqlens=None, worksp
                          B, H, N, d, scale, int(bool(causal)), sl_ptr, _DTYPES[q.dtype],
                          _stream_handle(dev))
     _lib.check("fa_bwd", st)
+    return dq, dk, dv
+
+
+def _block_mask_arg(block_mask, N, device):
+    nt = (N + 127) // 128
+    bm = block_mask
+    if not (torch.is_tensor(bm) and bm.is_cuda and bm.dtype == torch.uint8 and bm.is_contiguous()):
+        bm = torch.as_tensor(block_mask).to(device=device, dtype=torch.uint8).contiguous()
+    if tuple(bm.shape) != (nt, nt):
+        raise ValueError(f"block_mask must be [{nt}, {nt}] (128 x 128 tiles)")
+    return bm
+
+
+def forward_blocksparse(q, k, v, block_mask, scale=None, causal=False, seqlens=None, out=None,
+                        lse=None):
+    """O, LSE of block-sparse attention ([B, H, N, d]; block_mask [nt, nt] over
+    128 x 128 score tiles, shared by all (batch, head) slices)."""
+    B, H, N, d = q.shape
+    dev = q.device
+    if q.dtype not in _DTYPES:
+        raise ValueError("dtype must be bfloat16 or float16")
+    _check_inputs({"q": q, "k": k, "v": v}, (B, H, N, d), q.dtype, dev)
+    bm = _block_mask_arg(block_mask, N, dev)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev) if lse is None else lse
+    _check_inputs({"out": out}, (B, H, N, d), q.dtype, dev)
+    _check_inputs({"lse": lse}, (B, H, N), torch.float32, dev)
+    sl, sl_ptr = _seqlens_arg(seqlens, B, dev)
+    with torch.cuda.device(dev):
+        st = _lib.fa_fwd_blocksparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                     lse.data_ptr(), bm.data_ptr(), B, H, N, d, scale,
+                                     int(bool(causal)), sl_ptr, _DTYPES[q.dtype],
+                                     _stream_handle(dev))
+    _lib.check("fa_fwd_blocksparse", st)
+    return out, lse
+
+
+def backward_blocksparse(q, k, v, o, lse, do, block_mask, scale=None, causal=False, seqlens=None,
+                         workspace=None, dq=None, dk=None, dv=None):
+    """dQ, dK, dV of block-sparse attention for the loss <dO, O>."""
+    B, H, N, d = q.shape
+    dev = q.device
+    _check_inputs({"q": q, "k": k, "v": v, "o": o, "do": do}, (B, H, N, d), q.dtype, dev)
+    _check_inputs({"lse": lse}, (B, H, N), torch.float32, dev)
+    bm = _block_mask_arg(block_mask, N, dev)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check_inputs({"dq": dq, "dk": dk, "dv": dv}, (B, H, N, d), q.dtype, dev)
+    if workspace is None:
+        workspace = torch.empty(workspace_bytes(B, H, N, d), dtype=torch.uint8, device=dev)
+    sl, sl_ptr = _seqlens_arg(seqlens, B, dev)
+    with torch.cuda.device(dev):
+        st = _lib.fa_bwd_blocksparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                     do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                     dv.data_ptr(), workspace.data_ptr(),
+                                     workspace.numel() * workspace.element_size(), bm.data_ptr(),
+                                     B, H, N, d, scale, int(bool(causal)), sl_ptr,
+                                     _DTYPES[q.dtype], _stream_handle(dev))
+    _lib.check("fa_bwd_blocksparse", st)
     return dq, dk, dv
 
 

@@ -123,7 +123,8 @@ namespace {
 // [H, T = N, d]); arguments already checked except the pointers' alignment.
 int fwd_core(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
              int N, int d, float scale, int causal, const int32_t* seqlens,
-             const int32_t* cu_seqlens, int max_seqlen, int dtype, void* stream) {
+             const int32_t* cu_seqlens, int max_seqlen, int dtype, void* stream,
+             const uint8_t* block_mask = nullptr) {
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
       (seqlens && (reinterpret_cast<uintptr_t>(seqlens) & 3u)) ||
       (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)))
@@ -145,6 +146,7 @@ int fwd_core(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.seqlens = seqlens;
   p.cu_seqlens = cu_seqlens;
   p.max_seqlen = cu_seqlens ? max_seqlen : N;
+  p.block_mask = block_mask;
   p.B = B;
   p.H = H;
   p.N = N;
@@ -181,6 +183,17 @@ extern "C" int fa_fwd(const void* q, const void* k, const void* v, void* o, floa
   const int st = check_common(B, H, N, d, scale, dtype);
   if (st != FA_OK) return st;
   return fwd_core(q, k, v, o, lse, B, H, N, d, scale, causal, seqlens, nullptr, 0, dtype, stream);
+}
+
+extern "C" int fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o,
+                                  float* lse, const uint8_t* block_mask, int B, int H, int N,
+                                  int d, float scale, int causal, const int32_t* seqlens,
+                                  int dtype, void* stream) {
+  if (!q || !k || !v || !o || !lse || !block_mask) return FA_ERR_INVALID_ARG;
+  const int st = check_common(B, H, N, d, scale, dtype);
+  if (st != FA_OK) return st;
+  return fwd_core(q, k, v, o, lse, B, H, N, d, scale, causal, seqlens, nullptr, 0, dtype, stream,
+                  block_mask);
 }
 
 extern "C" int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -322,6 +335,46 @@ extern "C" int fa_bwd(const void* q, const void* k, const void* v, const void* o
                    causal, seqlens, dtype, stream);
   if (st != FA_OK) return st;
   return fa_bwd_postprocess(workspace, workspace_bytes, dq, B, H, N, d, scale, dtype, stream);
+}
+
+extern "C" int fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o,
+                                  const void* dout, const float* lse, void* dq, void* dk,
+                                  void* dv, void* workspace, size_t workspace_bytes,
+                                  const uint8_t* block_mask, int B, int H, int N, int d,
+                                  float scale, int causal, const int32_t* seqlens, int dtype,
+                                  void* stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !block_mask)
+    return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_ALIGNMENT;
+  BwdParams p;
+  DeviceInfo di;
+  int st = bwd_common(workspace, workspace_bytes, B, H, N, d, scale, dtype, seqlens, &p, &di);
+  if (st != FA_OK) return st;
+  CUtensorMap tq, tk, tv, tdo, tdq;
+  const int BH = B * H;
+  if (make_map(&tq, q, BH, N, d, dtype) != FA_OK || make_map(&tk, k, BH, N, d, dtype) != FA_OK ||
+      make_map(&tv, v, BH, N, d, dtype) != FA_OK || make_map(&tdo, dout, BH, N, d, dtype) != FA_OK ||
+      make_map_acc(&tdq, p.dq_acc, BH, N, d) != FA_OK)
+    return FA_ERR_CUDA;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.o = o;
+  p.dout = dout;
+  p.lse = lse;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.causal = causal ? 1 : 0;
+  p.block_mask = block_mask;
+  const bool bf16 = dtype == FA_BF16;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (launch_bwd_pre(d, bf16, p, di.num_sms, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (launch_bwd_main(d, bf16, tq, tk, tv, tdo, tdq, p, di.num_sms, s) != cudaSuccess)
+    return FA_ERR_CUDA;
+  return launch_bwd_post(d, bf16, p, di.num_sms, s) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 extern "C" int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o,

@@ -73,6 +73,7 @@ struct BwdLayout {
 
 struct BwdUnit {
   int bh, j, L, i0, ni;
+  int nq;             // query tiles of the slice that are computed
   int z, row0, rows;  // slice placement (SliceInfo)
   bool skip;          // packed key tile past its sequence: no role does anything
 };
@@ -91,7 +92,10 @@ static_assert(2 * kBwdSoftmaxRegs + kBwdDqRegs + kBwdOtherRegs <= 4 * kBwdLaunch
 
 // Unit (bh, key tile j).  The work order hands out key tiles mirrored
 // (j = n-1-idx), so the long tile of a causal super-unit (small j) runs first.
-template <bool PACKED>
+// The unit visits the ni query tiles i in [i0, nq) that see key tile j (with
+// SPARSE, those the block mask allows), in ascending order; every role walks
+// the same list with bwd_next_i.
+template <bool PACKED, bool SPARSE>
 __device__ __forceinline__ BwdUnit bwd_decode(int bh, int idx, const BwdParams& p) {
   BwdUnit w;
   w.bh = bh;
@@ -102,14 +106,29 @@ __device__ __forceinline__ BwdUnit bwd_decode(int bh, int idx, const BwdParams& 
   w.rows = si.rows;
   w.L = si.L;
   const int nq = min((si.rows + kBlockM - 1) / kBlockM, p.n_ktiles);  // query tiles computed
+  w.nq = nq;
   w.i0 = p.causal ? w.j : 0;
   // a key tile past L only gets zeros (fixed length) or nothing (packed)
   w.ni = (w.j * kBlockN < si.L) ? max(nq - w.i0, 0) : 0;
+  if constexpr (SPARSE) {
+    int n = 0;
+    for (int i = w.i0; i < w.i0 + w.ni; ++i) n += tile_allowed(p.block_mask, p.n_ktiles, i, w.j);
+    w.ni = n;  // a key tile no query tile sees still writes zero dK, dV
+  }
   w.skip = PACKED && w.ni == 0;
   return w;
 }
 
-template <int D, bool BF16, bool PACKED>
+// The next query tile >= i of the unit's list.
+template <bool SPARSE>
+__device__ __forceinline__ int bwd_next_i(const BwdParams& p, const BwdUnit& w, int i) {
+  if constexpr (SPARSE) {
+    while (i < w.nq && !tile_allowed(p.block_mask, p.n_ktiles, i, w.j)) ++i;
+  }
+  return i;
+}
+
+template <int D, bool BF16, bool PACKED, bool SPARSE>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdo,
@@ -201,7 +220,7 @@ __global__ void __launch_bounds__(512, 1)
         WorkItem wi;
         if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
         if (wi.idx < 0) continue;
-        const BwdUnit w = bwd_decode<PACKED>(wi.bh, wi.idx, p);
+        const BwdUnit w = bwd_decode<PACKED, SPARSE>(wi.bh, wi.idx, p);
         if (w.skip) continue;
         ok = mbar_wait(kv_empty, (nunit & 1) ^ 1, abort_flag, 20);
         if (!ok) break;
@@ -214,8 +233,9 @@ __global__ void __launch_bounds__(512, 1)
                       w.z);
         }
         ++nunit;
+        int i = w.i0 - 1;  // walks the unit's query tiles
         for (int idx = 0; idx < w.ni && ok; ++idx) {
-          const int i = w.i0 + idx;
+          i = bwd_next_i<SPARSE>(p, w, i + 1);
           for (int t = 0; t < 2 && ok; ++t) {  // Q_i, then dO_i
             const int slot = t == 0 ? (lt & 1) : 2;
             const int use = t == 0 ? (lt >> 1) : lt;  // earlier loads into this slot
@@ -250,11 +270,12 @@ __global__ void __launch_bounds__(512, 1)
       WorkItem wi;
       if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
       if (wi.idx < 0) continue;
-      const BwdUnit w = bwd_decode<PACKED>(wi.bh, wi.idx, p);
+      const BwdUnit w = bwd_decode<PACKED, SPARSE>(wi.bh, wi.idx, p);
       if (w.skip) continue;
       const size_t base = static_cast<size_t>(w.z) * p.N + w.row0;
+      int i = w.i0 - 1;  // walks the unit's query tiles
       for (int idx = 0; idx < w.ni && ok; ++idx) {
-        const int i = w.i0 + idx;
+        i = bwd_next_i<SPARSE>(p, w, i + 1);
         const int st = seq & 1;
         ok = mbar_wait_warp(&ld_empty[st], ((seq >> 1) & 1) ^ 1, abort_flag, 22);
         if (!ok) break;
@@ -299,7 +320,7 @@ __global__ void __launch_bounds__(512, 1)
         WorkItem wi;
         if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
         if (wi.idx < 0) continue;
-        const BwdUnit w = bwd_decode<PACKED>(wi.bh, wi.idx, p);
+        const BwdUnit w = bwd_decode<PACKED, SPARSE>(wi.bh, wi.idx, p);
         if (w.skip) continue;
         ok = mbar_wait(kv_full, nunit & 1, abort_flag, 23);
         if (!ok) break;
@@ -430,7 +451,7 @@ __global__ void __launch_bounds__(512, 1)
       WorkItem wi;
       if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
       if (wi.idx < 0) continue;
-      const BwdUnit w = bwd_decode<PACKED>(wi.bh, wi.idx, p);
+      const BwdUnit w = bwd_decode<PACKED, SPARSE>(wi.bh, wi.idx, p);
       if (w.skip) continue;
       if (w.ni > 0) {
         ok = seen(s_full, it & 1);
@@ -471,11 +492,12 @@ __global__ void __launch_bounds__(512, 1)
       WorkItem wi;
       if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
       if (wi.idx < 0) continue;
-      const BwdUnit w = bwd_decode<PACKED>(wi.bh, wi.idx, p);
+      const BwdUnit w = bwd_decode<PACKED, SPARSE>(wi.bh, wi.idx, p);
       if (w.skip) continue;
       const bool key_ok = w.j * kBlockN + r < w.L;
+      int i = w.i0 - 1;  // walks the unit's query tiles
       for (int idx = 0; idx < w.ni && ok; ++idx) {
-        const int i = w.i0 + idx;
+        i = bwd_next_i<SPARSE>(p, w, i + 1);
         const int st = it & 1;  // LSE/D staging advances with the iteration count
         // ---- phase 1: P^T = 2^(c S^T - LSE_i log2 e) from S^T, back to TMEM
         ok = mbar_wait_warp(&ld_full[st], (it >> 1) & 1, abort_flag, 28) &&
@@ -581,11 +603,12 @@ __global__ void __launch_bounds__(512, 1)
       WorkItem wi;
       if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
       if (wi.idx < 0) continue;
-      const BwdUnit w = bwd_decode<PACKED>(wi.bh, wi.idx, p);
+      const BwdUnit w = bwd_decode<PACKED, SPARSE>(wi.bh, wi.idx, p);
       if (w.skip) continue;
       const size_t base = static_cast<size_t>(w.z) * p.N + w.row0;
+      int i = w.i0 - 1;  // walks the unit's query tiles
       for (int idx = 0; idx < w.ni && ok; ++idx) {
-        const int i = w.i0 + idx;
+        i = bwd_next_i<SPARSE>(p, w, i + 1);
         ok = mbar_wait_warp(dq_full, it & 1, abort_flag, 32);
         if (!ok) break;
         tc_fence_after();
@@ -770,13 +793,13 @@ cudaError_t launch_bwd_pre(int d, bool bf16, const BwdParams& p, int num_sms,
   return cudaGetLastError();
 }
 
-template <int D, bool BF16, bool PACKED>
+template <int D, bool BF16, bool PACKED, bool SPARSE>
 static cudaError_t launch_bwd_main_t(const CUtensorMap& tmq, const CUtensorMap& tmk,
                                      const CUtensorMap& tmv, const CUtensorMap& tmdo,
                                      const CUtensorMap& tmdq, const BwdParams& p, int num_sms,
                                      cudaStream_t stream) {
   using Lay = BwdLayout<D>;
-  auto kern = fa_bwd_kernel<D, BF16, PACKED>;
+  auto kern = fa_bwd_kernel<D, BF16, PACKED, SPARSE>;
   cudaFuncAttributes attr;
   cudaError_t e = cudaFuncGetAttributes(&attr, kern);
   if (e != cudaSuccess) return e;
@@ -793,15 +816,16 @@ cudaError_t launch_bwd_main(int d, bool bf16, const CUtensorMap& tmq, const CUte
                             const CUtensorMap& tmv, const CUtensorMap& tmdo,
                             const CUtensorMap& tmdq, const BwdParams& p, int num_sms,
                             cudaStream_t stream) {
-  const bool packed = p.cu_seqlens != nullptr;
-#define FA_BWD_LAUNCH(DD, BB, PP) \
-  launch_bwd_main_t<DD, BB, PP>(tmq, tmk, tmv, tmdo, tmdq, p, num_sms, stream)
-  if (d == 128) {
-    if (packed) return bf16 ? FA_BWD_LAUNCH(128, true, true) : FA_BWD_LAUNCH(128, false, true);
-    return bf16 ? FA_BWD_LAUNCH(128, true, false) : FA_BWD_LAUNCH(128, false, false);
-  }
-  if (packed) return bf16 ? FA_BWD_LAUNCH(64, true, true) : FA_BWD_LAUNCH(64, false, true);
-  return bf16 ? FA_BWD_LAUNCH(64, true, false) : FA_BWD_LAUNCH(64, false, false);
+  const int mode = p.cu_seqlens != nullptr ? 1 : (p.block_mask != nullptr ? 2 : 0);
+#define FA_BWD_LAUNCH(DD, BB, PP, SS) \
+  launch_bwd_main_t<DD, BB, PP, SS>(tmq, tmk, tmv, tmdo, tmdq, p, num_sms, stream)
+#define FA_BWD_MODES(DD, BB)                                       \
+  (mode == 1 ? FA_BWD_LAUNCH(DD, BB, true, false)                  \
+             : mode == 2 ? FA_BWD_LAUNCH(DD, BB, false, true)      \
+                         : FA_BWD_LAUNCH(DD, BB, false, false))
+  if (d == 128) return bf16 ? FA_BWD_MODES(128, true) : FA_BWD_MODES(128, false);
+  return bf16 ? FA_BWD_MODES(64, true) : FA_BWD_MODES(64, false);
+#undef FA_BWD_MODES
 #undef FA_BWD_LAUNCH
 }
 

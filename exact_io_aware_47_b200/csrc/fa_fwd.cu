@@ -58,12 +58,33 @@ static_assert(2 * kFwdSoftmaxRegs + kFwdOtherRegs <= 3 * kFwdLaunchRegs, "regist
 
 struct FwdUnit {
   int bh, qt0, L, jend0, jend1;
-  int z, row0, rows;  // slice placement (SliceInfo)
+  int z, row0, rows;    // slice placement (SliceInfo)
+  int jlast0, jlast1;   // last key tile each query tile computes, -1 for none
 };
 
 // Unit (bh, pair): query tiles 2 pair and 2 pair + 1 of slice bh.  A query
-// tile that starts at or past the slice's computed rows has no work.
-template <bool PACKED>
+// tile that starts at or past the slice's computed rows has no work.  Query
+// tile t computes the key tiles j < jend_t (causal / key-length limit) that
+// the block mask allows (SPARSE); the unit streams the union of the two
+// lists in ascending order.
+template <bool SPARSE>
+__device__ __forceinline__ bool fwd_need(const FwdParams& p, const FwdUnit& w, int t, int j) {
+  if (j >= (t == 0 ? w.jend0 : w.jend1)) return false;
+  if constexpr (SPARSE) return tile_allowed(p.block_mask, p.n_qtiles, w.qt0 + t, j);
+  return true;
+}
+
+// Smallest key tile >= j that either query tile computes; max(jend) if none.
+template <bool SPARSE>
+__device__ __forceinline__ int fwd_next(const FwdParams& p, const FwdUnit& w, int j) {
+  const int jmax = max(w.jend0, w.jend1);
+  if constexpr (SPARSE) {
+    while (j < jmax && !fwd_need<SPARSE>(p, w, 0, j) && !fwd_need<SPARSE>(p, w, 1, j)) ++j;
+  }
+  return j < jmax ? j : jmax;
+}
+
+template <bool PACKED, bool SPARSE>
 __device__ __forceinline__ FwdUnit fwd_decode(int bh, int pair, const FwdParams& p) {
   FwdUnit w;
   w.bh = bh;
@@ -84,10 +105,18 @@ __device__ __forceinline__ FwdUnit fwd_decode(int bh, int pair, const FwdParams&
   }
   w.jend0 = je[0];
   w.jend1 = je[1];
+  int jl[2] = {je[0] - 1, je[1] - 1};
+  if constexpr (SPARSE) {
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+      while (jl[t] >= 0 && !tile_allowed(p.block_mask, p.n_qtiles, w.qt0 + t, jl[t])) --jl[t];
+  }
+  w.jlast0 = jl[0];
+  w.jlast1 = jl[1];
   return w;
 }
 
-template <int D, bool BF16, bool PACKED>
+template <int D, bool BF16, bool PACKED, bool SPARSE>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const FwdParams p) {
@@ -153,10 +182,11 @@ __global__ void __launch_bounds__(384, 1)
         WorkItem wi;
         if (!work_item(k, p.n_pairs, p.B * p.H, wi)) break;
         if (wi.idx < 0) continue;
-        const FwdUnit w = fwd_decode<PACKED>(wi.bh, wi.idx, p);
+        const FwdUnit w = fwd_decode<PACKED, SPARSE>(wi.bh, wi.idx, p);
         const int je[2] = {w.jend0, w.jend1};
+        const int jl[2] = {w.jlast0, w.jlast1};
         for (int t = 0; t < 2 && ok; ++t) {
-          if (je[t] == 0) continue;
+          if (jl[t] < 0) continue;
           ok = mbar_wait(&q_empty[t], (qload[t] & 1) ^ 1, abort_flag, 1);
           if (!ok) break;
           mbar_arrive_expect_tx(&q_full[t], Lay::kTileBytes);
@@ -167,7 +197,7 @@ __global__ void __launch_bounds__(384, 1)
           ++qload[t];
         }
         const int jmax = max(je[0], je[1]);
-        for (int j = 0; j < jmax && ok; ++j) {
+        for (int j = fwd_next<SPARSE>(p, w, 0); j < jmax && ok; j = fwd_next<SPARSE>(p, w, j + 1)) {
           for (int kv = 0; kv < 2; ++kv) {
             const int slot = kv_seq % kSlots;
             const int round = kv_seq / kSlots;
@@ -228,12 +258,15 @@ __global__ void __launch_bounds__(384, 1)
         WorkItem wi;
         if (!work_item(k, p.n_pairs, p.B * p.H, wi)) break;
         if (wi.idx < 0) continue;
-        const FwdUnit w = fwd_decode<PACKED>(wi.bh, wi.idx, p);
+        const FwdUnit w = fwd_decode<PACKED, SPARSE>(wi.bh, wi.idx, p);
         const int je[2] = {w.jend0, w.jend1};
+        const int jl[2] = {w.jlast0, w.jlast1};
         const int jmax = max(je[0], je[1]);
-        if (PACKED && jmax == 0) continue;  // both tiles past a packed sequence: nothing loaded
+        const int j0 = fwd_next<SPARSE>(p, w, 0);
+        // nothing loaded: both tiles past a packed sequence, or masked out
+        if ((PACKED || SPARSE) && j0 >= jmax) continue;
         for (int t = 0; t < 2 && ok; ++t) {
-          if (je[t] == 0) continue;
+          if (jl[t] < 0) continue;
           ok = mbar_wait(&q_full[t], qload[t] & 1, abort_flag, 3);
           ++qload[t];
         }
@@ -246,33 +279,36 @@ __global__ void __launch_bounds__(384, 1)
           if (!ok) break;
           tc_fence_after();
           for (int t = 0; t < 2; ++t) {
-            if (je[t] == 0) continue;
+            if (!fwd_need<SPARSE>(p, w, t, j0)) continue;
             issue_s(t, slot);
             umma_commit(&s_full[t]);
-            if (je[t] == 1) umma_commit(&q_empty[t]);
+            if (j0 == jl[t]) umma_commit(&q_empty[t]);
           }
           umma_commit(&kv_empty[slot]);
           ++kv_seq;
         }
-        for (int j = 0; j < jmax && ok; ++j) {
+        int npv[2] = {0, 0};  // P.V issued per query tile in this unit
+        for (int j = j0; j < jmax && ok;) {
           const int vslot = kv_seq % kSlots;
           ok = mbar_wait(&kv_full[vslot], (kv_seq / kSlots) & 1, abort_flag, 5);
           if (!ok) break;
           tc_fence_after();
           ++kv_seq;
+          const int jn = fwd_next<SPARSE>(p, w, j + 1);  // next streamed key tile
           const int kslot = kv_seq % kSlots;
           bool k_ready = false;
           for (int t = 0; t < 2 && ok; ++t) {
-            if (j < je[t]) {
+            if (fwd_need<SPARSE>(p, w, t, j)) {
               ok = mbar_wait(&p_full[t], pcnt[t] & 1, abort_flag, 6);
               if (!ok) break;
               FA_TRACE_AT(pcnt[t], t);
               ++pcnt[t];
               tc_fence_after();
-              issue_pv(t, vslot, j > 0);
-              if (j == je[t] - 1) umma_commit(&o_full[t]);
+              issue_pv(t, vslot, npv[t] > 0);
+              ++npv[t];
+              if (j == jl[t]) umma_commit(&o_full[t]);
             }
-            if (j + 1 < je[t]) {
+            if (jn < jmax && fwd_need<SPARSE>(p, w, t, jn)) {
               if (!k_ready) {
                 ok = mbar_wait(&kv_full[kslot], (kv_seq / kSlots) & 1, abort_flag, 7);
                 if (!ok) break;
@@ -281,15 +317,16 @@ __global__ void __launch_bounds__(384, 1)
               }
               issue_s(t, kslot);
               umma_commit(&s_full[t]);
-              if (j + 1 == je[t] - 1) umma_commit(&q_empty[t]);
+              if (jn == jl[t]) umma_commit(&q_empty[t]);
             }
           }
           if (!ok) break;
           umma_commit(&kv_empty[vslot]);
-          if (j + 1 < jmax) {
+          if (jn < jmax) {
             umma_commit(&kv_empty[kslot]);
             ++kv_seq;
           }
+          j = jn;
         }
       }
       // every MMA issued must be complete before TMEM is released
@@ -314,7 +351,7 @@ __global__ void __launch_bounds__(384, 1)
       WorkItem wi;
       if (!work_item(k, p.n_pairs, p.B * p.H, wi)) break;
       if (wi.idx < 0) continue;
-      const FwdUnit w = fwd_decode<PACKED>(wi.bh, wi.idx, p);
+      const FwdUnit w = fwd_decode<PACKED, SPARSE>(wi.bh, wi.idx, p);
       const int jend = t == 0 ? w.jend0 : w.jend1;
       if (jend == 0) continue;
       const int qt = w.qt0 + t;
@@ -323,9 +360,22 @@ __global__ void __launch_bounds__(384, 1)
         const int raw = p.seqlens[w.bh / p.H];
         if (raw < 1 || raw > p.N) record_error(kErrDeviceSeqlen, 0);
       }
+      if (SPARSE && (t == 0 ? w.jlast0 : w.jlast1) < 0) {
+        // the block mask leaves these rows no key: O = 0, LSE = -inf
+        if (row < w.rows) {
+          const size_t idx = static_cast<size_t>(w.z) * p.N + w.row0 + row;
+          uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) + idx * (D * 2);
+#pragma unroll
+          for (int c16 = 0; c16 < D * 2 / 16; ++c16) st_global_v4(orow + c16 * 16, 0u, 0u, 0u, 0u);
+          p.lse[idx] = -INFINITY;
+        }
+        continue;
+      }
       float m = -INFINITY;  // running max, log2 units
       float l = 0.f;        // running sum of unnormalised probabilities
+      int jj = 0;           // key tiles processed so far
       for (int j = 0; j < jend; ++j) {
+        if (!fwd_need<SPARSE>(p, w, t, j)) continue;
         ok = mbar_wait_warp(&s_full[t], scnt & 1, abort_flag, 8);
         if (!ok) break;
         if (r == 0) FA_TRACE_AT(scnt, 2 + 2 * t);
@@ -387,10 +437,10 @@ __global__ void __launch_bounds__(384, 1)
           l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
         }
         tmem_st64(tS, pk);
-        if (j > 0 && __any_sync(0xffffffffu, moved)) {
-          // O_t holds the sum up to tile j-1 (its MMA completed before S_t(j)
-          // was committed) and PV_t(j) waits for p_full: rescale it now; rows
-          // that did not move multiply by 1.
+        if (jj > 0 && __any_sync(0xffffffffu, moved)) {
+          // O_t holds the sum up to the previous key tile (its MMA completed
+          // before S_t(j) was committed) and PV_t(j) waits for p_full:
+          // rescale it now; rows that did not move multiply by 1.
           uint32_t ro[32];
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc) {
@@ -404,6 +454,7 @@ __global__ void __launch_bounds__(384, 1)
         tc_fence_before();
         mbar_arrive(&p_full[t]);
         if (r == 0) FA_TRACE_AT(scnt - 1, 3 + 2 * t);
+        ++jj;
       }
       if (!ok) break;
       // epilogue: O / l -> 16-bit, LSE
@@ -442,12 +493,12 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
-template <int D, bool BF16, bool PACKED>
+template <int D, bool BF16, bool PACKED, bool SPARSE>
 static cudaError_t launch_fwd_t(const CUtensorMap& tmq, const CUtensorMap& tmk,
                                 const CUtensorMap& tmv, const FwdParams& p, int num_sms,
                                 cudaStream_t stream) {
   using Lay = FwdLayout<D>;
-  auto kern = fa_fwd_kernel<D, BF16, PACKED>;
+  auto kern = fa_fwd_kernel<D, BF16, PACKED, SPARSE>;
   cudaFuncAttributes attr;
   cudaError_t e = cudaFuncGetAttributes(&attr, kern);
   if (e != cudaSuccess) return e;
@@ -463,19 +514,16 @@ static cudaError_t launch_fwd_t(const CUtensorMap& tmq, const CUtensorMap& tmk,
 cudaError_t launch_fwd(int d, bool bf16, const CUtensorMap& tmq, const CUtensorMap& tmk,
                        const CUtensorMap& tmv, const FwdParams& p, int num_sms,
                        cudaStream_t stream) {
-  const bool packed = p.cu_seqlens != nullptr;
-  if (d == 128) {
-    if (packed)
-      return bf16 ? launch_fwd_t<128, true, true>(tmq, tmk, tmv, p, num_sms, stream)
-                  : launch_fwd_t<128, false, true>(tmq, tmk, tmv, p, num_sms, stream);
-    return bf16 ? launch_fwd_t<128, true, false>(tmq, tmk, tmv, p, num_sms, stream)
-                : launch_fwd_t<128, false, false>(tmq, tmk, tmv, p, num_sms, stream);
-  }
-  if (packed)
-    return bf16 ? launch_fwd_t<64, true, true>(tmq, tmk, tmv, p, num_sms, stream)
-                : launch_fwd_t<64, false, true>(tmq, tmk, tmv, p, num_sms, stream);
-  return bf16 ? launch_fwd_t<64, true, false>(tmq, tmk, tmv, p, num_sms, stream)
-              : launch_fwd_t<64, false, false>(tmq, tmk, tmv, p, num_sms, stream);
+  const int mode = p.cu_seqlens != nullptr ? 1 : (p.block_mask != nullptr ? 2 : 0);
+#define FA_FWD_LAUNCH(DD, BB, PP, SS) launch_fwd_t<DD, BB, PP, SS>(tmq, tmk, tmv, p, num_sms, stream)
+#define FA_FWD_MODES(DD, BB)                                       \
+  (mode == 1 ? FA_FWD_LAUNCH(DD, BB, true, false)                  \
+             : mode == 2 ? FA_FWD_LAUNCH(DD, BB, false, true)      \
+                         : FA_FWD_LAUNCH(DD, BB, false, false))
+  if (d == 128) return bf16 ? FA_FWD_MODES(128, true) : FA_FWD_MODES(128, false);
+  return bf16 ? FA_FWD_MODES(64, true) : FA_FWD_MODES(64, false);
+#undef FA_FWD_MODES
+#undef FA_FWD_LAUNCH
 }
 
 }  // namespace fa

@@ -30,6 +30,7 @@ struct FwdParams {
   const int32_t* seqlens;   // [B] valid key lengths (fixed length), or nullptr
   const int32_t* cu_seqlens;  // [B + 1] sequence offsets (packed), or nullptr
   int max_seqlen;           // packed: upper bound of every sequence length
+  const uint8_t* block_mask;  // block-sparse: [n_qtiles][n_qtiles] tile mask, or nullptr
   int B, H, N;
   float scale_log2;         // scale * log2(e)
   int causal;
@@ -53,6 +54,7 @@ struct BwdParams {
   const int32_t* seqlens;
   const int32_t* cu_seqlens;  // as in FwdParams
   int max_seqlen;
+  const uint8_t* block_mask;  // as in FwdParams ([n_ktiles][n_ktiles])
   int B, H, N;
   float scale;
   float scale_log2;
@@ -113,6 +115,13 @@ template <class P>
 __host__ __device__ inline long long total_rows(const P& p) {
   return p.cu_seqlens != nullptr ? static_cast<long long>(p.H) * p.N
                                  : static_cast<long long>(p.B) * p.H * p.N;
+}
+
+// Block-sparse attention (kernels instantiated with SPARSE): the 128 x 128
+// score tile (query tile qt, key tile kt) is computed only if
+// block_mask[qt * ntiles + kt] != 0, for every (batch, head) slice.
+__device__ __forceinline__ bool tile_allowed(const uint8_t* block_mask, int ntiles, int qt, int kt) {
+  return block_mask[static_cast<size_t>(qt) * ntiles + kt] != 0;
 }
 
 struct WorkItem {

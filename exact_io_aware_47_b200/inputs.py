@@ -32,7 +32,8 @@ from dataclasses import dataclass, field
 import torch
 
 __all__ = ["Workload", "WORKLOADS", "make_inputs", "make_inputs_shape", "PackedWorkload",
-           "PACKED_WORKLOADS", "make_inputs_varlen", "make_inputs_packed"]
+           "PACKED_WORKLOADS", "make_inputs_varlen", "make_inputs_packed", "window_block_mask",
+           "BLOCKSPARSE_WORKLOADS"]
 
 
 @dataclass(frozen=True)
@@ -161,3 +162,20 @@ def make_inputs_packed(name, seed=0, with_do=True, device="cpu"):
     w = PACKED_WORKLOADS[name]
     return make_inputs_varlen(w.B, w.H, w.max_len, w.d, w.dtype, seed=seed, with_do=with_do,
                               device=device)
+
+
+def window_block_mask(n_tiles, window, n_global=0):
+    """Boolean [n_tiles, n_tiles] tile mask: query tile i sees key tiles
+    i - window + 1 .. i (a sliding window) and the first ``n_global`` key
+    tiles."""
+    i = torch.arange(n_tiles)[:, None]
+    j = torch.arange(n_tiles)[None, :]
+    return ((i - j >= 0) & (i - j < window)) | (j < n_global)
+
+
+# Block-sparse workloads: a dense workload's inputs plus a tile mask.
+BLOCKSPARSE_WORKLOADS = {
+    "sparse": dict(base="mid", window=8, n_global=1,
+                   description="B2 H32 N8192 d128 bf16 causal, 8-tile (1024-key) sliding window "
+                               "plus the first key tile, 128 x 128 tiles"),
+}

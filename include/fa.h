@@ -165,6 +165,33 @@ int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
                   int dtype, void* stream);
 
 /*
+ * Block-sparse attention ("sparse-attention-flashattention" glossary page,
+ * definition: the original paper's block-sparse extension, a separate
+ * configuration of the same exact attention).  Same layout, masks and
+ * numerics as fa_fwd / fa_bwd, plus a tile mask: the 128 x 128 block of
+ * scores (query tile qt, key tile kt) is computed only if
+ * block_mask[qt * nt + kt] != 0, nt = ceil(N / 128); the softmax runs over
+ * the scores that remain (block mask, causal and key-length masks together).
+ * Skipped blocks cost no work: a K/V tile is loaded only if some query tile
+ * of the CTA's pair needs it.
+ *   block_mask: device uint8 [nt, nt], row-major, shared by every (batch,
+ *     head) slice; no alignment requirement.
+ *   Rows that are left no visible key get O = 0 and LSE = -inf, dQ = 0, and
+ *     add nothing to dK and dV; keys no query sees get dK = dV = 0.
+ *   fa_bwd_blocksparse: workspace as fa_bwd (fa_bwd_workspace_size); the
+ *     mask must be the one the forward used; runs the three backward stages
+ *     on `stream`.
+ */
+int fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                       const uint8_t* block_mask, int B, int H, int N, int d, float scale,
+                       int causal, const int32_t* seqlens, int dtype, void* stream);
+int fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o,
+                       const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                       void* workspace, size_t workspace_bytes, const uint8_t* block_mask,
+                       int B, int H, int N, int d, float scale, int causal,
+                       const int32_t* seqlens, int dtype, void* stream);
+
+/*
  * Backward pass that allocates nothing and takes no workspace.  The pages
  * have no counterpart: it exists for callers that cannot allocate device
  * memory for a workspace, such as plugin hosts that hand an operator only its
