@@ -7,7 +7,10 @@ Python binding never import it, and it imports nothing from them.
 
 from .attention import (allowed_mask, ref_bwd, ref_bwd_slice, ref_fwd,
                         ref_fwd_slice)
+from .dropout import (keep_mask, keep_threshold, philox4x32_10, ref_bwd_dropout_slice,
+                      ref_fwd_dropout_slice)
 from .online_model import tiled_fwd_slice
 
 __all__ = ["allowed_mask", "ref_fwd_slice", "ref_fwd", "ref_bwd_slice",
-           "ref_bwd", "tiled_fwd_slice"]
+           "ref_bwd", "tiled_fwd_slice", "philox4x32_10", "keep_threshold", "keep_mask",
+           "ref_fwd_dropout_slice", "ref_bwd_dropout_slice"]

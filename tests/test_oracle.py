@@ -357,3 +357,97 @@ def test_block_sparse_backward_matches_central_differences(causal):
             lm = loss(args["q"], args["k"], args["v"])
             num[idx] = (lp - lm) / (2 * eps)
         assert np.abs(num - g).max() / max(np.abs(num).max(), 1e-30) < 1e-6, name
+
+
+# --- dropout on the probabilities --------------------------------------------------
+
+from oracle.dropout import (keep_mask, keep_threshold, philox4x32_10, ref_bwd_dropout_slice,
+                            ref_fwd_dropout_slice)
+
+
+@pytest.mark.parametrize("ctr,key,expect", [
+    ((0, 0, 0, 0), (0, 0), (0x6627e8d5, 0xe169c58d, 0xbc57ac4c, 0x9b00dbd8)),
+    ((0xffffffff,) * 4, (0xffffffff,) * 2, (0x408f276d, 0x41c83b0e, 0xa20bc7c6, 0x6d5451fd)),
+    ((0x243f6a88, 0x85a308d3, 0x13198a2e, 0x03707344), (0xa4093822, 0x299f31d0),
+     (0xd16cfe09, 0x94fdcceb, 0x5001e420, 0x24126ea1)),
+])
+def test_philox_known_answers(ctr, key, expect):
+    """Known-answer vectors of Philox4x32-10 distributed with the generator's
+    reference implementation (Random123, by the authors of the SC 2011 paper)."""
+    out = philox4x32_10(*ctr, *key)
+    assert tuple(int(x) for x in out) == expect
+
+
+def test_dropout_zero_rate_is_plain_attention():
+    n, d = 9, 4
+    q, k, v, do = (_rand((n, d), s) for s in (80, 81, 82, 83))
+    for causal in (False, True):
+        o, lse = ref_fwd_dropout_slice(q, k, v, 0.5, causal, 0.0, seed=5, offset=0, bh=0)
+        ro, rl = ref_fwd_slice(q, k, v, 0.5, causal)
+        np.testing.assert_allclose(o, ro, atol=1e-14)
+        np.testing.assert_allclose(lse, rl, atol=1e-14)
+        g = ref_bwd_dropout_slice(q, k, v, do, 0.5, causal, 0.0, 5, 0, 0)
+        r = ref_bwd_slice(q, k, v, do, 0.5, causal)
+        for a, b in zip(g, r):
+            np.testing.assert_allclose(a, b, atol=1e-13)
+
+
+def test_keep_fraction_and_threshold():
+    assert keep_threshold(0.0) == (256, 1.0)
+    assert keep_threshold(0.25) == (192, 0.75)
+    assert keep_threshold(0.999)[0] == 1
+    m = keep_mask(3, np.arange(512), 512, seed=123456789, offset=7, p_drop=0.3)
+    t, keep = keep_threshold(0.3)
+    frac = m.mean()
+    # 262144 Bernoulli(keep) draws: 6 standard deviations
+    assert abs(frac - keep) < 6 * np.sqrt(keep * (1 - keep) / m.size)
+    # different seeds, offsets and slices give different masks
+    m2 = keep_mask(3, np.arange(64), 64, seed=123456790, offset=7, p_drop=0.3)
+    m3 = keep_mask(3, np.arange(64), 64, seed=123456789, offset=8, p_drop=0.3)
+    m4 = keep_mask(4, np.arange(64), 64, seed=123456789, offset=7, p_drop=0.3)
+    for other in (m2, m3, m4):
+        assert (other != m[:64, :64]).mean() > 0.2
+
+
+def test_mask_rows_are_independent_of_the_row_set():
+    full = keep_mask(1, np.arange(40), 37, seed=99, offset=1, p_drop=0.5)
+    rows = np.array([0, 3, 4, 17, 39])
+    np.testing.assert_array_equal(keep_mask(1, rows, 37, seed=99, offset=1, p_drop=0.5), full[rows])
+
+
+def test_dropout_is_unbiased_over_seeds():
+    """E_Z[O] = plain attention: averaged over many independent masks the
+    dropout output approaches the undropped one (1/sqrt(#seeds) rate)."""
+    n, d = 8, 3
+    q, k, v = (_rand((n, d), s) for s in (84, 85, 86))
+    ro, _ = ref_fwd_slice(q, k, v, 0.7, False)
+    acc = np.zeros_like(ro)
+    S = 4000
+    for s in range(S):
+        o, _ = ref_fwd_dropout_slice(q, k, v, 0.7, False, 0.5, seed=1000 + s, offset=0, bh=0)
+        acc += o
+    err = np.abs(acc / S - ro).max()
+    assert err < 6 * np.abs(v).max() / np.sqrt(S), err
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_dropout_backward_matches_central_differences(causal):
+    n, d, sc, p = 10, 3, 0.6, 0.4
+    q, k, v, do = (_rand((n, d), s) for s in (87, 88, 89, 90))
+    dq, dk, dv = ref_bwd_dropout_slice(q, k, v, do, sc, causal, p, 77, 3, 2)
+
+    def loss(qq, kk, vv):
+        o, _ = ref_fwd_dropout_slice(qq, kk, vv, sc, causal, p, 77, 3, 2)
+        return float((o * do).sum())
+
+    eps = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            args = {"q": q.copy(), "k": k.copy(), "v": v.copy()}
+            args[name][idx] += eps
+            lp = loss(args["q"], args["k"], args["v"])
+            args[name][idx] -= 2 * eps
+            lm = loss(args["q"], args["k"], args["v"])
+            num[idx] = (lp - lm) / (2 * eps)
+        assert np.abs(num - g).max() / max(np.abs(num).max(), 1e-30) < 1e-6, name
