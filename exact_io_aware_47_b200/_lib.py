@@ -39,6 +39,11 @@ SIGNATURES = {
     "fa_bwd_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP,
                             _I, _I, _I, _I, _F, _I, _VP, _I, _VP]),
     "fa_bwd_noalloc_max_bytes": (_SZ, []),
+    "fa_fwd_dropout": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _VP, _F,
+                            ctypes.c_uint64, ctypes.c_uint32, _I, _VP]),
+    "fa_bwd_dropout": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ,
+                            _I, _I, _I, _I, _F, _I, _VP, _F, ctypes.c_uint64, ctypes.c_uint32,
+                            _I, _VP]),
     "fa_fwd_blocksparse": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _VP, _I,
                                 _VP]),
     "fa_bwd_blocksparse": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP,
@@ -122,6 +127,19 @@ def fa_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal,
                    stream):
     return load().fa_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, B, H, N, d, scale, causal,
                                  seqlens, dtype, stream)
+
+
+def fa_fwd_dropout(q, k, v, o, lse, B, H, N, d, scale, causal, seqlens, p_drop, seed, offset,
+                   dtype, stream):
+    return load().fa_fwd_dropout(q, k, v, o, lse, B, H, N, d, scale, causal, seqlens, p_drop,
+                                 seed, offset, dtype, stream)
+
+
+def fa_bwd_dropout(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, N, d,
+                   scale, causal, seqlens, p_drop, seed, offset, dtype, stream):
+    return load().fa_bwd_dropout(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes,
+                                 B, H, N, d, scale, causal, seqlens, p_drop, seed, offset, dtype,
+                                 stream)
 
 
 def fa_fwd_blocksparse(q, k, v, o, lse, block_mask, B, H, N, d, scale, causal, seqlens, dtype,

@@ -1,6 +1,7 @@
 """torch-facing calls of the CUDA library: allocate outputs, pass pointers.
 
-``forward`` and ``backward`` ([B, H, N, d]), ``forward_blocksparse`` /
+``forward`` and ``backward`` ([B, H, N, d]), ``forward_dropout`` /
+``backward_dropout`` (dropout on the probabilities), ``forward_blocksparse`` /
 ``backward_blocksparse`` (the same with a 128 x 128 tile mask) and
 ``forward_varlen`` / ``backward_varlen`` (packed [H, T, d] with cu_seqlens)
 validate tensor
@@ -104,6 +105,57 @@ def backward(q, k, v, o, lse, do, scale=None, causal=False, seqlens=None, worksp
                          B, H, N, d, scale, int(bool(causal)), sl_ptr, _DTYPES[q.dtype],
                          _stream_handle(dev))
     _lib.check("fa_bwd", st)
+    return dq, dk, dv
+
+
+def forward_dropout(q, k, v, p_drop, seed, offset=0, scale=None, causal=False, seqlens=None,
+                    out=None, lse=None):
+    """O, LSE of attention with dropout on the probabilities ([B, H, N, d];
+    the keep mask is a function of seed, offset and the score's position)."""
+    B, H, N, d = q.shape
+    dev = q.device
+    if q.dtype not in _DTYPES:
+        raise ValueError("dtype must be bfloat16 or float16")
+    _check_inputs({"q": q, "k": k, "v": v}, (B, H, N, d), q.dtype, dev)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev) if lse is None else lse
+    _check_inputs({"out": out}, (B, H, N, d), q.dtype, dev)
+    _check_inputs({"lse": lse}, (B, H, N), torch.float32, dev)
+    sl, sl_ptr = _seqlens_arg(seqlens, B, dev)
+    with torch.cuda.device(dev):
+        st = _lib.fa_fwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                 lse.data_ptr(), B, H, N, d, scale, int(bool(causal)), sl_ptr,
+                                 float(p_drop), int(seed), int(offset), _DTYPES[q.dtype],
+                                 _stream_handle(dev))
+    _lib.check("fa_fwd_dropout", st)
+    return out, lse
+
+
+def backward_dropout(q, k, v, o, lse, do, p_drop, seed, offset=0, scale=None, causal=False,
+                     seqlens=None, workspace=None, dq=None, dk=None, dv=None):
+    """dQ, dK, dV for the same dropout mask as forward_dropout (same p_drop,
+    seed and offset)."""
+    B, H, N, d = q.shape
+    dev = q.device
+    _check_inputs({"q": q, "k": k, "v": v, "o": o, "do": do}, (B, H, N, d), q.dtype, dev)
+    _check_inputs({"lse": lse}, (B, H, N), torch.float32, dev)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check_inputs({"dq": dq, "dk": dk, "dv": dv}, (B, H, N, d), q.dtype, dev)
+    if workspace is None:
+        workspace = torch.empty(workspace_bytes(B, H, N, d), dtype=torch.uint8, device=dev)
+    sl, sl_ptr = _seqlens_arg(seqlens, B, dev)
+    with torch.cuda.device(dev):
+        st = _lib.fa_bwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                 do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                 dv.data_ptr(), workspace.data_ptr(),
+                                 workspace.numel() * workspace.element_size(), B, H, N, d, scale,
+                                 int(bool(causal)), sl_ptr, float(p_drop), int(seed), int(offset),
+                                 _DTYPES[q.dtype], _stream_handle(dev))
+    _lib.check("fa_bwd_dropout", st)
     return dq, dk, dv
 
 

@@ -124,7 +124,8 @@ namespace {
 int fwd_core(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
              int N, int d, float scale, int causal, const int32_t* seqlens,
              const int32_t* cu_seqlens, int max_seqlen, int dtype, void* stream,
-             const uint8_t* block_mask = nullptr) {
+             const uint8_t* block_mask = nullptr, uint32_t keep_t = 256u, float inv_keep = 1.f,
+             uint64_t seed = 0, uint32_t drop_offset = 0) {
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
       (seqlens && (reinterpret_cast<uintptr_t>(seqlens) & 3u)) ||
       (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)))
@@ -147,6 +148,11 @@ int fwd_core(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.cu_seqlens = cu_seqlens;
   p.max_seqlen = cu_seqlens ? max_seqlen : N;
   p.block_mask = block_mask;
+  p.keep_t = keep_t;
+  p.inv_keep = inv_keep;
+  p.seed_lo = static_cast<uint32_t>(seed);
+  p.seed_hi = static_cast<uint32_t>(seed >> 32);
+  p.drop_offset = drop_offset;
   p.B = B;
   p.H = H;
   p.N = N;
@@ -158,6 +164,17 @@ int fwd_core(const void* q, const void* k, const void* v, void* o, float* lse, i
   const cudaError_t e =
       launch_fwd(d, dtype == FA_BF16, tq, tk, tv, p, di.num_sms, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// Dropout rate -> 8-bit keep threshold t = round(256 (1 - p)) (ties to even),
+// clamped to [1, 256], and the scale 256 / t of the kept scores.
+int dropout_threshold(float p_drop, uint32_t* keep_t, float* inv_keep) {
+  if (!(p_drop >= 0.f && p_drop < 1.f)) return FA_ERR_INVALID_ARG;
+  double t = std::nearbyint(256.0 * (1.0 - static_cast<double>(p_drop)));
+  t = t < 1.0 ? 1.0 : (t > 256.0 ? 256.0 : t);
+  *keep_t = static_cast<uint32_t>(t);
+  *inv_keep = static_cast<float>(256.0 / t);
+  return FA_OK;
 }
 
 // Packed-layout argument checks shared by the forward and the backward: the
@@ -194,6 +211,21 @@ extern "C" int fa_fwd_blocksparse(const void* q, const void* k, const void* v, v
   if (st != FA_OK) return st;
   return fwd_core(q, k, v, o, lse, B, H, N, d, scale, causal, seqlens, nullptr, 0, dtype, stream,
                   block_mask);
+}
+
+extern "C" int fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* lse,
+                              int B, int H, int N, int d, float scale, int causal,
+                              const int32_t* seqlens, float p_drop, uint64_t seed,
+                              uint32_t offset, int dtype, void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  int st = check_common(B, H, N, d, scale, dtype);
+  if (st != FA_OK) return st;
+  uint32_t keep_t;
+  float inv_keep;
+  st = dropout_threshold(p_drop, &keep_t, &inv_keep);
+  if (st != FA_OK) return st;
+  return fwd_core(q, k, v, o, lse, B, H, N, d, scale, causal, seqlens, nullptr, 0, dtype, stream,
+                  nullptr, keep_t, inv_keep, seed, offset);
 }
 
 extern "C" int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -234,6 +266,8 @@ int bwd_common(void* workspace, size_t workspace_bytes, int B, int H, int N, int
   if (st != FA_OK) return st;
   const size_t rows = static_cast<size_t>(cu_seqlens ? 1 : B) * H * N;
   std::memset(p, 0, sizeof(*p));
+  p->keep_t = 256u;  // no dropout unless a dropout entry point sets it
+  p->inv_keep = 1.f;
   p->dsum = static_cast<float*>(workspace);
   p->dq_acc =
       reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round256(rows * sizeof(float)));
@@ -369,6 +403,52 @@ extern "C" int fa_bwd_blocksparse(const void* q, const void* k, const void* v, c
   p.dv = dv;
   p.causal = causal ? 1 : 0;
   p.block_mask = block_mask;
+  const bool bf16 = dtype == FA_BF16;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (launch_bwd_pre(d, bf16, p, di.num_sms, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (launch_bwd_main(d, bf16, tq, tk, tv, tdo, tdq, p, di.num_sms, s) != cudaSuccess)
+    return FA_ERR_CUDA;
+  return launch_bwd_post(d, bf16, p, di.num_sms, s) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+extern "C" int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o,
+                              const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                              void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
+                              float scale, int causal, const int32_t* seqlens, float p_drop,
+                              uint64_t seed, uint32_t offset, int dtype, void* stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_ALIGNMENT;
+  uint32_t keep_t;
+  float inv_keep;
+  int st = dropout_threshold(p_drop, &keep_t, &inv_keep);
+  if (st != FA_OK) return st;
+  BwdParams p;
+  DeviceInfo di;
+  st = bwd_common(workspace, workspace_bytes, B, H, N, d, scale, dtype, seqlens, &p, &di);
+  if (st != FA_OK) return st;
+  CUtensorMap tq, tk, tv, tdo, tdq;
+  const int BH = B * H;
+  if (make_map(&tq, q, BH, N, d, dtype) != FA_OK || make_map(&tk, k, BH, N, d, dtype) != FA_OK ||
+      make_map(&tv, v, BH, N, d, dtype) != FA_OK || make_map(&tdo, dout, BH, N, d, dtype) != FA_OK ||
+      make_map_acc(&tdq, p.dq_acc, BH, N, d) != FA_OK)
+    return FA_ERR_CUDA;
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.o = o;
+  p.dout = dout;
+  p.lse = lse;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.causal = causal ? 1 : 0;
+  p.keep_t = keep_t;
+  p.inv_keep = inv_keep;
+  p.seed_lo = static_cast<uint32_t>(seed);
+  p.seed_hi = static_cast<uint32_t>(seed >> 32);
+  p.drop_offset = offset;
   const bool bf16 = dtype == FA_BF16;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (launch_bwd_pre(d, bf16, p, di.num_sms, s) != cudaSuccess) return FA_ERR_CUDA;

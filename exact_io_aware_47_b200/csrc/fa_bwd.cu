@@ -128,7 +128,7 @@ __device__ __forceinline__ int bwd_next_i(const BwdParams& p, const BwdUnit& w, 
   return i;
 }
 
-template <int D, bool BF16, bool PACKED, bool SPARSE>
+template <int D, bool BF16, bool PACKED, bool SPARSE, bool DROPOUT>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const __grid_constant__ CUtensorMap tmdo,
@@ -499,6 +499,19 @@ __global__ void __launch_bounds__(512, 1)
       for (int idx = 0; idx < w.ni && ok; ++idx) {
         i = bwd_next_i<SPARSE>(p, w, i + 1);
         const int st = it & 1;  // LSE/D staging advances with the iteration count
+        // dropout: keep bits of this key for the half's 64 queries (bit q of
+        // drop_keep[q / 32] = query 128 i + 64 half + q), made while S^T is
+        // computed; the first phase writes only kept P^T, the second scales
+        // the kept dP^T by 256 / t
+        uint32_t drop_keep[2] = {~0u, ~0u};
+        if constexpr (DROPOUT) {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const uint32_t m16 =
+                keep_bits_key16(p, w.bh, w.j * kBlockN + r, i * kBlockM + 64 * half + 16 * g, lane & 3);
+            drop_keep[g >> 1] = (g & 1) ? (drop_keep[g >> 1] & 0xFFFFu) | (m16 << 16) : m16;
+          }
+        }
         // ---- phase 1: P^T = 2^(c S^T - LSE_i log2 e) from S^T, back to TMEM
         ok = mbar_wait_warp(&ld_full[st], (it >> 1) & 1, abort_flag, 28) &&
              mbar_wait_warp(s_full, it & 1, abort_flag, 29);
@@ -529,8 +542,12 @@ __global__ void __launch_bounds__(512, 1)
               const float x = fmaf(__uint_as_float(sr[e + k4]), cl, -lv[k4]);
               pv[cc * 32 + e + k4] = vis ? ex2_approx(x) : 0.f;
             }
-            pp[(e >> 1)] = pack2<BF16>(pv[cc * 32 + e], pv[cc * 32 + e + 1]);
-            pp[(e >> 1) + 1] = pack2<BF16>(pv[cc * 32 + e + 2], pv[cc * 32 + e + 3]);
+            float pd[4];  // P^T as dV sees it: dropped scores are zero
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4)
+              pd[k4] = DROPOUT && !((drop_keep[cc] >> (e + k4)) & 1u) ? 0.f : pv[cc * 32 + e + k4];
+            pp[(e >> 1)] = pack2<BF16>(pd[0], pd[1]);
+            pp[(e >> 1) + 1] = pack2<BF16>(pd[2], pd[3]);
           }
           // P^T of queries [32c, 32c+32) goes to columns 64 half + 16 (c & 1): only
           // over S^T columns this thread has already read, never the other
@@ -561,6 +578,13 @@ __global__ void __launch_bounds__(512, 1)
           for (int e = 0; e < 32; e += 4) {
             const int q0 = c * 32 + e;
             const float4 nd = *reinterpret_cast<const float4*>(dsm + q0);  // -D
+            if constexpr (DROPOUT) {  // dP of the kept scores, scaled by 256 / t
+#pragma unroll
+              for (int k4 = 0; k4 < 4; ++k4)
+                dr[e + k4] = (drop_keep[cc] >> (e + k4)) & 1u
+                                 ? __float_as_uint(__uint_as_float(dr[e + k4]) * p.inv_keep)
+                                 : 0u;
+            }
             // packed pairs: (dP - D) then P (dP - D)
             const int b0 = cc * 32 + e;
             const auto x01 = fadd2(f2pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])),
@@ -668,7 +692,7 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
         const uint32_t col = part == 0 ? Lay::kColDV : Lay::kColDK;
-        const float mul = part == 0 ? 1.f : p.scale;
+        const float mul = part == 0 ? (DROPOUT ? p.inv_keep : 1.f) : p.scale;
         uint8_t* rowp = part == 0 ? dvrow : dkrow;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
@@ -793,13 +817,13 @@ cudaError_t launch_bwd_pre(int d, bool bf16, const BwdParams& p, int num_sms,
   return cudaGetLastError();
 }
 
-template <int D, bool BF16, bool PACKED, bool SPARSE>
+template <int D, bool BF16, bool PACKED, bool SPARSE, bool DROPOUT>
 static cudaError_t launch_bwd_main_t(const CUtensorMap& tmq, const CUtensorMap& tmk,
                                      const CUtensorMap& tmv, const CUtensorMap& tmdo,
                                      const CUtensorMap& tmdq, const BwdParams& p, int num_sms,
                                      cudaStream_t stream) {
   using Lay = BwdLayout<D>;
-  auto kern = fa_bwd_kernel<D, BF16, PACKED, SPARSE>;
+  auto kern = fa_bwd_kernel<D, BF16, PACKED, SPARSE, DROPOUT>;
   cudaFuncAttributes attr;
   cudaError_t e = cudaFuncGetAttributes(&attr, kern);
   if (e != cudaSuccess) return e;
@@ -816,13 +840,17 @@ cudaError_t launch_bwd_main(int d, bool bf16, const CUtensorMap& tmq, const CUte
                             const CUtensorMap& tmv, const CUtensorMap& tmdo,
                             const CUtensorMap& tmdq, const BwdParams& p, int num_sms,
                             cudaStream_t stream) {
-  const int mode = p.cu_seqlens != nullptr ? 1 : (p.block_mask != nullptr ? 2 : 0);
-#define FA_BWD_LAUNCH(DD, BB, PP, SS) \
-  launch_bwd_main_t<DD, BB, PP, SS>(tmq, tmk, tmv, tmdo, tmdq, p, num_sms, stream)
-#define FA_BWD_MODES(DD, BB)                                       \
-  (mode == 1 ? FA_BWD_LAUNCH(DD, BB, true, false)                  \
-             : mode == 2 ? FA_BWD_LAUNCH(DD, BB, false, true)      \
-                         : FA_BWD_LAUNCH(DD, BB, false, false))
+  const int mode = p.cu_seqlens != nullptr ? 1
+                   : p.block_mask != nullptr ? 2
+                   : p.keep_t < 256u        ? 3
+                                            : 0;
+#define FA_BWD_LAUNCH(DD, BB, PP, SS, RR) \
+  launch_bwd_main_t<DD, BB, PP, SS, RR>(tmq, tmk, tmv, tmdo, tmdq, p, num_sms, stream)
+#define FA_BWD_MODES(DD, BB)                                                \
+  (mode == 1   ? FA_BWD_LAUNCH(DD, BB, true, false, false)                  \
+   : mode == 2 ? FA_BWD_LAUNCH(DD, BB, false, true, false)                  \
+   : mode == 3 ? FA_BWD_LAUNCH(DD, BB, false, false, true)                  \
+               : FA_BWD_LAUNCH(DD, BB, false, false, false))
   if (d == 128) return bf16 ? FA_BWD_MODES(128, true) : FA_BWD_MODES(128, false);
   return bf16 ? FA_BWD_MODES(64, true) : FA_BWD_MODES(64, false);
 #undef FA_BWD_MODES

@@ -116,7 +116,7 @@ __device__ __forceinline__ FwdUnit fwd_decode(int bh, int pair, const FwdParams&
   return w;
 }
 
-template <int D, bool BF16, bool PACKED, bool SPARSE>
+template <int D, bool BF16, bool PACKED, bool SPARSE, bool DROPOUT>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const FwdParams p) {
@@ -376,6 +376,16 @@ __global__ void __launch_bounds__(384, 1)
       int jj = 0;           // key tiles processed so far
       for (int j = 0; j < jend; ++j) {
         if (!fwd_need<SPARSE>(p, w, t, j)) continue;
+        // dropout: keep bits of this row for key tile j, made while the
+        // tensor core computes S (bit c of drop_keep[c / 32] = key 128 j + c)
+        uint32_t drop_keep[4] = {~0u, ~0u, ~0u, ~0u};
+        if constexpr (DROPOUT) {
+#pragma unroll
+          for (int g = 0; g < 8; ++g) {
+            const uint32_t m16 = keep_bits_row16(p, w.bh, row, j, g, lane & 3);
+            drop_keep[g >> 1] = (g & 1) ? (drop_keep[g >> 1] & 0xFFFFu) | (m16 << 16) : m16;
+          }
+        }
         ok = mbar_wait_warp(&s_full[t], scnt & 1, abort_flag, 8);
         if (!ok) break;
         if (r == 0) FA_TRACE_AT(scnt, 2 + 2 * t);
@@ -426,6 +436,10 @@ __global__ void __launch_bounds__(384, 1)
           acc[i & 3] = fadd2(acc[i & 3], p2);
           float p0, p1;
           f2unpack(p2, p0, p1);
+          if constexpr (DROPOUT) {  // dropped scores leave the row sum, not P V
+            p0 = (drop_keep[i >> 4] >> ((2 * i) & 31)) & 1u ? p0 : 0.f;
+            p1 = (drop_keep[i >> 4] >> ((2 * i + 1) & 31)) & 1u ? p1 : 0.f;
+          }
           pk[i] = pack2<BF16>(p0, p1);
         }
         {
@@ -462,7 +476,8 @@ __global__ void __launch_bounds__(384, 1)
       if (!ok) break;
       ++ocnt;
       tc_fence_after();
-      const float inv_l = 1.f / l;
+      // (with dropout the kept scores are scaled by 256 / t once, here)
+      const float inv_l = DROPOUT ? p.inv_keep / l : 1.f / l;
       const bool store = row < w.rows;
       const size_t orow_idx = static_cast<size_t>(w.z) * p.N + w.row0 + (store ? row : 0);
       uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) + orow_idx * (D * 2);
@@ -493,12 +508,12 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
-template <int D, bool BF16, bool PACKED, bool SPARSE>
+template <int D, bool BF16, bool PACKED, bool SPARSE, bool DROPOUT>
 static cudaError_t launch_fwd_t(const CUtensorMap& tmq, const CUtensorMap& tmk,
                                 const CUtensorMap& tmv, const FwdParams& p, int num_sms,
                                 cudaStream_t stream) {
   using Lay = FwdLayout<D>;
-  auto kern = fa_fwd_kernel<D, BF16, PACKED, SPARSE>;
+  auto kern = fa_fwd_kernel<D, BF16, PACKED, SPARSE, DROPOUT>;
   cudaFuncAttributes attr;
   cudaError_t e = cudaFuncGetAttributes(&attr, kern);
   if (e != cudaSuccess) return e;
@@ -514,12 +529,17 @@ static cudaError_t launch_fwd_t(const CUtensorMap& tmq, const CUtensorMap& tmk,
 cudaError_t launch_fwd(int d, bool bf16, const CUtensorMap& tmq, const CUtensorMap& tmk,
                        const CUtensorMap& tmv, const FwdParams& p, int num_sms,
                        cudaStream_t stream) {
-  const int mode = p.cu_seqlens != nullptr ? 1 : (p.block_mask != nullptr ? 2 : 0);
-#define FA_FWD_LAUNCH(DD, BB, PP, SS) launch_fwd_t<DD, BB, PP, SS>(tmq, tmk, tmv, p, num_sms, stream)
-#define FA_FWD_MODES(DD, BB)                                       \
-  (mode == 1 ? FA_FWD_LAUNCH(DD, BB, true, false)                  \
-             : mode == 2 ? FA_FWD_LAUNCH(DD, BB, false, true)      \
-                         : FA_FWD_LAUNCH(DD, BB, false, false))
+  const int mode = p.cu_seqlens != nullptr ? 1
+                   : p.block_mask != nullptr ? 2
+                   : p.keep_t < 256u        ? 3
+                                            : 0;
+#define FA_FWD_LAUNCH(DD, BB, PP, SS, RR) \
+  launch_fwd_t<DD, BB, PP, SS, RR>(tmq, tmk, tmv, p, num_sms, stream)
+#define FA_FWD_MODES(DD, BB)                                                \
+  (mode == 1   ? FA_FWD_LAUNCH(DD, BB, true, false, false)                  \
+   : mode == 2 ? FA_FWD_LAUNCH(DD, BB, false, true, false)                  \
+   : mode == 3 ? FA_FWD_LAUNCH(DD, BB, false, false, true)                  \
+               : FA_FWD_LAUNCH(DD, BB, false, false, false))
   if (d == 128) return bf16 ? FA_FWD_MODES(128, true) : FA_FWD_MODES(128, false);
   return bf16 ? FA_FWD_MODES(64, true) : FA_FWD_MODES(64, false);
 #undef FA_FWD_MODES

@@ -31,6 +31,10 @@ struct FwdParams {
   const int32_t* cu_seqlens;  // [B + 1] sequence offsets (packed), or nullptr
   int max_seqlen;           // packed: upper bound of every sequence length
   const uint8_t* block_mask;  // block-sparse: [n_qtiles][n_qtiles] tile mask, or nullptr
+  // dropout (kernels instantiated with DROPOUT): Philox key, counter word 3,
+  // 8-bit keep threshold t (1..256) and 256 / t
+  uint32_t seed_lo, seed_hi, drop_offset, keep_t;
+  float inv_keep;
   int B, H, N;
   float scale_log2;         // scale * log2(e)
   int causal;
@@ -55,6 +59,8 @@ struct BwdParams {
   const int32_t* cu_seqlens;  // as in FwdParams
   int max_seqlen;
   const uint8_t* block_mask;  // as in FwdParams ([n_ktiles][n_ktiles])
+  uint32_t seed_lo, seed_hi, drop_offset, keep_t;  // as in FwdParams
+  float inv_keep;
   int B, H, N;
   float scale;
   float scale_log2;
@@ -122,6 +128,44 @@ __host__ __device__ inline long long total_rows(const P& p) {
 // block_mask[qt * ntiles + kt] != 0, for every (batch, head) slice.
 __device__ __forceinline__ bool tile_allowed(const uint8_t* block_mask, int ntiles, int qt, int kt) {
   return block_mask[static_cast<size_t>(qt) * ntiles + kt] != 0;
+}
+
+// Dropout keep bits of one 4 x 4 block of scores, as the four lanes of a quad
+// need them.  The generator call for block (query block qb, key block kb) of
+// slice bh uses counter (kb, qb, bh, offset); word w of its result belongs to
+// query row 4 qb + w and byte c of that word to key 4 kb + c; a score is kept
+// iff its byte is below keep_t.
+//
+// Forward (lanes = 4 consecutive query rows, lane w = row & 3): 16 keys
+// 16 g .. 16 g + 15 of key tile j for this thread's row; bit c of the result
+// is key 16 g + c.
+template <class P>
+__device__ __forceinline__ uint32_t keep_bits_row16(const P& p, int bh, int row, int j, int g,
+                                                    int w) {
+  uint32_t a[4] = {static_cast<uint32_t>(32 * j + 4 * g + w), static_cast<uint32_t>(row >> 2),
+                   static_cast<uint32_t>(bh), p.drop_offset};
+  philox4x32_10(a, p.seed_lo, p.seed_hi);
+  quad_transpose4(a, w);  // a[s] = this row's word of key block 4 g + s
+  uint32_t m = 0;
+#pragma unroll
+  for (int s = 0; s < 4; ++s) m |= bytes_below(a[s], p.keep_t) << (4 * s);
+  return m;
+}
+
+// Backward (lanes = 4 consecutive keys, lane w = key & 3): 16 queries
+// q0 .. q0 + 15 (q0 a multiple of 16) for this thread's key; bit c of the
+// result is query q0 + c.
+template <class P>
+__device__ __forceinline__ uint32_t keep_bits_key16(const P& p, int bh, int key, int q0, int w) {
+  uint32_t a[4] = {static_cast<uint32_t>(key >> 2), static_cast<uint32_t>((q0 >> 2) + w),
+                   static_cast<uint32_t>(bh), p.drop_offset};
+  philox4x32_10(a, p.seed_lo, p.seed_hi);
+  byte_transpose4(a);     // a[c] = key c's bytes of the 4 queries
+  quad_transpose4(a, w);  // a[s] = this key's bytes of query block q0 / 4 + s
+  uint32_t m = 0;
+#pragma unroll
+  for (int s = 0; s < 4; ++s) m |= bytes_below(a[s], p.keep_t) << (4 * s);
+  return m;
 }
 
 struct WorkItem {

@@ -423,6 +423,72 @@ __device__ __forceinline__ void tmem_st_wait() {
 }
 
 // ---------------------------------------------------------------------------
+// Dropout masks: the counter-based generator Philox4x32-10 (Salmon, Moraes,
+// Dror, Shaw, "Parallel random numbers: as easy as 1, 2, 3", SC 2011), from
+// its published definition, and the quad-level data movement that hands each
+// thread the bytes of its own scores.
+// ---------------------------------------------------------------------------
+// One call: 128-bit counter c, 64-bit key (k0, k1), 10 rounds.  A round forms
+// the 64-bit products M0 c0 and M1 c2 and sets c = (hi1 ^ c1 ^ k0, lo1,
+// hi0 ^ c3 ^ k1, lo0); the key is bumped by (W0, W1) between rounds.
+__device__ __forceinline__ void philox4x32_10(uint32_t (&c)[4], uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint32_t hi0 = __umulhi(0xD2511F53u, c[0]), lo0 = 0xD2511F53u * c[0];
+    const uint32_t hi1 = __umulhi(0xCD9E8D57u, c[2]), lo1 = 0xCD9E8D57u * c[2];
+    const uint32_t n0 = hi1 ^ c[1] ^ k0, n2 = hi0 ^ c[3] ^ k1;
+    c[0] = n0;
+    c[1] = lo1;
+    c[2] = n2;
+    c[3] = lo0;
+  }
+}
+
+// 4 x 4 transpose of words across the 4 lanes of a quad (w = lane & 3): on
+// return a[s] holds what lane s held in a[w].  Two butterfly stages (lane
+// distance 1, then 2); every lane of the warp must take part.
+__device__ __forceinline__ void quad_transpose4(uint32_t (&a)[4], int w) {
+#pragma unroll
+  for (int m = 1; m <= 2; m <<= 1) {
+    const bool hi = (w & m) != 0;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (c & m) continue;
+      const uint32_t send = hi ? a[c] : a[c | m];
+      const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, m);
+      if (hi) a[c] = recv;
+      else a[c | m] = recv;
+    }
+  }
+}
+
+// 4 x 4 byte transpose inside four words: byte q of x[c] becomes byte c of
+// x[q] (byte permutes only).
+__device__ __forceinline__ void byte_transpose4(uint32_t (&x)[4]) {
+  const uint32_t t0 = __byte_perm(x[0], x[1], 0x5140), t1 = __byte_perm(x[0], x[1], 0x7362);
+  const uint32_t t2 = __byte_perm(x[2], x[3], 0x5140), t3 = __byte_perm(x[2], x[3], 0x7362);
+  x[0] = __byte_perm(t0, t2, 0x5410);
+  x[1] = __byte_perm(t0, t2, 0x7632);
+  x[2] = __byte_perm(t1, t3, 0x5410);
+  x[3] = __byte_perm(t1, t3, 0x7632);
+}
+
+// Bit k (k = 0..3) = (byte k of a) < t, for a threshold t in 1..256: per-byte
+// unsigned compare without carries between bytes (high bit of each byte),
+// then the four flags gathered by one multiply.
+__device__ __forceinline__ uint32_t bytes_below(uint32_t a, uint32_t t) {
+  if (t >= 256u) return 0xFu;
+  const uint32_t H = 0x80808080u, T = t * 0x01010101u;
+  const uint32_t d = (a | H) - (T & ~H);
+  const uint32_t lt = ((~a & T) | (~(a ^ T) & ~d)) & H;
+  return (((lt >> 7) * 0x00204081u) >> 21) & 0xFu;
+}
+
+// ---------------------------------------------------------------------------
 // small numeric helpers (hardware instructions, no library math)
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;

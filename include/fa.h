@@ -128,6 +128,37 @@ int fa_bwd_postprocess(void* workspace, size_t workspace_bytes, void* dq,
                        void* stream);
 
 /*
+ * Dropout on the attention probabilities, fused into both passes ("How Flash
+ * Attention Works", sections "Why Standard Attention Becomes a GPU Memory
+ * I/O Bottleneck": dropout comes after the softmax and before the product
+ * with V; "Kernel Fusion and Incremental Output Accumulation": it is fused,
+ * so the mask is regenerated, never stored).  Same layout, masks and checks
+ * as fa_fwd / fa_bwd, plus:
+ *   p_drop in [0, 1): scores are kept with probability t / 256, where
+ *     t = round(256 (1 - p_drop)) (ties to even, clamped to [1, 256]), and
+ *     kept probabilities are scaled by 256 / t:  O = (P * Z) V * 256 / t.
+ *     LSE is that of the scores (unaffected by dropout).  t = 256 (p_drop
+ *     below 1/512) runs the plain kernels.
+ *   seed, offset: the keep mask Z is a function of (seed, offset, batch,
+ *     head, query, key) only, from the counter-based generator Philox4x32-10
+ *     (Salmon et al., SC 2011): the call with counter (key / 4, query / 4,
+ *     b * H + h, offset) and key seed covers a 4 x 4 block; its word
+ *     query % 4, byte key % 4 is compared with t.  fa_bwd_dropout must get
+ *     the seed, offset and p_drop of the forward call.
+ *   Gradients are those of the loss <dO, O> for that fixed mask.
+ *   Returns FA_ERR_INVALID_ARG for p_drop outside [0, 1).
+ */
+int fa_fwd_dropout(const void* q, const void* k, const void* v, void* o, float* lse,
+                   int B, int H, int N, int d, float scale, int causal,
+                   const int32_t* seqlens, float p_drop, uint64_t seed, uint32_t offset,
+                   int dtype, void* stream);
+int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o,
+                   const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                   void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
+                   float scale, int causal, const int32_t* seqlens, float p_drop,
+                   uint64_t seed, uint32_t offset, int dtype, void* stream);
+
+/*
  * Packed variable-length batches: B sequences of different lengths stored
  * back to back, with no padding rows.  Same method, masks and numerics as
  * fa_fwd / fa_bwd, with each sequence its own attention problem: queries of
