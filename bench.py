@@ -1,7 +1,7 @@
 """Throughput of exact tiled attention (forward + backward) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload mid|small|long|ragged|tiny|varlen|sparse]
+                    [--workload mid|small|long|ragged|tiny|varlen|sparse|dropout]
 
 One step is the whole hot path over one batch: fa_fwd, then the three
 backward stages (row-dot preprocess, main kernel, dQ convert), on the
@@ -20,6 +20,9 @@ fa_bwd_varlen) on 8 sequences of lengths ~ U{1..4099}, H16, d128, bf16.
 ``--workload sparse`` times block-sparse attention (fa_fwd_blocksparse +
 fa_bwd_blocksparse) on the mid workload with an 8-tile sliding window plus
 the first key tile.
+
+``--workload dropout`` times dropout on the probabilities (fa_fwd_dropout +
+fa_bwd_dropout, p = 0.1) on the mid workload.
 
 ``--impl reference`` times the float64 CPU oracle (test infrastructure, the
 only other place this script runs it) on bounded samples of the same
@@ -592,9 +595,11 @@ def flops_fwd_blocksparse(mask, B, H, d, causal):
     return 4.0 * B * H * d * 128 * 128 * f
 
 
-def run_ours_blocksparse(args, spec):
-    """``--workload sparse``: one step = fa_fwd_blocksparse + fa_bwd_blocksparse
-    (its three kernels in one call) on a dense workload's inputs and a tile mask."""
+def run_ours_variant(args, spec):
+    """``--workload sparse`` / ``dropout``: one step = the variant's forward
+    entry point + its backward entry point (three kernels in one call) on a
+    dense workload's inputs: a tile mask (fa_*_blocksparse) or dropout on the
+    probabilities (fa_*_dropout)."""
     import torch
     world, rank, local = dist_setup()
     torch.cuda.set_device(local)
@@ -604,12 +609,11 @@ def run_ours_blocksparse(args, spec):
     import exact_io_aware_47_b200 as fa
     from exact_io_aware_47_b200.inputs import WORKLOADS, make_inputs, window_block_mask
 
+    kind = spec["kind"]
     w = WORKLOADS[spec["base"]]
     B, H, N, d = w.B, w.H, w.N, w.d
     dtype, causal, scale = w.dtypes[0], w.causal, w.scale
     nt = (N + 127) // 128
-    mask_b = window_block_mask(nt, spec["window"], spec["n_global"])
-    mask = mask_b.to(torch.uint8).to(dev).contiguous()
     inp = make_inputs(w.name, dtype=dtype, seed=rank, device=dev)
     q, k, v, do = inp["q"], inp["k"], inp["v"], inp["do"]
     o, lse = torch.empty_like(q), torch.empty((B, H, N), dtype=torch.float32, device=dev)
@@ -619,19 +623,69 @@ def run_ours_blocksparse(args, spec):
     stream = torch.cuda.current_stream(dev)
     sh = stream.cuda_stream
     dt_code = _lib.FA_BF16 if dtype == torch.bfloat16 else _lib.FA_FP16
+    ptrs = dict(q=q.data_ptr(), k=k.data_ptr(), v=v.data_ptr(), o=o.data_ptr(),
+                lse=lse.data_ptr(), do=do.data_ptr(), dq=dq.data_ptr(), dk=dk.data_ptr(),
+                dv=dv.data_ptr(), ws=ws.data_ptr())
+    extra_h2d = []
+    if kind == "sparse":
+        mask_b = window_block_mask(nt, spec["window"], spec["n_global"])
+        mask = mask_b.to(torch.uint8).to(dev).contiguous()
+        mask_list = mask_b.tolist()
+        extra_h2d = [(mask.cpu().pin_memory(), mask)]
+        f_fwd = flops_fwd_blocksparse(mask_list, B, H, d, causal)
+        names = ("fa_fwd_blocksparse", "fa_bwd_blocksparse")
+
+        def fwd_call():
+            return _lib.fa_fwd_blocksparse(ptrs["q"], ptrs["k"], ptrs["v"], ptrs["o"], ptrs["lse"],
+                                           mask.data_ptr(), B, H, N, d, scale, int(causal), None,
+                                           dt_code, sh)
+
+        def bwd_call():
+            return _lib.fa_bwd_blocksparse(ptrs["q"], ptrs["k"], ptrs["v"], ptrs["o"], ptrs["do"],
+                                           ptrs["lse"], ptrs["dq"], ptrs["dk"], ptrs["dv"],
+                                           ptrs["ws"], ws_bytes, mask.data_ptr(), B, H, N, d,
+                                           scale, int(causal), None, dt_code, sh)
+
+        def api_fwd():
+            fa.forward_blocksparse(q, k, v, mask, scale=scale, causal=causal, out=o, lse=lse)
+
+        def api_bwd():
+            fa.backward_blocksparse(q, k, v, o, lse, do, mask, scale=scale, causal=causal,
+                                    workspace=ws, dq=dq, dk=dk, dv=dv)
+        cfg = {"tiles_computed": sum(1 for i in range(nt) for j in range(nt)
+                                     if mask_list[i][j] and not (causal and j > i)),
+               "tiles_total": nt * nt}
+    else:
+        p_drop, seed = spec["p_drop"], spec["seed"]
+        f_fwd = flops_fwd(B, H, N, d, causal)
+        names = ("fa_fwd_dropout", "fa_bwd_dropout")
+
+        def fwd_call():
+            return _lib.fa_fwd_dropout(ptrs["q"], ptrs["k"], ptrs["v"], ptrs["o"], ptrs["lse"],
+                                       B, H, N, d, scale, int(causal), None, p_drop, seed, 0,
+                                       dt_code, sh)
+
+        def bwd_call():
+            return _lib.fa_bwd_dropout(ptrs["q"], ptrs["k"], ptrs["v"], ptrs["o"], ptrs["do"],
+                                       ptrs["lse"], ptrs["dq"], ptrs["dk"], ptrs["dv"], ptrs["ws"],
+                                       ws_bytes, B, H, N, d, scale, int(causal), None, p_drop,
+                                       seed, 0, dt_code, sh)
+
+        def api_fwd():
+            fa.forward_dropout(q, k, v, p_drop, seed, 0, scale=scale, causal=causal, out=o, lse=lse)
+
+        def api_bwd():
+            fa.backward_dropout(q, k, v, o, lse, do, p_drop, seed, 0, scale=scale, causal=causal,
+                                workspace=ws, dq=dq, dk=dk, dv=dv)
+        cfg = {"p_drop": p_drop, "seed": seed}
 
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        _lib.check("fa_fwd_blocksparse", _lib.fa_fwd_blocksparse(
-            q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-            mask.data_ptr(), B, H, N, d, scale, int(causal), None, dt_code, sh))
+        _lib.check(names[0], fwd_call())
         if ev is not None:
             ev[1].record(stream)
-        _lib.check("fa_bwd_blocksparse", _lib.fa_bwd_blocksparse(
-            q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
-            dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws_bytes, mask.data_ptr(),
-            B, H, N, d, scale, int(causal), None, dt_code, sh))
+        _lib.check(names[1], bwd_call())
         if ev is not None:
             ev[2].record(stream)
 
@@ -664,8 +718,6 @@ def run_ours_blocksparse(args, spec):
     total_ms = dist_max(t0.elapsed_time(t1), world)
     fwd_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
     bwd_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / K
-    mask_list = mask_b.tolist()
-    f_fwd = flops_fwd_blocksparse(mask_list, B, H, d, causal)
     f_bwd = 2.5 * f_fwd
     step_flops = f_fwd + f_bwd
     value = world * step_flops * K / (total_ms / 1e3) / 1e12
@@ -673,23 +725,21 @@ def run_ours_blocksparse(args, spec):
     peak = float(peaks["bf16_tflops"])
     fwd_tf = f_fwd / (fwd_ms / 1e3) / 1e12
     bwd_tf = f_bwd / (bwd_ms / 1e3) / 1e12
-    allowed = sum(1 for i in range(nt) for j in range(nt) if mask_list[i][j] and not (causal and j > i))
 
     e2e = None
     if not args.no_e2e:
         hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
         ho, hdq, hdk, hdv = (torch.empty(q.shape, dtype=dtype, pin_memory=True) for _ in range(4))
         hlse = torch.empty((B, H, N), dtype=torch.float32, pin_memory=True)
-        hmask = mask.cpu().pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo, hmask))
+        ins = [(hq, q), (hk, k), (hv, v), (hdo, do)] + extra_h2d
+        h2d = sum(src.numel() * src.element_size() for src, _ in ins)
         d2h = sum(t.numel() * t.element_size() for t in (ho, hlse, hdq, hdk, hdv))
 
         def e2e_step():
-            for src, dst in ((hq, q), (hk, k), (hv, v), (hdo, do), (hmask, mask)):
+            for src, dst in ins:
                 dst.copy_(src, non_blocking=True)
-            fa.forward_blocksparse(q, k, v, mask, scale=scale, causal=causal, out=o, lse=lse)
-            fa.backward_blocksparse(q, k, v, o, lse, do, mask, scale=scale, causal=causal,
-                                    workspace=ws, dq=dq, dk=dk, dv=dv)
+            api_fwd()
+            api_bwd()
             for src, dst in ((o, ho), (lse, hlse), (dq, hdq), (dk, hdk), (dv, hdv)):
                 dst.copy_(src, non_blocking=True)
 
@@ -712,18 +762,26 @@ def run_ours_blocksparse(args, spec):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         from threadpoolctl import threadpool_info
-        from oracle import ref_bwd_slice, ref_fwd_slice
         import numpy as np
-        mnp = np.array(mask_list, dtype=bool)
+        from oracle import (ref_bwd_dropout_slice, ref_bwd_slice, ref_fwd_dropout_slice,
+                            ref_fwd_slice)
+        n_rows = min(2048, N)  # slices cut to their first n_rows queries and keys
+        nt_cut = (n_rows + 127) // 128
         dt, fl, n_done = 0.0, 0.0, 0
-        for b in range(B):  # whole (batch, head) slices until ~10 s of CPU work
+        for b in range(B):  # until ~10 s of CPU work
             for h in range(H):
-                qq, kk, vv, dd = (t[b, h].double().cpu().numpy() for t in (q, k, v, do))
+                qq, kk, vv, dd = (t[b, h, :n_rows].double().cpu().numpy() for t in (q, k, v, do))
                 tc = time.perf_counter()
-                ref_fwd_slice(qq, kk, vv, scale, causal, block_mask=mnp)
-                ref_bwd_slice(qq, kk, vv, dd, scale, causal, block_mask=mnp)
+                if kind == "sparse":
+                    mnp = np.array(mask_list, dtype=bool)[:nt_cut, :nt_cut]
+                    ref_fwd_slice(qq, kk, vv, scale, causal, block_mask=mnp)
+                    ref_bwd_slice(qq, kk, vv, dd, scale, causal, block_mask=mnp)
+                    fl += 3.5 * flops_fwd_blocksparse(mnp.tolist(), 1, 1, d, causal)
+                else:
+                    ref_fwd_dropout_slice(qq, kk, vv, scale, causal, p_drop, seed, 0, b * H + h)
+                    ref_bwd_dropout_slice(qq, kk, vv, dd, scale, causal, p_drop, seed, 0, b * H + h)
+                    fl += 3.5 * flops_fwd(1, 1, n_rows, d, causal)
                 dt += time.perf_counter() - tc
-                fl += 3.5 * flops_fwd_blocksparse(mask_list, 1, 1, d, causal)
                 n_done += 1
                 if dt >= 10.0:
                     break
@@ -731,27 +789,25 @@ def run_ours_blocksparse(args, spec):
                 break
         thr = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
         cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
-               "sample": f"float64 oracle forward+backward (dense S, block mask applied) of "
-                         f"{n_done} whole (batch, head) slices ({dt:.1f} s); FLOPs counted "
-                         f"over the allowed tiles only"}
+               "sample": f"float64 oracle forward+backward ({kind}) of {n_done} (batch, head) "
+                         f"slices cut to their first {n_rows} queries and keys ({dt:.1f} s)"}
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
         "warmup": warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if dtype == torch.bfloat16 else "f16", "data": "synthetic",
-        "config": {"workload": spec["description"], "B": B, "H": H, "N": N, "d": d,
-                   "causal": causal, "tiles_computed": allowed, "tiles_total": nt * nt,
-                   "step": "fa_fwd_blocksparse + fa_bwd_blocksparse",
-                   "flops_per_step": step_flops, "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (4 x 128 MiB per step), no flush"},
+        "config": dict({"workload": spec["description"], "B": B, "H": H, "N": N, "d": d,
+                        "causal": causal, "step": f"{names[0]} + {names[1]}",
+                        "flops_per_step": step_flops, "parallelism": f"replicas x{world}",
+                        "l2": "inputs larger than L2 (4 x 128 MiB per step), no flush"}, **cfg),
         "fwd": {"ms": fwd_ms, "tflops": fwd_tf, "frac": fwd_tf / peak},
         "bwd": {"ms": bwd_ms, "tflops": bwd_tf, "frac": bwd_tf / peak},
-        "roofline": {"bound": "tensor", "kernel": "fa_bwd_blocksparse (preprocess + main + postprocess)",
+        "roofline": {"bound": "tensor", "kernel": f"{names[1]} (preprocess + main + postprocess)",
                      "achieved": bwd_tf, "peak": peak, "unit": "TFLOP/s", "frac": bwd_tf / peak,
                      "traffic": None, "peak_source": f"{peak_src} bf16 dense (burst)",
                      "flops_per_launch": f_bwd},
-        "roofline_fwd": {"bound": "tensor", "kernel": "fa_fwd_kernel (fa_fwd_blocksparse)",
+        "roofline_fwd": {"bound": "tensor", "kernel": f"fa_fwd_kernel ({names[0]})",
                          "achieved": fwd_tf, "peak": peak, "unit": "TFLOP/s",
                          "frac": fwd_tf / peak, "traffic": None,
                          "peak_source": f"{peak_src} bf16 dense (burst)", "flops_per_launch": f_fwd},
@@ -771,7 +827,7 @@ def main():
     if args.workload in BLOCKSPARSE_WORKLOADS:
         if args.impl == "reference":
             raise SystemExit("--impl reference times the dense workloads")
-        return run_ours_blocksparse(args, BLOCKSPARSE_WORKLOADS[args.workload])
+        return run_ours_variant(args, BLOCKSPARSE_WORKLOADS[args.workload])
     if args.workload in PACKED_WORKLOADS:
         if args.impl == "reference":
             raise SystemExit("--impl reference times the fixed-length workloads")

@@ -175,7 +175,12 @@ def window_block_mask(n_tiles, window, n_global=0):
 
 # Block-sparse workloads: a dense workload's inputs plus a tile mask.
 BLOCKSPARSE_WORKLOADS = {
-    "sparse": dict(base="mid", window=8, n_global=1,
+    "sparse": dict(kind="sparse", base="mid", window=8, n_global=1,
                    description="B2 H32 N8192 d128 bf16 causal, 8-tile (1024-key) sliding window "
                                "plus the first key tile, 128 x 128 tiles"),
+    # dropout on the probabilities (the mask is regenerated from seed and
+    # position inside both kernels)
+    "dropout": dict(kind="dropout", base="mid", p_drop=0.1, seed=0x5EED,
+                    description="B2 H32 N8192 d128 bf16 causal with dropout p = 0.1 on the "
+                                "probabilities"),
 }
