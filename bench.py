@@ -74,13 +74,19 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+# Files that hold device code (the kernels and the device helpers they use);
+# the host API in fa_api.cu does not change what a kernel moves.
+KERNEL_SOURCES = ("fa_bwd.cu", "fa_fwd.cu", "fa_internal.h", "sm100.cuh")
+
+
 def kernel_source_sha():
+    """Hash of the kernels' sources: recorded DRAM traffic is reported only
+    while it matches (profiles/traffic.json)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_io_aware_47_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
-        if fn.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, fn), "rb") as f:
-                h.update(fn.encode() + f.read())
+    for fn in KERNEL_SOURCES:
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode() + f.read())
     return h.hexdigest()[:16]
 
 

@@ -371,26 +371,22 @@ extern "C" int fa_bwd(const void* q, const void* k, const void* v, const void* o
   return fa_bwd_postprocess(workspace, workspace_bytes, dq, B, H, N, d, scale, dtype, stream);
 }
 
-extern "C" int fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o,
-                                  const void* dout, const float* lse, void* dq, void* dk,
-                                  void* dv, void* workspace, size_t workspace_bytes,
-                                  const uint8_t* block_mask, int B, int H, int N, int d,
-                                  float scale, int causal, const int32_t* seqlens, int dtype,
-                                  void* stream) {
-  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !block_mask)
-    return FA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
-      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
-    return FA_ERR_ALIGNMENT;
-  BwdParams p;
-  DeviceInfo di;
-  int st = bwd_common(workspace, workspace_bytes, B, H, N, d, scale, dtype, seqlens, &p, &di);
-  if (st != FA_OK) return st;
+namespace fa {
+namespace {
+
+// The three backward stages in one call for a variant (block mask, dropout,
+// packed layout): p has passed bwd_common and carries the variant's fields;
+// blocks x rows is the TMA view of the tensors (B*H x N, or H x T packed).
+int bwd_variant_run(BwdParams& p, const DeviceInfo& di, const void* q, const void* k,
+                    const void* v, const void* o, const void* dout, const float* lse, void* dq,
+                    void* dk, void* dv, int blocks, int rows, int d, int causal, int dtype,
+                    void* stream) {
   CUtensorMap tq, tk, tv, tdo, tdq;
-  const int BH = B * H;
-  if (make_map(&tq, q, BH, N, d, dtype) != FA_OK || make_map(&tk, k, BH, N, d, dtype) != FA_OK ||
-      make_map(&tv, v, BH, N, d, dtype) != FA_OK || make_map(&tdo, dout, BH, N, d, dtype) != FA_OK ||
-      make_map_acc(&tdq, p.dq_acc, BH, N, d) != FA_OK)
+  if (make_map(&tq, q, blocks, rows, d, dtype) != FA_OK ||
+      make_map(&tk, k, blocks, rows, d, dtype) != FA_OK ||
+      make_map(&tv, v, blocks, rows, d, dtype) != FA_OK ||
+      make_map(&tdo, dout, blocks, rows, d, dtype) != FA_OK ||
+      make_map_acc(&tdq, p.dq_acc, blocks, rows, d) != FA_OK)
     return FA_ERR_CUDA;
   p.q = q;
   p.k = k;
@@ -402,7 +398,6 @@ extern "C" int fa_bwd_blocksparse(const void* q, const void* k, const void* v, c
   p.dk = dk;
   p.dv = dv;
   p.causal = causal ? 1 : 0;
-  p.block_mask = block_mask;
   const bool bf16 = dtype == FA_BF16;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (launch_bwd_pre(d, bf16, p, di.num_sms, s) != cudaSuccess) return FA_ERR_CUDA;
@@ -411,15 +406,46 @@ extern "C" int fa_bwd_blocksparse(const void* q, const void* k, const void* v, c
   return launch_bwd_post(d, bf16, p, di.num_sms, s) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+bool bwd_pointers_ok(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                     const float* lse, const void* dq, const void* dk, const void* dv) {
+  return q && k && v && o && dout && lse && dq && dk && dv;
+}
+
+bool bwd_pointers_aligned(const void* q, const void* k, const void* v, const void* o,
+                          const void* dout, const float* lse, const void* dq, const void* dk,
+                          const void* dv) {
+  return aligned16(q) && aligned16(k) && aligned16(v) && aligned16(o) && aligned16(dout) &&
+         aligned16(lse) && aligned16(dq) && aligned16(dk) && aligned16(dv);
+}
+
+}  // namespace
+}  // namespace fa
+
+extern "C" int fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o,
+                                  const void* dout, const float* lse, void* dq, void* dk,
+                                  void* dv, void* workspace, size_t workspace_bytes,
+                                  const uint8_t* block_mask, int B, int H, int N, int d,
+                                  float scale, int causal, const int32_t* seqlens, int dtype,
+                                  void* stream) {
+  if (!bwd_pointers_ok(q, k, v, o, dout, lse, dq, dk, dv) || !block_mask)
+    return FA_ERR_INVALID_ARG;
+  if (!bwd_pointers_aligned(q, k, v, o, dout, lse, dq, dk, dv)) return FA_ERR_ALIGNMENT;
+  BwdParams p;
+  DeviceInfo di;
+  const int st = bwd_common(workspace, workspace_bytes, B, H, N, d, scale, dtype, seqlens, &p, &di);
+  if (st != FA_OK) return st;
+  p.block_mask = block_mask;
+  return bwd_variant_run(p, di, q, k, v, o, dout, lse, dq, dk, dv, B * H, N, d, causal, dtype,
+                         stream);
+}
+
 extern "C" int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o,
                               const void* dout, const float* lse, void* dq, void* dk, void* dv,
                               void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
                               float scale, int causal, const int32_t* seqlens, float p_drop,
                               uint64_t seed, uint32_t offset, int dtype, void* stream) {
-  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
-      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
-    return FA_ERR_ALIGNMENT;
+  if (!bwd_pointers_ok(q, k, v, o, dout, lse, dq, dk, dv)) return FA_ERR_INVALID_ARG;
+  if (!bwd_pointers_aligned(q, k, v, o, dout, lse, dq, dk, dv)) return FA_ERR_ALIGNMENT;
   uint32_t keep_t;
   float inv_keep;
   int st = dropout_threshold(p_drop, &keep_t, &inv_keep);
@@ -428,33 +454,13 @@ extern "C" int fa_bwd_dropout(const void* q, const void* k, const void* v, const
   DeviceInfo di;
   st = bwd_common(workspace, workspace_bytes, B, H, N, d, scale, dtype, seqlens, &p, &di);
   if (st != FA_OK) return st;
-  CUtensorMap tq, tk, tv, tdo, tdq;
-  const int BH = B * H;
-  if (make_map(&tq, q, BH, N, d, dtype) != FA_OK || make_map(&tk, k, BH, N, d, dtype) != FA_OK ||
-      make_map(&tv, v, BH, N, d, dtype) != FA_OK || make_map(&tdo, dout, BH, N, d, dtype) != FA_OK ||
-      make_map_acc(&tdq, p.dq_acc, BH, N, d) != FA_OK)
-    return FA_ERR_CUDA;
-  p.q = q;
-  p.k = k;
-  p.v = v;
-  p.o = o;
-  p.dout = dout;
-  p.lse = lse;
-  p.dq = dq;
-  p.dk = dk;
-  p.dv = dv;
-  p.causal = causal ? 1 : 0;
   p.keep_t = keep_t;
   p.inv_keep = inv_keep;
   p.seed_lo = static_cast<uint32_t>(seed);
   p.seed_hi = static_cast<uint32_t>(seed >> 32);
   p.drop_offset = offset;
-  const bool bf16 = dtype == FA_BF16;
-  const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (launch_bwd_pre(d, bf16, p, di.num_sms, s) != cudaSuccess) return FA_ERR_CUDA;
-  if (launch_bwd_main(d, bf16, tq, tk, tv, tdo, tdq, p, di.num_sms, s) != cudaSuccess)
-    return FA_ERR_CUDA;
-  return launch_bwd_post(d, bf16, p, di.num_sms, s) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  return bwd_variant_run(p, di, q, k, v, o, dout, lse, dq, dk, dv, B * H, N, d, causal, dtype,
+                         stream);
 }
 
 extern "C" int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
@@ -462,36 +468,14 @@ extern "C" int fa_bwd_varlen(const void* q, const void* k, const void* v, const 
                              void* workspace, size_t workspace_bytes, const int32_t* cu_seqlens,
                              int B, int H, int T, int max_seqlen, int d, float scale, int causal,
                              int dtype, void* stream) {
-  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
-      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
-    return FA_ERR_ALIGNMENT;
+  if (!bwd_pointers_ok(q, k, v, o, dout, lse, dq, dk, dv)) return FA_ERR_INVALID_ARG;
+  if (!bwd_pointers_aligned(q, k, v, o, dout, lse, dq, dk, dv)) return FA_ERR_ALIGNMENT;
   BwdParams p;
   DeviceInfo di;
-  int st = bwd_common(workspace, workspace_bytes, B, H, T, d, scale, dtype, nullptr, &p, &di,
-                      cu_seqlens, max_seqlen < T ? max_seqlen : T);
+  const int st = bwd_common(workspace, workspace_bytes, B, H, T, d, scale, dtype, nullptr, &p,
+                            &di, cu_seqlens, max_seqlen < T ? max_seqlen : T);
   if (st != FA_OK) return st;
-  CUtensorMap tq, tk, tv, tdo, tdq;
-  if (make_map(&tq, q, H, T, d, dtype) != FA_OK || make_map(&tk, k, H, T, d, dtype) != FA_OK ||
-      make_map(&tv, v, H, T, d, dtype) != FA_OK || make_map(&tdo, dout, H, T, d, dtype) != FA_OK ||
-      make_map_acc(&tdq, p.dq_acc, H, T, d) != FA_OK)
-    return FA_ERR_CUDA;
-  p.q = q;
-  p.k = k;
-  p.v = v;
-  p.o = o;
-  p.dout = dout;
-  p.lse = lse;
-  p.dq = dq;
-  p.dk = dk;
-  p.dv = dv;
-  p.causal = causal ? 1 : 0;
-  const bool bf16 = dtype == FA_BF16;
-  const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (launch_bwd_pre(d, bf16, p, di.num_sms, s) != cudaSuccess) return FA_ERR_CUDA;
-  if (launch_bwd_main(d, bf16, tq, tk, tv, tdo, tdq, p, di.num_sms, s) != cudaSuccess)
-    return FA_ERR_CUDA;
-  return launch_bwd_post(d, bf16, p, di.num_sms, s) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  return bwd_variant_run(p, di, q, k, v, o, dout, lse, dq, dk, dv, H, T, d, causal, dtype, stream);
 }
 
 // ---------------------------------------------------------------------------
