@@ -230,7 +230,8 @@ def run_reference(args, w):
 
 
 # ----------------------------------------------------------------- CUDA path
-def run_ours(args, w):
+def _cuda_setup():
+    """Rank, device and the CUDA library (built in-tree)."""
     import torch
     world, rank, local = dist_setup()
     torch.cuda.set_device(local)
@@ -238,6 +239,126 @@ def run_ours(args, w):
     from exact_io_aware_47_b200 import _lib, build
     build.build()
     import exact_io_aware_47_b200 as fa
+    return torch, world, rank, dev, _lib, fa
+
+
+def _timed_steps(torch, step, n_marks, args, world, dev, stream, lib):
+    """max(3, W) warm-up steps, then K steps between barriers with CUDA events
+    recorded at n_marks points of every step on the launch stream; clocks
+    sampled meanwhile.  Returns (warm-up steps, max over ranks of the timed
+    region in ms, mean ms between consecutive marks, clock summary)."""
+    sh = stream.cuda_stream
+    warmup = max(3, args.warmup)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    st, word = lib.fa_device_status(sh)
+    if st != 0:
+        raise RuntimeError(f"device status {st} ({word:#x}) after warm-up")
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_marks)] for _ in range(K)]
+    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    if not args.no_clocks:
+        clocks.start()
+        time.sleep(0.3)
+    dist_barrier(world)
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(K):
+        step(evs[i])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    dist_barrier(world)
+    clk = None if args.no_clocks else clocks.stop()
+    st, word = lib.fa_device_status(sh)
+    if st != 0:
+        raise RuntimeError(f"device status {st} ({word:#x}) after timing")
+    total_ms = dist_max(t0.elapsed_time(t1), world)
+    seg = [sum(e[m].elapsed_time(e[m + 1]) for e in evs) / K for m in range(n_marks - 1)]
+    return warmup, total_ms, seg, clk
+
+
+def _e2e(torch, dev_inputs, dev_outputs, api_step, K, world, dev, stream, step_flops):
+    """End to end through the public API: every step copies its inputs from
+    pinned host memory, runs api_step and copies its results back."""
+    ins = [(t.cpu().pin_memory(), t) for t in dev_inputs]
+    outs = [(t, torch.empty(t.shape, dtype=t.dtype, pin_memory=True)) for t in dev_outputs]
+    h2d = sum(src.numel() * src.element_size() for src, _ in ins)
+    d2h = sum(dst.numel() * dst.element_size() for _, dst in outs)
+
+    def e2e_step():
+        for src, dst in ins:
+            dst.copy_(src, non_blocking=True)
+        api_step()
+        for src, dst in outs:
+            dst.copy_(src, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    ke = max(3, min(K, 10))
+    dist_barrier(world)
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(ke):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    dist_barrier(world)
+    e_ms = dist_max(a.elapsed_time(b), world)
+    return {"value": world * step_flops * ke / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / ke}
+
+
+def _roof(kernel, flops, ms, peak, peak_src, traffic=None):
+    tf = flops / (ms / 1e3) / 1e12
+    return {"bound": "tensor", "kernel": kernel, "achieved": tf, "peak": peak, "unit": "TFLOP/s",
+            "frac": tf / peak, "traffic": traffic, "peak_source": f"{peak_src} bf16 dense (burst)",
+            "flops_per_launch": flops}
+
+
+def _cpu_oracle(samples):
+    """Run (fn, flops) samples until about 10 s of CPU work; (TFLOP/s, threads,
+    samples run, seconds)."""
+    from threadpoolctl import threadpool_info
+    dt, fl, n_done = 0.0, 0.0, 0
+    for fn, f in samples:
+        tc = time.perf_counter()
+        fn()
+        dt += time.perf_counter() - tc
+        fl += f
+        n_done += 1
+        if dt >= 10.0:
+            break
+    thr = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    return fl / dt / 1e12, thr, n_done, dt
+
+
+def _emit(line, rank, world):
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def _base_line(value, K, warmup, total_ms, world, dtype_name, config, fwd, bwd, roofline,
+               roofline_fwd, cpu, e2e, clk, launches_per_step):
+    return {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": dtype_name, "data": "synthetic",
+        "config": config, "fwd": fwd, "bwd": bwd, "roofline": roofline,
+        "roofline_fwd": roofline_fwd, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": launches_per_step * K, "clocks": clk,
+    }
+
+
+def run_ours(args, w):
+    """Headline: fa_fwd and the three backward stages, each timed by events."""
+    torch, world, rank, dev, _lib, fa = _cuda_setup()
     from exact_io_aware_47_b200.inputs import make_inputs
 
     B, H, N, d = w.B, w.H, w.N, w.d
@@ -279,103 +400,33 @@ def run_ours(args, w):
         if ev is not None:
             ev[4].record(stream)
 
-    warmup = max(3, args.warmup)
-    for _ in range(warmup):
-        step()
-    torch.cuda.synchronize(dev)
-    st, word = _lib.fa_device_status(sh)
-    if st != 0:
-        raise RuntimeError(f"device status {st} ({word:#x}) after warm-up")
-
+    warmup, total_ms, seg, clk = _timed_steps(torch, step, 5, args, world, dev, stream, _lib)
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
-    clocks = ClockSampler(dev.index if dev.index is not None else 0)
-    if not args.no_clocks:
-        clocks.start()
-        time.sleep(0.3)
-    dist_barrier(world)
-    torch.cuda.synchronize(dev)
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    t_start.record(stream)
-    for i in range(K):
-        step(evs[i])
-    t_end.record(stream)
-    torch.cuda.synchronize(dev)
-    dist_barrier(world)
-    clk = None if args.no_clocks else clocks.stop()
-    st, word = _lib.fa_device_status(sh)
-    if st != 0:
-        raise RuntimeError(f"device status {st} ({word:#x}) after timing")
-
-    total_ms = dist_max(t_start.elapsed_time(t_end), world)
-    parts = {"fa_fwd_kernel": [], "fa_bwd_pre": [], "fa_bwd_kernel": [], "fa_bwd_post": []}
-    for e in evs:
-        parts["fa_fwd_kernel"].append(e[0].elapsed_time(e[1]))
-        parts["fa_bwd_pre"].append(e[1].elapsed_time(e[2]))
-        parts["fa_bwd_kernel"].append(e[2].elapsed_time(e[3]))
-        parts["fa_bwd_post"].append(e[3].elapsed_time(e[4]))
-    avg = {n: sum(v_) / len(v_) for n, v_ in parts.items()}
-
+    avg = dict(zip(("fa_fwd_kernel", "fa_bwd_pre", "fa_bwd_kernel", "fa_bwd_post"), seg))
     f_fwd = flops_fwd(B, H, N, d, causal)
     f_bwd = 2.5 * f_fwd
     step_flops = f_fwd + f_bwd
     ms_per_step = total_ms / K
     value = world * step_flops * K / (total_ms / 1e3) / 1e12
-
     peaks, peak_src = load_peaks()
     peak = float(peaks["bf16_tflops"])
     dom = max(("fa_fwd_kernel", "fa_bwd_kernel"), key=lambda n: avg[n])
-    dom_flops = f_fwd if dom == "fa_fwd_kernel" else f_bwd
-    achieved = dom_flops / (avg[dom] / 1e3) / 1e12
-    traffic = recorded_traffic(dom, w.name)
-    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
-                "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
-                "peak_source": f"{peak_src} bf16 dense (burst)",
-                "flops_per_launch": dom_flops}
-    fwd_tf = f_fwd / (avg["fa_fwd_kernel"] / 1e3) / 1e12
-    roofline_fwd = {"bound": "tensor", "kernel": "fa_fwd_kernel", "achieved": fwd_tf, "peak": peak,
-                    "unit": "TFLOP/s", "frac": fwd_tf / peak,
-                    "traffic": recorded_traffic("fa_fwd_kernel", w.name),
-                    "peak_source": f"{peak_src} bf16 dense (burst)", "flops_per_launch": f_fwd}
+    roofline = _roof(dom, f_fwd if dom == "fa_fwd_kernel" else f_bwd, avg[dom], peak, peak_src,
+                     recorded_traffic(dom, w.name))
+    roofline_fwd = _roof("fa_fwd_kernel", f_fwd, avg["fa_fwd_kernel"], peak, peak_src,
+                         recorded_traffic("fa_fwd_kernel", w.name))
     bwd_ms = avg["fa_bwd_pre"] + avg["fa_bwd_kernel"] + avg["fa_bwd_post"]
+    fwd_tf = roofline_fwd["achieved"]
     bwd_tf = f_bwd / (bwd_ms / 1e3) / 1e12
-    kernels = {n: {"ms": avg[n], "share": avg[n] / ms_per_step} for n in avg}
 
-    # end to end through the public API: pinned host inputs in, results out
     e2e = None
     if not args.no_e2e:
-        hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
-        ho, hdq, hdk, hdv = (torch.empty(q.shape, dtype=dtype, pin_memory=True) for _ in range(4))
-        hlse = torch.empty((B, H, N), dtype=torch.float32, pin_memory=True)
-        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
-        d2h = sum(t.numel() * t.element_size() for t in (ho, hlse, hdq, hdk, hdv))
-
-        def e2e_step():
-            for src, dst in ((hq, q), (hk, k), (hv, v), (hdo, do)):
-                dst.copy_(src, non_blocking=True)
+        def api_step():
             fa.forward(q, k, v, scale=scale, causal=causal, seqlens=sl, out=o, lse=lse)
             fa.backward(q, k, v, o, lse, do, scale=scale, causal=causal, seqlens=sl,
                         workspace=ws, dq=dq, dk=dk, dv=dv)
-            for src, dst in ((o, ho), (lse, hlse), (dq, hdq), (dk, hdk), (dv, hdv)):
-                dst.copy_(src, non_blocking=True)
-
-        for _ in range(2):
-            e2e_step()
-        ke = max(3, min(K, 10))
-        dist_barrier(world)
-        torch.cuda.synchronize(dev)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(ke):
-            e2e_step()
-        b.record(stream)
-        torch.cuda.synchronize(dev)
-        dist_barrier(world)
-        e_ms = dist_max(a.elapsed_time(b), world)
-        e2e = {"value": world * step_flops * ke / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": e_ms / ke}
+        e2e = _e2e(torch, (q, k, v, do), (o, lse, dq, dk, dv), api_step, K, world, dev, stream,
+                   step_flops)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -385,31 +436,17 @@ def run_ours(args, w):
                "sample": f"float64 oracle forward+backward of {n_slices} whole (batch, head) "
                          f"slices of '{w.name}' ({dt:.1f} s)"}
 
-    line = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
-        "warmup": warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if dtype == torch.bfloat16 else "f16",
-        "data": "synthetic",
-        "config": {"workload": w.description, "B": B, "H": H, "N": N, "d": d, "causal": causal,
-                   "step": "fa_fwd + fa_bwd_preprocess + fa_bwd_main + fa_bwd_postprocess",
-                   "flops_per_step": step_flops, "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (4 x 128 MiB per step), no flush"},
-        "fwd": {"ms": avg["fa_fwd_kernel"], "tflops": fwd_tf, "frac": fwd_tf / peak},
-        "bwd": {"ms": bwd_ms, "tflops": bwd_tf, "frac": bwd_tf / peak},
-        "kernels": kernels,
-        "roofline": roofline,
-        "roofline_fwd": roofline_fwd,
-        "cpu_baseline": cpu,
-        "e2e": e2e,
-        "gpu_launches": 4 * K,
-        "clocks": clk,
-    }
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
-    return 0
+    config = {"workload": w.description, "B": B, "H": H, "N": N, "d": d, "causal": causal,
+              "step": "fa_fwd + fa_bwd_preprocess + fa_bwd_main + fa_bwd_postprocess",
+              "flops_per_step": step_flops, "parallelism": f"replicas x{world}",
+              "l2": "inputs larger than L2 (4 x 128 MiB per step), no flush"}
+    line = _base_line(value, K, warmup, total_ms, world,
+                      "bf16" if dtype == torch.bfloat16 else "f16", config,
+                      {"ms": avg["fa_fwd_kernel"], "tflops": fwd_tf, "frac": fwd_tf / peak},
+                      {"ms": bwd_ms, "tflops": bwd_tf, "frac": bwd_tf / peak},
+                      roofline, roofline_fwd, cpu, e2e, clk, 4)
+    line["kernels"] = {n: {"ms": avg[n], "share": avg[n] / ms_per_step} for n in avg}
+    return _emit(line, rank, world)
 
 
 # ------------------------------------------------------ packed (variable length)
@@ -420,13 +457,7 @@ def flops_fwd_packed(lengths, H, d, causal):
 def run_ours_packed(args, w):
     """``--workload varlen``: one step = fa_fwd_varlen + fa_bwd_varlen (its
     three kernels in one call) on a packed batch; FLOPs summed per sequence."""
-    import torch
-    world, rank, local = dist_setup()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    from exact_io_aware_47_b200 import _lib, build
-    build.build()
-    import exact_io_aware_47_b200 as fa
+    torch, world, rank, dev, _lib, fa = _cuda_setup()
     from exact_io_aware_47_b200.inputs import make_inputs_packed
 
     inp = make_inputs_packed(w.name, seed=rank, device=dev)
@@ -457,137 +488,65 @@ def run_ours_packed(args, w):
         if ev is not None:
             ev[2].record(stream)
 
-    warmup = max(3, args.warmup)
-    for _ in range(warmup):
-        step()
-    torch.cuda.synchronize(dev)
-    st, word = _lib.fa_device_status(sh)
-    if st != 0:
-        raise RuntimeError(f"device status {st} ({word:#x}) after warm-up")
+    warmup, total_ms, (fwd_ms, bwd_ms), clk = _timed_steps(torch, step, 3, args, world, dev,
+                                                           stream, _lib)
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
-    clocks = ClockSampler(dev.index if dev.index is not None else 0)
-    if not args.no_clocks:
-        clocks.start()
-        time.sleep(0.3)
-    dist_barrier(world)
-    torch.cuda.synchronize(dev)
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for i in range(K):
-        step(evs[i])
-    t1.record(stream)
-    torch.cuda.synchronize(dev)
-    dist_barrier(world)
-    clk = None if args.no_clocks else clocks.stop()
-    st, word = _lib.fa_device_status(sh)
-    if st != 0:
-        raise RuntimeError(f"device status {st} ({word:#x}) after timing")
-    total_ms = dist_max(t0.elapsed_time(t1), world)
-    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
-    bwd_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / K
     f_fwd = flops_fwd_packed(lengths, H, d, causal)
     f_bwd = 2.5 * f_fwd
     step_flops = f_fwd + f_bwd
     value = world * step_flops * K / (total_ms / 1e3) / 1e12
     peaks, peak_src = load_peaks()
     peak = float(peaks["bf16_tflops"])
-    fwd_tf = f_fwd / (fwd_ms / 1e3) / 1e12
-    bwd_tf = f_bwd / (bwd_ms / 1e3) / 1e12
-    roofline = {"bound": "tensor", "kernel": "fa_bwd_varlen (preprocess + main + postprocess)",
-                "achieved": bwd_tf, "peak": peak, "unit": "TFLOP/s", "frac": bwd_tf / peak,
-                "traffic": None, "peak_source": f"{peak_src} bf16 dense (burst)",
-                "flops_per_launch": f_bwd}
-    roofline_fwd = {"bound": "tensor", "kernel": "fa_fwd_kernel (fa_fwd_varlen)",
-                    "achieved": fwd_tf, "peak": peak, "unit": "TFLOP/s", "frac": fwd_tf / peak,
-                    "traffic": None, "peak_source": f"{peak_src} bf16 dense (burst)",
-                    "flops_per_launch": f_fwd}
+    roofline = _roof("fa_bwd_varlen (preprocess + main + postprocess)", f_bwd, bwd_ms, peak,
+                     peak_src)
+    roofline_fwd = _roof("fa_fwd_kernel (fa_fwd_varlen)", f_fwd, fwd_ms, peak, peak_src)
 
     e2e = None
     if not args.no_e2e:
-        hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
-        ho, hdq, hdk, hdv = (torch.empty(q.shape, dtype=w.dtype, pin_memory=True)
-                             for _ in range(4))
-        hlse = torch.empty((H, T), dtype=torch.float32, pin_memory=True)
-        hcu = cu.cpu().pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo, hcu))
-        d2h = sum(t.numel() * t.element_size() for t in (ho, hlse, hdq, hdk, hdv))
-
-        def e2e_step():
-            for src, dst in ((hq, q), (hk, k), (hv, v), (hdo, do), (hcu, cu)):
-                dst.copy_(src, non_blocking=True)
+        def api_step():
             fa.forward_varlen(q, k, v, cu, ms, scale=scale, causal=causal, out=o, lse=lse)
             fa.backward_varlen(q, k, v, o, lse, do, cu, ms, scale=scale, causal=causal,
                                workspace=ws, dq=dq, dk=dk, dv=dv)
-            for src, dst in ((o, ho), (lse, hlse), (dq, hdq), (dk, hdk), (dv, hdv)):
-                dst.copy_(src, non_blocking=True)
-
-        for _ in range(2):
-            e2e_step()
-        ke = max(3, min(K, 10))
-        dist_barrier(world)
-        torch.cuda.synchronize(dev)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(ke):
-            e2e_step()
-        b.record(stream)
-        torch.cuda.synchronize(dev)
-        dist_barrier(world)
-        e_ms = dist_max(a.elapsed_time(b), world)
-        e2e = {"value": world * step_flops * ke / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / ke}
+        e2e = _e2e(torch, (q, k, v, do, cu), (o, lse, dq, dk, dv), api_step, K, world, dev,
+                   stream, step_flops)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        from threadpoolctl import threadpool_info
         from oracle import ref_bwd_slice, ref_fwd_slice
         cuh = [int(x) for x in cu.cpu()]
-        dt, fl, n_done = 0.0, 0.0, 0
-        for h in range(H):  # whole (head, sequence) slices until ~10 s of CPU work
-            for b in range(B):
-                s0, s1 = cuh[b], cuh[b + 1]
-                if s1 == s0:
-                    continue
-                qq, kk, vv, dd = (t[h, s0:s1].double().cpu().numpy() for t in (q, k, v, do))
-                tc = time.perf_counter()
-                ref_fwd_slice(qq, kk, vv, scale, causal)
-                ref_bwd_slice(qq, kk, vv, dd, scale, causal)
-                dt += time.perf_counter() - tc
-                fl += 3.5 * flops_fwd(1, 1, s1 - s0, d, causal)
-                n_done += 1
-            if dt >= 10.0:
-                break
-        thr = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+        host = {n: t.double().cpu() for n, t in (("q", q), ("k", k), ("v", v), ("do", do))}
+
+        def samples():  # whole (head, sequence) slices, all sequences of the first heads
+            for h in range(H):
+                for b in range(B):
+                    s0, s1 = cuh[b], cuh[b + 1]
+                    if s1 == s0:
+                        continue
+                    qq, kk, vv, dd = (host[n][h, s0:s1].numpy() for n in ("q", "k", "v", "do"))
+                    yield ((lambda qq=qq, kk=kk, vv=vv, dd=dd: (
+                        ref_fwd_slice(qq, kk, vv, scale, causal),
+                        ref_bwd_slice(qq, kk, vv, dd, scale, causal))),
+                           3.5 * flops_fwd(1, 1, s1 - s0, d, causal))
+        val, thr, n_done, dt = _cpu_oracle(samples())
+        cpu = {"value": val, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
                "sample": f"float64 oracle forward+backward of {n_done} whole (head, sequence) "
                          f"slices, all sequences of the first heads ({dt:.1f} s)"}
 
-    line = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
-        "warmup": warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if w.dtype == torch.bfloat16 else "f16", "data": "synthetic",
-        "config": {"workload": w.description, "B": B, "H": H, "T": T, "max_seqlen": ms, "d": d,
-                   "causal": causal, "lengths": lengths,
-                   "step": "fa_fwd_varlen + fa_bwd_varlen", "flops_per_step": step_flops,
-                   "parallelism": f"replicas x{world}",
-                   "l2": f"inputs {4 * q.numel() * q.element_size() / 2**20:.0f} MiB per step, "
-                         "no flush"},
-        "fwd": {"ms": fwd_ms, "tflops": fwd_tf, "frac": fwd_tf / peak},
-        "bwd": {"ms": bwd_ms, "tflops": bwd_tf, "frac": bwd_tf / peak},
-        "roofline": roofline, "roofline_fwd": roofline_fwd,
-        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 4 * K, "clocks": clk,
-    }
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
-    return 0
+    config = {"workload": w.description, "B": B, "H": H, "T": T, "max_seqlen": ms, "d": d,
+              "causal": causal, "lengths": lengths, "step": "fa_fwd_varlen + fa_bwd_varlen",
+              "flops_per_step": step_flops, "parallelism": f"replicas x{world}",
+              "l2": f"inputs {4 * q.numel() * q.element_size() / 2**20:.0f} MiB per step, "
+                    "no flush"}
+    line = _base_line(value, K, warmup, total_ms, world,
+                      "bf16" if w.dtype == torch.bfloat16 else "f16", config,
+                      {"ms": fwd_ms, "tflops": roofline_fwd["achieved"],
+                       "frac": roofline_fwd["frac"]},
+                      {"ms": bwd_ms, "tflops": roofline["achieved"], "frac": roofline["frac"]},
+                      roofline, roofline_fwd, cpu, e2e, clk, 4)
+    return _emit(line, rank, world)
 
 
-# ----------------------------------------------------------------- block-sparse
+# ------------------------------------------------- block-sparse and dropout
 def flops_fwd_blocksparse(mask, B, H, d, causal):
     """Scores actually computed: 128 x 128 per allowed tile below the diagonal,
     half a tile on the diagonal when causal (the dense causal convention)."""
@@ -606,13 +565,7 @@ def run_ours_variant(args, spec):
     entry point + its backward entry point (three kernels in one call) on a
     dense workload's inputs: a tile mask (fa_*_blocksparse) or dropout on the
     probabilities (fa_*_dropout)."""
-    import torch
-    world, rank, local = dist_setup()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    from exact_io_aware_47_b200 import _lib, build
-    build.build()
-    import exact_io_aware_47_b200 as fa
+    torch, world, rank, dev, _lib, fa = _cuda_setup()
     from exact_io_aware_47_b200.inputs import WORKLOADS, make_inputs, window_block_mask
 
     kind = spec["kind"]
@@ -629,33 +582,31 @@ def run_ours_variant(args, spec):
     stream = torch.cuda.current_stream(dev)
     sh = stream.cuda_stream
     dt_code = _lib.FA_BF16 if dtype == torch.bfloat16 else _lib.FA_FP16
-    ptrs = dict(q=q.data_ptr(), k=k.data_ptr(), v=v.data_ptr(), o=o.data_ptr(),
-                lse=lse.data_ptr(), do=do.data_ptr(), dq=dq.data_ptr(), dk=dk.data_ptr(),
-                dv=dv.data_ptr(), ws=ws.data_ptr())
-    extra_h2d = []
+    P = dict(q=q.data_ptr(), k=k.data_ptr(), v=v.data_ptr(), o=o.data_ptr(), lse=lse.data_ptr(),
+             do=do.data_ptr(), dq=dq.data_ptr(), dk=dk.data_ptr(), dv=dv.data_ptr(),
+             ws=ws.data_ptr())
+    extra_inputs = ()
     if kind == "sparse":
         mask_b = window_block_mask(nt, spec["window"], spec["n_global"])
         mask = mask_b.to(torch.uint8).to(dev).contiguous()
         mask_list = mask_b.tolist()
-        extra_h2d = [(mask.cpu().pin_memory(), mask)]
+        extra_inputs = (mask,)
         f_fwd = flops_fwd_blocksparse(mask_list, B, H, d, causal)
         names = ("fa_fwd_blocksparse", "fa_bwd_blocksparse")
 
         def fwd_call():
-            return _lib.fa_fwd_blocksparse(ptrs["q"], ptrs["k"], ptrs["v"], ptrs["o"], ptrs["lse"],
+            return _lib.fa_fwd_blocksparse(P["q"], P["k"], P["v"], P["o"], P["lse"],
                                            mask.data_ptr(), B, H, N, d, scale, int(causal), None,
                                            dt_code, sh)
 
         def bwd_call():
-            return _lib.fa_bwd_blocksparse(ptrs["q"], ptrs["k"], ptrs["v"], ptrs["o"], ptrs["do"],
-                                           ptrs["lse"], ptrs["dq"], ptrs["dk"], ptrs["dv"],
-                                           ptrs["ws"], ws_bytes, mask.data_ptr(), B, H, N, d,
-                                           scale, int(causal), None, dt_code, sh)
+            return _lib.fa_bwd_blocksparse(P["q"], P["k"], P["v"], P["o"], P["do"], P["lse"],
+                                           P["dq"], P["dk"], P["dv"], P["ws"], ws_bytes,
+                                           mask.data_ptr(), B, H, N, d, scale, int(causal), None,
+                                           dt_code, sh)
 
-        def api_fwd():
+        def api_step():
             fa.forward_blocksparse(q, k, v, mask, scale=scale, causal=causal, out=o, lse=lse)
-
-        def api_bwd():
             fa.backward_blocksparse(q, k, v, o, lse, do, mask, scale=scale, causal=causal,
                                     workspace=ws, dq=dq, dk=dk, dv=dv)
         cfg = {"tiles_computed": sum(1 for i in range(nt) for j in range(nt)
@@ -667,22 +618,19 @@ def run_ours_variant(args, spec):
         names = ("fa_fwd_dropout", "fa_bwd_dropout")
 
         def fwd_call():
-            return _lib.fa_fwd_dropout(ptrs["q"], ptrs["k"], ptrs["v"], ptrs["o"], ptrs["lse"],
-                                       B, H, N, d, scale, int(causal), None, p_drop, seed, 0,
-                                       dt_code, sh)
+            return _lib.fa_fwd_dropout(P["q"], P["k"], P["v"], P["o"], P["lse"], B, H, N, d, scale,
+                                       int(causal), None, p_drop, seed, 0, dt_code, sh)
 
         def bwd_call():
-            return _lib.fa_bwd_dropout(ptrs["q"], ptrs["k"], ptrs["v"], ptrs["o"], ptrs["do"],
-                                       ptrs["lse"], ptrs["dq"], ptrs["dk"], ptrs["dv"], ptrs["ws"],
-                                       ws_bytes, B, H, N, d, scale, int(causal), None, p_drop,
-                                       seed, 0, dt_code, sh)
+            return _lib.fa_bwd_dropout(P["q"], P["k"], P["v"], P["o"], P["do"], P["lse"], P["dq"],
+                                       P["dk"], P["dv"], P["ws"], ws_bytes, B, H, N, d, scale,
+                                       int(causal), None, p_drop, seed, 0, dt_code, sh)
 
-        def api_fwd():
-            fa.forward_dropout(q, k, v, p_drop, seed, 0, scale=scale, causal=causal, out=o, lse=lse)
-
-        def api_bwd():
-            fa.backward_dropout(q, k, v, o, lse, do, p_drop, seed, 0, scale=scale, causal=causal,
-                                workspace=ws, dq=dq, dk=dk, dv=dv)
+        def api_step():
+            fa.forward_dropout(q, k, v, p_drop, seed, 0, scale=scale, causal=causal, out=o,
+                               lse=lse)
+            fa.backward_dropout(q, k, v, o, lse, do, p_drop, seed, 0, scale=scale,
+                                causal=causal, workspace=ws, dq=dq, dk=dk, dv=dv)
         cfg = {"p_drop": p_drop, "seed": seed}
 
     def step(ev=None):
@@ -695,136 +643,65 @@ def run_ours_variant(args, spec):
         if ev is not None:
             ev[2].record(stream)
 
-    warmup = max(3, args.warmup)
-    for _ in range(warmup):
-        step()
-    torch.cuda.synchronize(dev)
-    st, word = _lib.fa_device_status(sh)
-    if st != 0:
-        raise RuntimeError(f"device status {st} ({word:#x}) after warm-up")
+    warmup, total_ms, (fwd_ms, bwd_ms), clk = _timed_steps(torch, step, 3, args, world, dev,
+                                                           stream, _lib)
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
-    clocks = ClockSampler(dev.index if dev.index is not None else 0)
-    if not args.no_clocks:
-        clocks.start()
-        time.sleep(0.3)
-    dist_barrier(world)
-    torch.cuda.synchronize(dev)
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for i in range(K):
-        step(evs[i])
-    t1.record(stream)
-    torch.cuda.synchronize(dev)
-    dist_barrier(world)
-    clk = None if args.no_clocks else clocks.stop()
-    st, word = _lib.fa_device_status(sh)
-    if st != 0:
-        raise RuntimeError(f"device status {st} ({word:#x}) after timing")
-    total_ms = dist_max(t0.elapsed_time(t1), world)
-    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
-    bwd_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / K
     f_bwd = 2.5 * f_fwd
     step_flops = f_fwd + f_bwd
     value = world * step_flops * K / (total_ms / 1e3) / 1e12
     peaks, peak_src = load_peaks()
     peak = float(peaks["bf16_tflops"])
-    fwd_tf = f_fwd / (fwd_ms / 1e3) / 1e12
-    bwd_tf = f_bwd / (bwd_ms / 1e3) / 1e12
+    roofline = _roof(f"{names[1]} (preprocess + main + postprocess)", f_bwd, bwd_ms, peak,
+                     peak_src)
+    roofline_fwd = _roof(f"fa_fwd_kernel ({names[0]})", f_fwd, fwd_ms, peak, peak_src)
 
     e2e = None
     if not args.no_e2e:
-        hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
-        ho, hdq, hdk, hdv = (torch.empty(q.shape, dtype=dtype, pin_memory=True) for _ in range(4))
-        hlse = torch.empty((B, H, N), dtype=torch.float32, pin_memory=True)
-        ins = [(hq, q), (hk, k), (hv, v), (hdo, do)] + extra_h2d
-        h2d = sum(src.numel() * src.element_size() for src, _ in ins)
-        d2h = sum(t.numel() * t.element_size() for t in (ho, hlse, hdq, hdk, hdv))
-
-        def e2e_step():
-            for src, dst in ins:
-                dst.copy_(src, non_blocking=True)
-            api_fwd()
-            api_bwd()
-            for src, dst in ((o, ho), (lse, hlse), (dq, hdq), (dk, hdk), (dv, hdv)):
-                dst.copy_(src, non_blocking=True)
-
-        for _ in range(2):
-            e2e_step()
-        ke = max(3, min(K, 10))
-        dist_barrier(world)
-        torch.cuda.synchronize(dev)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(ke):
-            e2e_step()
-        b.record(stream)
-        torch.cuda.synchronize(dev)
-        dist_barrier(world)
-        e_ms = dist_max(a.elapsed_time(b), world)
-        e2e = {"value": world * step_flops * ke / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / ke}
+        e2e = _e2e(torch, (q, k, v, do) + extra_inputs, (o, lse, dq, dk, dv), api_step, K,
+                   world, dev, stream, step_flops)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        from threadpoolctl import threadpool_info
         import numpy as np
         from oracle import (ref_bwd_dropout_slice, ref_bwd_slice, ref_fwd_dropout_slice,
                             ref_fwd_slice)
         n_rows = min(2048, N)  # slices cut to their first n_rows queries and keys
         nt_cut = (n_rows + 127) // 128
-        dt, fl, n_done = 0.0, 0.0, 0
-        for b in range(B):  # until ~10 s of CPU work
-            for h in range(H):
-                qq, kk, vv, dd = (t[b, h, :n_rows].double().cpu().numpy() for t in (q, k, v, do))
-                tc = time.perf_counter()
-                if kind == "sparse":
-                    mnp = np.array(mask_list, dtype=bool)[:nt_cut, :nt_cut]
-                    ref_fwd_slice(qq, kk, vv, scale, causal, block_mask=mnp)
-                    ref_bwd_slice(qq, kk, vv, dd, scale, causal, block_mask=mnp)
-                    fl += 3.5 * flops_fwd_blocksparse(mnp.tolist(), 1, 1, d, causal)
-                else:
-                    ref_fwd_dropout_slice(qq, kk, vv, scale, causal, p_drop, seed, 0, b * H + h)
-                    ref_bwd_dropout_slice(qq, kk, vv, dd, scale, causal, p_drop, seed, 0, b * H + h)
-                    fl += 3.5 * flops_fwd(1, 1, n_rows, d, causal)
-                dt += time.perf_counter() - tc
-                n_done += 1
-                if dt >= 10.0:
-                    break
-            if dt >= 10.0:
-                break
-        thr = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+
+        def samples():
+            for b in range(B):
+                for h in range(H):
+                    qq, kk, vv, dd = (t[b, h, :n_rows].double().cpu().numpy()
+                                      for t in (q, k, v, do))
+                    if kind == "sparse":
+                        mnp = np.array(mask_list, dtype=bool)[:nt_cut, :nt_cut]
+                        yield ((lambda qq=qq, kk=kk, vv=vv, dd=dd, mnp=mnp: (
+                            ref_fwd_slice(qq, kk, vv, scale, causal, block_mask=mnp),
+                            ref_bwd_slice(qq, kk, vv, dd, scale, causal, block_mask=mnp))),
+                               3.5 * flops_fwd_blocksparse(mnp.tolist(), 1, 1, d, causal))
+                    else:
+                        bh = b * H + h
+                        yield ((lambda qq=qq, kk=kk, vv=vv, dd=dd, bh=bh: (
+                            ref_fwd_dropout_slice(qq, kk, vv, scale, causal, p_drop, seed, 0, bh),
+                            ref_bwd_dropout_slice(qq, kk, vv, dd, scale, causal, p_drop, seed, 0,
+                                                  bh))),
+                               3.5 * flops_fwd(1, 1, n_rows, d, causal))
+        val, thr, n_done, dt = _cpu_oracle(samples())
+        cpu = {"value": val, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
                "sample": f"float64 oracle forward+backward ({kind}) of {n_done} (batch, head) "
                          f"slices cut to their first {n_rows} queries and keys ({dt:.1f} s)"}
 
-    line = {
-        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
-        "warmup": warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if dtype == torch.bfloat16 else "f16", "data": "synthetic",
-        "config": dict({"workload": spec["description"], "B": B, "H": H, "N": N, "d": d,
-                        "causal": causal, "step": f"{names[0]} + {names[1]}",
-                        "flops_per_step": step_flops, "parallelism": f"replicas x{world}",
-                        "l2": "inputs larger than L2 (4 x 128 MiB per step), no flush"}, **cfg),
-        "fwd": {"ms": fwd_ms, "tflops": fwd_tf, "frac": fwd_tf / peak},
-        "bwd": {"ms": bwd_ms, "tflops": bwd_tf, "frac": bwd_tf / peak},
-        "roofline": {"bound": "tensor", "kernel": f"{names[1]} (preprocess + main + postprocess)",
-                     "achieved": bwd_tf, "peak": peak, "unit": "TFLOP/s", "frac": bwd_tf / peak,
-                     "traffic": None, "peak_source": f"{peak_src} bf16 dense (burst)",
-                     "flops_per_launch": f_bwd},
-        "roofline_fwd": {"bound": "tensor", "kernel": f"fa_fwd_kernel ({names[0]})",
-                         "achieved": fwd_tf, "peak": peak, "unit": "TFLOP/s",
-                         "frac": fwd_tf / peak, "traffic": None,
-                         "peak_source": f"{peak_src} bf16 dense (burst)", "flops_per_launch": f_fwd},
-        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 4 * K, "clocks": clk,
-    }
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
-    return 0
+    config = dict({"workload": spec["description"], "B": B, "H": H, "N": N, "d": d,
+                   "causal": causal, "step": f"{names[0]} + {names[1]}",
+                   "flops_per_step": step_flops, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (4 x 128 MiB per step), no flush"}, **cfg)
+    line = _base_line(value, K, warmup, total_ms, world,
+                      "bf16" if dtype == torch.bfloat16 else "f16", config,
+                      {"ms": fwd_ms, "tflops": roofline_fwd["achieved"],
+                       "frac": roofline_fwd["frac"]},
+                      {"ms": bwd_ms, "tflops": roofline["achieved"], "frac": roofline["frac"]},
+                      roofline, roofline_fwd, cpu, e2e, clk, 4)
+    return _emit(line, rank, world)
 
 
 def main():
