@@ -1,7 +1,7 @@
 """Throughput of exact tiled attention (forward + backward) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload mid|small|long|ragged|tiny|varlen|sparse|dropout]
+                    [--workload mid|small|long|ragged|tiny|varlen|sparse|dropout|fp8]
 
 One step is the whole hot path over one batch: fa_fwd, then the three
 backward stages (row-dot preprocess, main kernel, dQ convert), on the
@@ -23,6 +23,11 @@ the first key tile.
 
 ``--workload dropout`` times dropout on the probabilities (fa_fwd_dropout +
 fa_bwd_dropout, p = 0.1) on the mid workload.
+
+``--workload fp8`` times the 8-bit path on the mid workload's draws:
+fa_quantize_e4m3 of Q, K and V, then fa_fwd_e4m3 (forward only; its FLOPs
+are the forward's, against the bf16 peak times the nominal e4m3 : bf16
+ratio of 2).
 
 ``--impl reference`` times the float64 CPU oracle (test infrastructure, the
 only other place this script runs it) on bounded samples of the same
@@ -76,7 +81,7 @@ def load_peaks():
 
 # Files that hold device code (the kernels and the device helpers they use);
 # the host API in fa_api.cu does not change what a kernel moves.
-KERNEL_SOURCES = ("fa_bwd.cu", "fa_fwd.cu", "fa_internal.h", "sm100.cuh")
+KERNEL_SOURCES = ("fa_bwd.cu", "fa_fwd.cu", "fa_internal.h", "fa_quant.cu", "sm100.cuh")
 
 
 def kernel_source_sha():
@@ -704,9 +709,107 @@ def run_ours_variant(args, spec):
     return _emit(line, rank, world)
 
 
+# --------------------------------------------------------------- 8-bit path
+def run_ours_fp8(args, spec):
+    """``--workload fp8``: one step = fa_quantize_e4m3 of Q, K and V (bf16 to
+    e4m3 with one descale per 128-row tile) + fa_fwd_e4m3."""
+    torch, world, rank, dev, _lib, fa = _cuda_setup()
+    from exact_io_aware_47_b200.inputs import WORKLOADS, make_inputs
+
+    w = WORKLOADS[spec["base"]]
+    B, H, N, d = w.B, w.H, w.N, w.d
+    causal, scale = w.causal, w.scale
+    nt = (N + 127) // 128
+    inp = make_inputs(w.name, dtype=torch.bfloat16, seed=rank, with_do=False, device=dev)
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    q8, k8, v8 = (torch.empty(q.shape, dtype=torch.float8_e4m3fn, device=dev) for _ in range(3))
+    sq, sk, sv = (torch.empty((B, H, nt), dtype=torch.float32, device=dev) for _ in range(3))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    trio = ((q, q8, sq), (k, k8, sk), (v, v8, sv))
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        for x, x8, ds in trio:
+            _lib.check("fa_quantize_e4m3", _lib.fa_quantize_e4m3(
+                x.data_ptr(), x8.data_ptr(), ds.data_ptr(), B, H, N, d, _lib.FA_BF16, sh))
+        if ev is not None:
+            ev[1].record(stream)
+        _lib.check("fa_fwd_e4m3", _lib.fa_fwd_e4m3(
+            q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), sq.data_ptr(), sk.data_ptr(),
+            sv.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, N, d, scale, int(causal), None,
+            _lib.FA_BF16, sh))
+        if ev is not None:
+            ev[2].record(stream)
+
+    warmup, total_ms, (quant_ms, fwd_ms), clk = _timed_steps(torch, step, 3, args, world, dev,
+                                                             stream, _lib)
+    K = args.steps
+    f_fwd = flops_fwd(B, H, N, d, causal)
+    value = world * f_fwd * K / (total_ms / 1e3) / 1e12
+    peaks, peak_src = load_peaks()
+    peak8 = 2.0 * float(peaks["bf16_tflops"])
+    roofline = _roof("fa_fwd_kernel (e4m3)", f_fwd, fwd_ms, peak8, peak_src)
+    roofline["peak_source"] = (f"{peak_src} bf16 dense (burst) x 2, the nominal e4m3 : bf16 dense "
+                               "ratio (4.5 : 2.25 PFLOP/s)")
+    q_bytes = 3 * (q.numel() * (2 + 1) + B * H * nt * 4)      # read bf16, write codes, descales
+    q_gbs = q_bytes / (quant_ms / 1e3) / 1e9
+    hbm = float(peaks["hbm_gbs"])
+    roof_q = {"bound": "hbm", "kernel": "fa_quantize_e4m3 (Q, K, V)", "achieved": q_gbs,
+              "peak": hbm, "unit": "GB/s", "frac": q_gbs / hbm, "traffic": None,
+              "peak_source": f"{peak_src} HBM copy", "bytes_per_step": q_bytes}
+
+    e2e = None
+    if not args.no_e2e:
+        def api_step():
+            for x, x8, ds in trio:
+                fa.quantize_e4m3(x, out=x8, descale=ds)
+            fa.forward_e4m3(q8, k8, v8, sq, sk, sv, scale=scale, causal=causal, out=o, lse=lse)
+        e2e = _e2e(torch, (q, k, v), (o, lse), api_step, K, world, dev, stream, f_fwd)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle.fp8 import quantize_tiles, ref_fwd_fp8_slice
+        n_rows = min(2048, N)  # slices cut to their first n_rows queries and keys
+
+        def samples():
+            for b in range(B):
+                for h in range(H):
+                    xs = [t[b, h, :n_rows].float().cpu().numpy() for t in (q, k, v)]
+
+                    def one(xs=xs):
+                        (qc, qs), (kc, ks), (vc, vs) = (quantize_tiles(x) for x in xs)
+                        return ref_fwd_fp8_slice(qc, kc, vc, qs, ks, vs, scale, causal)
+                    yield one, flops_fwd(1, 1, n_rows, d, causal)
+        val, thr, n_done, dt = _cpu_oracle(samples())
+        cpu = {"value": val, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+               "sample": f"oracle quantisation + e4m3 forward of {n_done} (batch, head) slices "
+                         f"cut to their first {n_rows} queries and keys ({dt:.1f} s)"}
+
+    config = {"workload": spec["description"], "B": B, "H": H, "N": N, "d": d, "causal": causal,
+              "step": "fa_quantize_e4m3 (Q, K, V) + fa_fwd_e4m3 (forward only)",
+              "flops_per_step": f_fwd, "parallelism": f"replicas x{world}",
+              "l2": "inputs larger than L2 (3 x 128 MiB bf16 per step), no flush"}
+    line = _base_line(value, K, warmup, total_ms, world, "e4m3", config,
+                      {"ms": fwd_ms, "tflops": roofline["achieved"], "frac": roofline["frac"]},
+                      None, roofline, roofline, cpu, e2e, clk, 4)
+    line["kernels"] = {"fa_quantize_e4m3 (x3)": {"ms": quant_ms, "share": quant_ms * K / total_ms},
+                       "fa_fwd_kernel (e4m3)": {"ms": fwd_ms, "share": fwd_ms * K / total_ms}}
+    line["roofline_quantize"] = roof_q
+    return _emit(line, rank, world)
+
+
 def main():
     args = parse()
-    from exact_io_aware_47_b200.inputs import BLOCKSPARSE_WORKLOADS, PACKED_WORKLOADS, WORKLOADS
+    from exact_io_aware_47_b200.inputs import (BLOCKSPARSE_WORKLOADS, E4M3_WORKLOADS,
+                                               PACKED_WORKLOADS, WORKLOADS)
+    if args.workload in E4M3_WORKLOADS:
+        if args.impl == "reference":
+            raise SystemExit("--impl reference times the dense workloads")
+        return run_ours_fp8(args, E4M3_WORKLOADS[args.workload])
     if args.workload in BLOCKSPARSE_WORKLOADS:
         if args.impl == "reference":
             raise SystemExit("--impl reference times the dense workloads")

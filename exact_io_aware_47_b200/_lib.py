@@ -21,6 +21,7 @@ FA_ERR_DEVICE_SEQLEN = 7
 FA_ERR_WORKSPACE = 8
 FA_ERR_DEVICE_LAYOUT = 9
 FA_ERR_SCRATCH_LIMIT = 10
+FA_ERR_DEVICE_SCALE = 11
 
 FA_BF16 = 0
 FA_FP16 = 1
@@ -51,6 +52,9 @@ SIGNATURES = {
     "fa_fwd_varlen": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _I, _VP]),
     "fa_bwd_varlen": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP,
                            _I, _I, _I, _I, _I, _F, _I, _I, _VP]),
+    "fa_quantize_e4m3": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP]),
+    "fa_fwd_e4m3": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _VP, _I,
+                         _VP]),
     "fa_device_status": (_I, [_VP, ctypes.POINTER(ctypes.c_uint32)]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_version": (_I, []),
@@ -165,6 +169,16 @@ def fa_bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes,
                   T, max_seqlen, d, scale, causal, dtype, stream):
     return load().fa_bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes,
                                 cu_seqlens, B, H, T, max_seqlen, d, scale, causal, dtype, stream)
+
+
+def fa_quantize_e4m3(x, x8, descale, B, H, N, d, dtype, stream):
+    return load().fa_quantize_e4m3(x, x8, descale, B, H, N, d, dtype, stream)
+
+
+def fa_fwd_e4m3(q8, k8, v8, q_descale, k_descale, v_descale, o, lse, B, H, N, d, scale, causal,
+                seqlens, out_dtype, stream):
+    return load().fa_fwd_e4m3(q8, k8, v8, q_descale, k_descale, v_descale, o, lse, B, H, N, d,
+                              scale, causal, seqlens, out_dtype, stream)
 
 
 def fa_bwd_noalloc_max_bytes():

@@ -3,7 +3,8 @@
 ``forward`` and ``backward`` ([B, H, N, d]), ``forward_dropout`` /
 ``backward_dropout`` (dropout on the probabilities), ``forward_blocksparse`` /
 ``backward_blocksparse`` (the same with a 128 x 128 tile mask) and
-``forward_varlen`` / ``backward_varlen`` (packed [H, T, d] with cu_seqlens)
+``forward_varlen`` / ``backward_varlen`` (packed [H, T, d] with cu_seqlens),
+``quantize_e4m3`` / ``forward_e4m3`` (8-bit inputs with per-tile descales)
 validate tensor
 properties that ctypes cannot see (device, dtype, contiguity, shapes),
 allocate the outputs and the backward workspace with torch, and call the
@@ -278,6 +279,69 @@ def backward_varlen(q, k, v, o, lse, do, cu_seqlens, max_seqlen, scale=None, cau
                                 _stream_handle(dev))
     _lib.check("fa_bwd_varlen", st)
     return dq, dk, dv
+
+
+_E4M3 = (torch.float8_e4m3fn, torch.uint8)
+
+
+def quantize_e4m3(x, out=None, descale=None):
+    """Per-tile e4m3 quantisation of x [B, H, N, d] bf16/fp16 on the GPU.
+
+    Returns (x8 [B, H, N, d] float8_e4m3fn, descale [B, H, ceil(N / 128)]
+    float32): tile t of a slice (rows 128 t ..) stands for x8 * descale[t].
+    """
+    if x.dim() != 4:
+        raise ValueError("x must be [B, H, N, d]")
+    B, H, N, d = x.shape
+    dev = x.device
+    if x.dtype not in _DTYPES:
+        raise ValueError("dtype must be bfloat16 or float16")
+    _check_inputs({"x": x}, (B, H, N, d), x.dtype, dev)
+    nt = (N + 127) // 128
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.float8_e4m3fn, device=dev)
+    if descale is None:
+        descale = torch.empty((B, H, nt), dtype=torch.float32, device=dev)
+    _check_inputs({"out": out}, (B, H, N, d), out.dtype if out.dtype in _E4M3 else None, dev)
+    _check_inputs({"descale": descale}, (B, H, nt), torch.float32, dev)
+    with torch.cuda.device(dev):
+        st = _lib.fa_quantize_e4m3(x.data_ptr(), out.data_ptr(), descale.data_ptr(), B, H, N, d,
+                                   _DTYPES[x.dtype], _stream_handle(dev))
+    _lib.check("fa_quantize_e4m3", st)
+    return out, descale
+
+
+def forward_e4m3(q8, k8, v8, q_descale, k_descale, v_descale, scale=None, causal=False,
+                 seqlens=None, out_dtype=torch.bfloat16, out=None, lse=None):
+    """O, LSE of attention on e4m3 inputs ([B, H, N, 128] float8_e4m3fn or
+    uint8 codes, descales [B, H, ceil(N / 128)] float32); O in out_dtype."""
+    if q8.dim() != 4:
+        raise ValueError("q8 must be [B, H, N, d]")
+    B, H, N, d = q8.shape
+    dev = q8.device
+    if q8.dtype not in _E4M3:
+        raise ValueError("q8 must be float8_e4m3fn or uint8 codes")
+    if out_dtype not in _DTYPES:
+        raise ValueError("out_dtype must be bfloat16 or float16")
+    _check_inputs({"q8": q8, "k8": k8, "v8": v8}, (B, H, N, d), q8.dtype, dev)
+    nt = (N + 127) // 128
+    _check_inputs({"q_descale": q_descale, "k_descale": k_descale, "v_descale": v_descale},
+                  (B, H, nt), torch.float32, dev)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=out_dtype, device=dev)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    _check_inputs({"out": out}, (B, H, N, d), out_dtype, dev)
+    _check_inputs({"lse": lse}, (B, H, N), torch.float32, dev)
+    sl, sl_ptr = _seqlens_arg(seqlens, B, dev)
+    with torch.cuda.device(dev):
+        st = _lib.fa_fwd_e4m3(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), q_descale.data_ptr(),
+                              k_descale.data_ptr(), v_descale.data_ptr(), out.data_ptr(),
+                              lse.data_ptr(), B, H, N, d, scale, int(bool(causal)), sl_ptr,
+                              _DTYPES[out_dtype], _stream_handle(dev))
+    _lib.check("fa_fwd_e4m3", st)
+    return out, lse
 
 
 def device_status(device=None):

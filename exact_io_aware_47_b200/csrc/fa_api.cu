@@ -91,6 +91,21 @@ int make_map(CUtensorMap* map, const void* ptr, int BH, int N, int d, int dtype)
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
+// [B*H, N, 128] e4m3 view: box = 128 columns (128 bytes) x 128 rows, 128-byte
+// swizzle; in bytes the same tiles as the 16-bit d = 64 layout.
+int make_map_e4m3(CUtensorMap* map, const void* ptr, int BH, int N, int d) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N) * d};
+  const cuuint32_t box[3] = {128, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims,
+                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
 // [B*H, N, d] fp32 view of the dQ accumulator for TMA reduce-adds of 128 rows
 // x 32 columns; rows past N inside a head are skipped.
 int make_map_acc(CUtensorMap* map, void* ptr, int BH, int N, int d) {
@@ -125,7 +140,9 @@ int fwd_core(const void* q, const void* k, const void* v, void* o, float* lse, i
              int N, int d, float scale, int causal, const int32_t* seqlens,
              const int32_t* cu_seqlens, int max_seqlen, int dtype, void* stream,
              const uint8_t* block_mask = nullptr, uint32_t keep_t = 256u, float inv_keep = 1.f,
-             uint64_t seed = 0, uint32_t drop_offset = 0) {
+             uint64_t seed = 0, uint32_t drop_offset = 0, const float* q_descale = nullptr,
+             const float* k_descale = nullptr, const float* v_descale = nullptr) {
+  const bool e4m3 = q_descale != nullptr;  // q, k, v are e4m3 codes; dtype is O's type
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
       (seqlens && (reinterpret_cast<uintptr_t>(seqlens) & 3u)) ||
       (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)))
@@ -136,10 +153,16 @@ int fwd_core(const void* q, const void* k, const void* v, void* o, float* lse, i
 
   CUtensorMap tq, tk, tv;
   const int blocks = cu_seqlens ? H : B * H;  // row blocks of N rows
-  if (make_map(&tq, q, blocks, N, d, dtype) != FA_OK ||
-      make_map(&tk, k, blocks, N, d, dtype) != FA_OK ||
-      make_map(&tv, v, blocks, N, d, dtype) != FA_OK)
+  if (e4m3) {
+    if (make_map_e4m3(&tq, q, blocks, N, d) != FA_OK ||
+        make_map_e4m3(&tk, k, blocks, N, d) != FA_OK ||
+        make_map_e4m3(&tv, v, blocks, N, d) != FA_OK)
+      return FA_ERR_CUDA;
+  } else if (make_map(&tq, q, blocks, N, d, dtype) != FA_OK ||
+             make_map(&tk, k, blocks, N, d, dtype) != FA_OK ||
+             make_map(&tv, v, blocks, N, d, dtype) != FA_OK) {
     return FA_ERR_CUDA;
+  }
 
   FwdParams p;
   p.o = o;
@@ -153,6 +176,9 @@ int fwd_core(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.seed_lo = static_cast<uint32_t>(seed);
   p.seed_hi = static_cast<uint32_t>(seed >> 32);
   p.drop_offset = drop_offset;
+  p.q_descale = q_descale;
+  p.k_descale = k_descale;
+  p.v_descale = v_descale;
   p.B = B;
   p.H = H;
   p.N = N;
@@ -162,7 +188,10 @@ int fwd_core(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.n_pairs = (p.n_qtiles + 1) / 2;
   p.n_units = B * H * ((p.n_pairs + 1) / 2);
   const cudaError_t e =
-      launch_fwd(d, dtype == FA_BF16, tq, tk, tv, p, di.num_sms, static_cast<cudaStream_t>(stream));
+      e4m3 ? launch_fwd_e4m3(dtype == FA_BF16, tq, tk, tv, p, di.num_sms,
+                             static_cast<cudaStream_t>(stream))
+           : launch_fwd(d, dtype == FA_BF16, tq, tk, tv, p, di.num_sms,
+                        static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -236,6 +265,39 @@ extern "C" int fa_fwd_varlen(const void* q, const void* k, const void* v, void* 
   if (st != FA_OK) return st;
   return fwd_core(q, k, v, o, lse, B, H, T, d, scale, causal, nullptr, cu_seqlens,
                   max_seqlen < T ? max_seqlen : T, dtype, stream);
+}
+
+extern "C" int fa_fwd_e4m3(const void* q8, const void* k8, const void* v8, const float* q_descale,
+                           const float* k_descale, const float* v_descale, void* o, float* lse,
+                           int B, int H, int N, int d, float scale, int causal,
+                           const int32_t* seqlens, int out_dtype, void* stream) {
+  if (!q8 || !k8 || !v8 || !q_descale || !k_descale || !v_descale || !o || !lse)
+    return FA_ERR_INVALID_ARG;
+  const int st = check_common(B, H, N, d, scale, out_dtype);
+  if (st != FA_OK) return st;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  const uintptr_t ds_bits = reinterpret_cast<uintptr_t>(q_descale) |
+                            reinterpret_cast<uintptr_t>(k_descale) |
+                            reinterpret_cast<uintptr_t>(v_descale);
+  if (ds_bits & 3u) return FA_ERR_ALIGNMENT;
+  return fwd_core(q8, k8, v8, o, lse, B, H, N, d, scale, causal, seqlens, nullptr, 0, out_dtype,
+                  stream, nullptr, 256u, 1.f, 0, 0, q_descale, k_descale, v_descale);
+}
+
+extern "C" int fa_quantize_e4m3(const void* x, void* x8, float* descale, int B, int H, int N,
+                                int d, int dtype, void* stream) {
+  if (!x || !x8 || !descale) return FA_ERR_INVALID_ARG;
+  const int st = check_common(B, H, N, d, 1.f, dtype);
+  if (st != FA_OK) return st;
+  if (!aligned16(x) || !aligned16(x8) || (reinterpret_cast<uintptr_t>(descale) & 3u))
+    return FA_ERR_ALIGNMENT;
+  DeviceInfo di;
+  const int dst = current_device_info(&di);
+  if (dst != FA_OK) return dst;
+  const cudaError_t e =
+      launch_quantize_e4m3(d, dtype == FA_BF16, x, x8, descale, static_cast<long long>(B) * H, N,
+                           di.num_sms, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 extern "C" size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
@@ -550,6 +612,7 @@ extern "C" int fa_device_status(void* stream, uint32_t* detail) {
   if (code == kErrDeviceTimeout) return FA_ERR_DEVICE_TIMEOUT;
   if (code == kErrDeviceSeqlen) return FA_ERR_DEVICE_SEQLEN;
   if (code == kErrDeviceLayout) return FA_ERR_DEVICE_LAYOUT;
+  if (code == kErrDeviceScale) return FA_ERR_DEVICE_SCALE;
   return word == 0 ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -567,6 +630,7 @@ extern "C" const char* fa_status_string(int status) {
     case FA_ERR_DEVICE_LAYOUT: return "kernel refused: shared-memory window misaligned";
     case FA_ERR_SCRATCH_LIMIT:
       return "problem needs more backward scratch than fa_bwd_noalloc's static array holds";
+    case FA_ERR_DEVICE_SCALE: return "e4m3 descale factor not finite and positive, or infinite input";
     default: return "unknown status";
   }
 }

@@ -33,12 +33,14 @@
 
 namespace fa {
 
-template <int D>
+template <int D, int ESZ>
 struct FwdLayout {
-  static constexpr int kTileBytes = kBlockM * D * 2;  // one 128-row, d-wide 16-bit tile
-  static constexpr int kPanelBytes = 128 * 64 * 2;    // one 64-column swizzle panel (16 KB)
-  static constexpr int kPanels = D / 64;
-  static constexpr int kSlots = (D == 128) ? 4 : 8;   // K/V ring depth
+  static constexpr int kRowBytes = D * ESZ;            // ESZ = element bytes (2, or 1 for e4m3)
+  static constexpr int kTileBytes = kBlockM * kRowBytes;  // one 128-row, d-wide tile
+  static constexpr int kPanelBytes = 128 * 128;        // 128 rows x 128 bytes: one swizzle panel
+  static constexpr int kPanels = kRowBytes / 128;
+  static constexpr int kPanelElems = 128 / ESZ;        // row elements inside one panel
+  static constexpr int kSlots = (kTileBytes == 32768) ? 4 : 8;  // K/V ring depth
   static constexpr int kQ0 = 0;
   static constexpr int kSlot0 = 2 * kTileBytes;
   static constexpr int kBar = kSlot0 + kSlots * kTileBytes;
@@ -116,11 +118,12 @@ __device__ __forceinline__ FwdUnit fwd_decode(int bh, int pair, const FwdParams&
   return w;
 }
 
-template <int D, bool BF16, bool PACKED, bool SPARSE, bool DROPOUT>
+template <int D, bool BF16, bool PACKED, bool SPARSE, bool DROPOUT, bool FP8>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv, const FwdParams p) {
-  using Lay = FwdLayout<D>;
+  using Lay = FwdLayout<D, FP8 ? 1 : 2>;
+  static_assert(!FP8 || (D == 128 && !PACKED && !SPARSE && !DROPOUT), "e4m3: dense, d = 128");
   constexpr int kSlots = Lay::kSlots;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -193,7 +196,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int pn = 0; pn < Lay::kPanels; ++pn)
             tma_load_3d(sq + t * Lay::kTileBytes + pn * Lay::kPanelBytes, &tmq, &q_full[t],
-                        pn * 64, w.row0 + (w.qt0 + t) * kBlockM, w.z);
+                        pn * Lay::kPanelElems, w.row0 + (w.qt0 + t) * kBlockM, w.z);
           ++qload[t];
         }
         const int jmax = max(je[0], je[1]);
@@ -207,8 +210,8 @@ __global__ void __launch_bounds__(384, 1)
             uint8_t* dst = skv + slot * Lay::kTileBytes;
 #pragma unroll
             for (int pn = 0; pn < Lay::kPanels; ++pn)
-              tma_load_3d(dst + pn * Lay::kPanelBytes, kv ? &tmv : &tmk, &kv_full[slot], pn * 64,
-                          w.row0 + j * kBlockN, w.z);
+              tma_load_3d(dst + pn * Lay::kPanelBytes, kv ? &tmv : &tmk, &kv_full[slot],
+                          pn * Lay::kPanelElems, w.row0 + j * kBlockN, w.z);
             ++kv_seq;
           }
         }
@@ -228,8 +231,10 @@ __global__ void __launch_bounds__(384, 1)
   } else if (warp == 8) {
     // ------------------------------------------------------------- MMA issue
     if (lane == 0) {
-      constexpr uint32_t kIdescQK = idesc_f16(BF16, 128, 128, false, false);
-      constexpr uint32_t kIdescPV = idesc_f16(BF16, 128, D, false, true);
+      constexpr uint32_t kIdescQK =
+          FP8 ? idesc_e4m3(128, 128, false, false) : idesc_f16(BF16, 128, 128, false, false);
+      constexpr uint32_t kIdescPV =
+          FP8 ? idesc_e4m3(128, D, false, true) : idesc_f16(BF16, 128, D, false, true);
       const uint32_t sq_addr = smem_addr(sq);
       const uint32_t skv_addr = smem_addr(skv);
       int qload[2] = {0, 0};
@@ -244,14 +249,22 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t lKV_k = sdesc_lo(skv_addr, false), lKV_m = sdesc_lo(skv_addr, true);
       // S_t = Q_t K^T: A = Q tile (K-major), B = K tile (K-major).
       auto issue_s = [&](int t, int kslot) {
-        umma_ss_group<D / 16, false, false>(tmem + t * 128, lQ_k + t * kTileLo,
-                                            lKV_k + kslot * kTileLo, kIdescQK, 0u);
+        if constexpr (FP8)
+          umma_ss_group4_e4m3(tmem + t * 128, lQ_k + t * kTileLo, lKV_k + kslot * kTileLo,
+                              kIdescQK, 0u);
+        else
+          umma_ss_group<D / 16, false, false>(tmem + t * 128, lQ_k + t * kTileLo,
+                                              lKV_k + kslot * kTileLo, kIdescQK, 0u);
       };
-      // O_t += P_t V: A = P (16-bit, TMEM, over S_t, 8 columns per 16 keys),
-      // B = V tile read MN-major (d contiguous).
+      // O_t += P_t V: A = P (TMEM, over S_t: 16-bit, 8 columns per 16 keys, or
+      // e4m3, 8 columns per 32 keys), B = V tile read MN-major (d contiguous).
       auto issue_pv = [&](int t, int vslot, bool acc) {
-        umma_ts_group8<true, false>(tmem + Lay::kColO + t * D, tmem + t * 128,
-                                    lKV_m + vslot * kTileLo, kIdescPV, acc ? 1u : 0u);
+        if constexpr (FP8)
+          umma_ts_group4_e4m3(tmem + Lay::kColO + t * D, tmem + t * 128,
+                              lKV_m + vslot * kTileLo, kIdescPV, acc ? 1u : 0u);
+        else
+          umma_ts_group8<true, false>(tmem + Lay::kColO + t * D, tmem + t * 128,
+                                      lKV_m + vslot * kTileLo, kIdescPV, acc ? 1u : 0u);
       };
 
       for (int k = 0; ok; ++k) {
@@ -371,6 +384,24 @@ __global__ void __launch_bounds__(384, 1)
         }
         continue;
       }
+      // e4m3 inputs: the query tile's descale and the largest V descale of
+      // the slice's valid key tiles; key tile j's probabilities are scaled by
+      // sv_j / sv_max before they are rounded to 8 bits, and O by sv_max at
+      // the end, so one TMEM accumulator serves tiles of any V scale
+      float sq_t = 1.f, sv_max = 1.f;
+      const float* kds = nullptr;
+      const float* vds = nullptr;
+      if constexpr (FP8) {
+        const size_t base = static_cast<size_t>(w.bh) * p.n_qtiles;
+        kds = p.k_descale + base;
+        vds = p.v_descale + base;
+        sq_t = p.q_descale[base + qt];
+        const int nkb = (w.L + kBlockN - 1) / kBlockN;
+        sv_max = 0.f;
+        for (int jv = 0; jv < nkb; ++jv) sv_max = fmaxf(sv_max, vds[jv]);
+        if (!(sq_t > 0.f && sq_t < INFINITY && sv_max > 0.f && sv_max < INFINITY))
+          record_error(kErrDeviceScale, 0);
+      }
       float m = -INFINITY;  // running max, log2 units
       float l = 0.f;        // running sum of unnormalised probabilities
       int jj = 0;           // key tiles processed so far
@@ -385,6 +416,15 @@ __global__ void __launch_bounds__(384, 1)
             const uint32_t m16 = keep_bits_row16(p, w.bh, row, j, g, lane & 3);
             drop_keep[g >> 1] = (g & 1) ? (drop_keep[g >> 1] & 0xFFFFu) | (m16 << 16) : m16;
           }
+        }
+        // scores of this tile are raw * cj in log2 units
+        float cj = c, rho = 1.f;
+        if constexpr (FP8) {
+          const float skj = kds[j], svj = vds[j];
+          if (!(skj > 0.f && skj < INFINITY && svj > 0.f && svj < INFINITY))
+            record_error(kErrDeviceScale, 1);
+          cj = c * sq_t * skj;
+          rho = svj / sv_max;
         }
         ok = mbar_wait_warp(&s_full[t], scnt & 1, abort_flag, 8);
         if (!ok) break;
@@ -413,7 +453,7 @@ __global__ void __launch_bounds__(384, 1)
           for (int q4 = 0; q4 < 4; ++q4)
             mc[q4] = fmax3(mc[q4], __uint_as_float(sr[i + 2 * q4]), __uint_as_float(sr[i + 2 * q4 + 1]));
         }
-        const float mx = fmax3(mc[0], mc[1], fmaxf(mc[2], mc[3])) * c;  // log2 units (c > 0)
+        const float mx = fmax3(mc[0], mc[1], fmaxf(mc[2], mc[3])) * cj;  // log2 units (cj > 0)
         const float m_new = (mx > m + kRescaleThreshold) ? mx : m;
         const bool moved = m_new != m;
         const float alpha = moved ? ex2_approx(m - m_new) : 1.f;  // 0 when m was -inf
@@ -422,10 +462,10 @@ __global__ void __launch_bounds__(384, 1)
         // p = 2^(c s - m): packed FMA on pairs, then ex2; row sum in fp32 over
         // four packed accumulators
         const float mu = (m == -INFINITY) ? 0.f : m;
-        const unsigned long long c2 = f2pack(c, c);
+        const unsigned long long c2 = f2pack(cj, cj);
         const unsigned long long nm2 = f2pack(-mu, -mu);
         unsigned long long acc[4] = {0ull, 0ull, 0ull, 0ull};
-        uint32_t pk[64];
+        uint32_t pk[FP8 ? 32 : 64];  // P as the A operand: 16-bit pairs or e4m3 quads
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
           const unsigned long long x2 =
@@ -440,7 +480,12 @@ __global__ void __launch_bounds__(384, 1)
             p0 = (drop_keep[i >> 4] >> ((2 * i) & 31)) & 1u ? p0 : 0.f;
             p1 = (drop_keep[i >> 4] >> ((2 * i + 1) & 31)) & 1u ? p1 : 0.f;
           }
-          pk[i] = pack2<BF16>(p0, p1);
+          if constexpr (FP8) {
+            const uint32_t h = pack_e4m3x2(p0 * rho, p1 * rho);
+            pk[i >> 1] = (i & 1) ? (pk[i >> 1] | (h << 16)) : h;
+          } else {
+            pk[i] = pack2<BF16>(p0, p1);
+          }
         }
         {
           float a0, a1, b0, b1, c0, c1, d0, d1;
@@ -450,7 +495,8 @@ __global__ void __launch_bounds__(384, 1)
           f2unpack(acc[3], d0, d1);
           l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
         }
-        tmem_st64(tS, pk);
+        if constexpr (FP8) tmem_st32(tS, pk);
+        else tmem_st64(tS, pk);
         if (jj > 0 && __any_sync(0xffffffffu, moved)) {
           // O_t holds the sum up to the previous key tile (its MMA completed
           // before S_t(j) was committed) and PV_t(j) waits for p_full:
@@ -476,8 +522,9 @@ __global__ void __launch_bounds__(384, 1)
       if (!ok) break;
       ++ocnt;
       tc_fence_after();
-      // (with dropout the kept scores are scaled by 256 / t once, here)
-      const float inv_l = DROPOUT ? p.inv_keep / l : 1.f / l;
+      // (with dropout the kept scores are scaled by 256 / t once, here; with
+      // e4m3 inputs the V descale ratio is undone)
+      const float inv_l = FP8 ? sv_max / l : (DROPOUT ? p.inv_keep / l : 1.f / l);
       const bool store = row < w.rows;
       const size_t orow_idx = static_cast<size_t>(w.z) * p.N + w.row0 + (store ? row : 0);
       uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) + orow_idx * (D * 2);
@@ -508,12 +555,12 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
-template <int D, bool BF16, bool PACKED, bool SPARSE, bool DROPOUT>
+template <int D, bool BF16, bool PACKED, bool SPARSE, bool DROPOUT, bool FP8 = false>
 static cudaError_t launch_fwd_t(const CUtensorMap& tmq, const CUtensorMap& tmk,
                                 const CUtensorMap& tmv, const FwdParams& p, int num_sms,
                                 cudaStream_t stream) {
-  using Lay = FwdLayout<D>;
-  auto kern = fa_fwd_kernel<D, BF16, PACKED, SPARSE, DROPOUT>;
+  using Lay = FwdLayout<D, FP8 ? 1 : 2>;
+  auto kern = fa_fwd_kernel<D, BF16, PACKED, SPARSE, DROPOUT, FP8>;
   cudaFuncAttributes attr;
   cudaError_t e = cudaFuncGetAttributes(&attr, kern);
   if (e != cudaSuccess) return e;
@@ -544,6 +591,14 @@ cudaError_t launch_fwd(int d, bool bf16, const CUtensorMap& tmq, const CUtensorM
   return bf16 ? FA_FWD_MODES(64, true) : FA_FWD_MODES(64, false);
 #undef FA_FWD_MODES
 #undef FA_FWD_LAUNCH
+}
+
+cudaError_t launch_fwd_e4m3(bool bf16, const CUtensorMap& tmq, const CUtensorMap& tmk,
+                            const CUtensorMap& tmv, const FwdParams& p, int num_sms,
+                            cudaStream_t stream) {
+  return bf16 ? launch_fwd_t<128, true, false, false, false, true>(tmq, tmk, tmv, p, num_sms, stream)
+              : launch_fwd_t<128, false, false, false, false, true>(tmq, tmk, tmv, p, num_sms,
+                                                                    stream);
 }
 
 }  // namespace fa

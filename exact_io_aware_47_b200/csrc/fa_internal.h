@@ -35,6 +35,11 @@ struct FwdParams {
   // 8-bit keep threshold t (1..256) and 256 / t
   uint32_t seed_lo, seed_hi, drop_offset, keep_t;
   float inv_keep;
+  // e4m3 inputs (kernels instantiated with FP8): one descale factor per
+  // 128-row tile, [B, H, n_qtiles] each; the tensors stand for code * descale
+  const float* q_descale;
+  const float* k_descale;
+  const float* v_descale;
   int B, H, N;
   float scale_log2;         // scale * log2(e)
   int causal;
@@ -189,6 +194,13 @@ __device__ __forceinline__ bool work_item(int k, int per_head, int heads, WorkIt
 cudaError_t launch_fwd(int d, bool bf16, const CUtensorMap& tmq, const CUtensorMap& tmk,
                        const CUtensorMap& tmv, const FwdParams& p, int num_sms,
                        cudaStream_t stream);
+// e4m3 inputs (p.q_descale set), d = 128; bf16 selects the output type.
+cudaError_t launch_fwd_e4m3(bool bf16, const CUtensorMap& tmq, const CUtensorMap& tmk,
+                            const CUtensorMap& tmv, const FwdParams& p, int num_sms,
+                            cudaStream_t stream);
+// Per-tile e4m3 quantisation of a [rows_total / n_rows, n_rows, d] 16-bit tensor.
+cudaError_t launch_quantize_e4m3(int d, bool bf16, const void* x, void* x8, float* descale,
+                                 long long slices, int n_rows, int num_sms, cudaStream_t stream);
 
 cudaError_t launch_bwd_pre(int d, bool bf16, const BwdParams& p, int num_sms,
                            cudaStream_t stream);

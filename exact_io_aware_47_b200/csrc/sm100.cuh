@@ -19,7 +19,12 @@ namespace fa {
 // ---------------------------------------------------------------------------
 __device__ unsigned int g_error_word = 0;
 
-enum : unsigned { kErrDeviceTimeout = 6u, kErrDeviceSeqlen = 7u, kErrDeviceLayout = 9u };
+enum : unsigned {
+  kErrDeviceTimeout = 6u,
+  kErrDeviceSeqlen = 7u,
+  kErrDeviceLayout = 9u,
+  kErrDeviceScale = 11u  // an 8-bit descale factor (or a quantised tile's amax) not finite and > 0
+};
 
 __device__ __forceinline__ void record_error(unsigned code, unsigned site) {
   unsigned w = (code & 0xffu) | ((site & 0xffu) << 8) | ((blockIdx.x & 0xffffu) << 16);
@@ -232,6 +237,18 @@ __host__ __device__ constexpr uint32_t idesc_f16(bool bf16, int M, int N, bool a
          | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
 
+// Instruction descriptor, kind::f8f6f4 with fp32 accumulation and both
+// operands e4m3 (format code 0 for A and B; the same bit positions as
+// kind::f16).  8-bit operands may be MN-major (e4m3 and e5m2 allow it).
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4)                                   // D format: f32
+         | (0u << 7) | (0u << 10)                    // A, B format: e4m3
+         | ((a_mn_major ? 1u : 0u) << 15)
+         | ((b_mn_major ? 1u : 0u) << 16)
+         | (static_cast<uint32_t>(N >> 3) << 17)
+         | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
 // ---------------------------------------------------------------------------
 // Grouped MMAs: a whole K = 64 or K = 128 contraction (4 or 8 tcgen05.mma of
 // K = 16) into one accumulator from one asm statement.  Every descriptor of
@@ -328,6 +345,58 @@ __device__ __forceinline__ void umma_ts_group8(uint32_t d_tmem, uint32_t a_tmem,
                "n"(sw128_step(B_MN, 6)), "n"(sw128_step(B_MN, 7))
                : "memory");
 }
+// 8-bit (e4m3) groups: K = 128 as 4 tcgen05.mma of K = 32 (32 bytes), kind
+// f8f6f4.  In bytes the operands are laid out like a 16-bit operand with 64
+// elements per row: K-major steps walk 32 bytes inside the 128-byte swizzled
+// row, MN-major steps walk 32 rows (4096 bytes), and an A operand in TMEM
+// holds four elements per 32-bit column (8 columns per step).
+#define FA_MMA8_SS_FIRST                                                       \
+  "mov.b64 da, {%1, h};\n\tmov.b64 db, {%2, h};\n\t"                           \
+  "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], da, db, %3, p;\n\t"
+#define FA_MMA8_SS_STEP(ao, bo)                                                \
+  "add.u32 a, %1, %" #ao ";\n\tadd.u32 b, %2, %" #bo ";\n\t"                   \
+  "mov.b64 da, {a, h};\n\tmov.b64 db, {b, h};\n\t"                             \
+  "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], da, db, %3, t;\n\t"
+#define FA_MMA8_TS_FIRST                                                       \
+  "mov.b64 db, {%2, h};\n\t"                                                   \
+  "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], db, %3, p;\n\t"
+#define FA_MMA8_TS_STEP(ao, bo)                                                \
+  "add.u32 a, %1, %" #ao ";\n\tadd.u32 b, %2, %" #bo ";\n\t"                   \
+  "mov.b64 db, {b, h};\n\t"                                                    \
+  "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [a], db, %3, t;\n\t"
+
+// Start-address step (16-byte units) of 8-bit K-step kk (32 elements).
+__host__ __device__ constexpr uint32_t sw128_step8(bool mn_major, int kk) {
+  return mn_major ? static_cast<uint32_t>(kk) * 256u : static_cast<uint32_t>(kk) * 2u;
+}
+
+// D (+)= A B over K = 128 e4m3 elements, A and B in shared memory (K-major).
+__device__ __forceinline__ void umma_ss_group4_e4m3(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
+                                                    uint32_t idesc, uint32_t accumulate) {
+  asm volatile(FA_MMA_PROLOGUE FA_MMA8_SS_FIRST FA_MMA8_SS_STEP(6, 9) FA_MMA8_SS_STEP(7, 10)
+                   FA_MMA8_SS_STEP(8, 11) "}" ::"r"(d_tmem),
+               "r"(a_lo), "r"(b_lo), "r"(idesc), "r"(accumulate), "n"(kSdescHi),
+               "n"(sw128_step8(false, 1)), "n"(sw128_step8(false, 2)), "n"(sw128_step8(false, 3)),
+               "n"(sw128_step8(false, 1)), "n"(sw128_step8(false, 2)), "n"(sw128_step8(false, 3))
+               : "memory");
+}
+
+// D (+)= A B over K = 128 e4m3 elements, A in TMEM (32 columns, 4 elements
+// per column, ascending K in ascending bytes), B in shared memory MN-major.
+__device__ __forceinline__ void umma_ts_group4_e4m3(uint32_t d_tmem, uint32_t a_tmem,
+                                                    uint32_t b_lo, uint32_t idesc,
+                                                    uint32_t accumulate) {
+  asm volatile(FA_MMA_PROLOGUE FA_MMA8_TS_FIRST FA_MMA8_TS_STEP(6, 9) FA_MMA8_TS_STEP(7, 10)
+                   FA_MMA8_TS_STEP(8, 11) "}" ::"r"(d_tmem),
+               "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(accumulate), "n"(kSdescHi),
+               "n"(8u), "n"(16u), "n"(24u),
+               "n"(sw128_step8(true, 1)), "n"(sw128_step8(true, 2)), "n"(sw128_step8(true, 3))
+               : "memory");
+}
+#undef FA_MMA8_SS_FIRST
+#undef FA_MMA8_SS_STEP
+#undef FA_MMA8_TS_FIRST
+#undef FA_MMA8_TS_STEP
 #undef FA_MMA_PROLOGUE
 #undef FA_MMA_SS_FIRST
 #undef FA_MMA_SS_STEP
@@ -543,6 +612,18 @@ template <bool BF16>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   if constexpr (BF16) return pack_bf16x2(lo, hi);
   else return pack_f16x2(lo, hi);
+}
+
+// Two fp32 values to two e4m3 bytes (round to nearest even, saturating to
+// +-448): lo in bits 0..7, hi in bits 8..15.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
+  unsigned short r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return static_cast<uint32_t>(r);
+}
+// Four fp32 values to one word of e4m3 bytes, a0 in bits 0..7.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a0, float a1, float a2, float a3) {
+  return pack_e4m3x2(a0, a1) | (pack_e4m3x2(a2, a3) << 16);
 }
 
 // Make this thread's generic-proxy shared-memory writes visible to the async

@@ -184,3 +184,11 @@ BLOCKSPARSE_WORKLOADS = {
                     description="B2 H32 N8192 d128 bf16 causal with dropout p = 0.1 on the "
                                 "probabilities"),
 }
+
+# 8-bit inputs: the dense workload's bf16 draws, quantised to e4m3 with one
+# descale per 128-row tile by the library itself (forward only)
+E4M3_WORKLOADS = {
+    "fp8": dict(base="mid",
+                description="B2 H32 N8192 d128 causal, bf16 draws quantised to e4m3 with one "
+                            "descale per 128-row tile, forward only"),
+}

@@ -67,7 +67,9 @@ typedef enum {
   FA_ERR_DEVICE_SEQLEN = 7,   /* device: seqlens[b] outside [1, N] (fa_device_status) */
   FA_ERR_WORKSPACE = 8,       /* backward workspace missing or too small        */
   FA_ERR_DEVICE_LAYOUT = 9,   /* device: shared-memory window misaligned, kernel refused (fa_device_status) */
-  FA_ERR_SCRATCH_LIMIT = 10   /* fa_bwd_noalloc: workspace would exceed its static array */
+  FA_ERR_SCRATCH_LIMIT = 10,  /* fa_bwd_noalloc: workspace would exceed its static array */
+  FA_ERR_DEVICE_SCALE = 11    /* device: e4m3 descale not finite and > 0, or infinite input to
+                                 fa_quantize_e4m3 (fa_device_status) */
 } fa_status;
 
 typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
@@ -157,6 +159,44 @@ int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o,
                    void* workspace, size_t workspace_bytes, int B, int H, int N, int d,
                    float scale, int causal, const int32_t* seqlens, float p_drop,
                    uint64_t seed, uint32_t offset, int dtype, void* stream);
+
+/*
+ * 8-bit (e4m3) inputs with per-tile scaling: the lower-precision path that
+ * "How Flash Attention Works" (section "FlashAttention 2 and 3") names.
+ *   Format.  e4m3 as in the OCP 8-bit floating-point specification (sign,
+ *     4 exponent bits with bias 7, 3 mantissa bits, largest finite 448, no
+ *     infinities); one byte per element.
+ *   fa_quantize_e4m3: x [B, H, N, d] 16-bit (dtype FA_BF16 / FA_FP16, finite
+ *     values) -> x8 [B, H, N, d] e4m3 codes and descale [B, H, ceil(N/128)]
+ *     float32.  Tile t of a (batch, head) slice is rows 128 t .. 128 t + 127
+ *     (the last tile may be short).  With amax = max |x| over the tile:
+ *     descale = amax / 448 and each code = e4m3(x * (448 / amax)), both
+ *     divisions and the product in fp32 rounded to nearest, the conversion
+ *     round-to-nearest-even and saturating; a tile of zeros gets descale 1.
+ *     d in {64, 128}.  An infinite input is reported as FA_ERR_DEVICE_SCALE.
+ *   fa_fwd_e4m3: forward attention of Q, K, V given as e4m3 codes
+ *     [B, H, N, 128] with descales [B, H, ceil(N/128)] (any positive finite
+ *     values; the quantiser's output is one choice): the tensors stand for
+ *     code * descale of the row's tile.  Scores, masks, seqlens and LSE are
+ *     as in fa_fwd, on those values.  For the product with V the
+ *     probabilities of key tile j (against the running row max, which moves
+ *     only by more than 8 in log2 units) are multiplied by
+ *     sv_j / max sv (the largest V descale of the slice's valid key tiles)
+ *     and rounded to e4m3; the row sum uses them before rounding; O =
+ *     max sv * sum / l in out_dtype (FA_BF16 or FA_FP16) [B, H, N, 128].
+ *     d must be 128 (FA_ERR_UNSUPPORTED otherwise).  Descale pointers must be
+ *     4-byte aligned, the others 16-byte aligned.  A descale that is not
+ *     finite and positive is reported as FA_ERR_DEVICE_SCALE (the results are
+ *     then unspecified).
+ *   Ownership and errors as in fa_fwd: the caller owns every buffer; nothing
+ *   is allocated; the calls enqueue on `stream` and never synchronise.
+ */
+int fa_quantize_e4m3(const void* x, void* x8, float* descale, int B, int H, int N, int d,
+                     int dtype, void* stream);
+int fa_fwd_e4m3(const void* q8, const void* k8, const void* v8, const float* q_descale,
+                const float* k_descale, const float* v_descale, void* o, float* lse,
+                int B, int H, int N, int d, float scale, int causal,
+                const int32_t* seqlens, int out_dtype, void* stream);
 
 /*
  * Packed variable-length batches: B sequences of different lengths stored
@@ -252,8 +292,8 @@ size_t fa_bwd_noalloc_max_bytes(void);
 
 /*
  * Synchronises `stream`, then returns and clears the device status word of
- * the current device: FA_OK, FA_ERR_DEVICE_SEQLEN, FA_ERR_DEVICE_TIMEOUT or
- * FA_ERR_DEVICE_LAYOUT
+ * the current device: FA_OK, FA_ERR_DEVICE_SEQLEN, FA_ERR_DEVICE_TIMEOUT,
+ * FA_ERR_DEVICE_LAYOUT or FA_ERR_DEVICE_SCALE
  * (FA_ERR_CUDA if the synchronisation itself failed).  *detail, if not NULL,
  * receives the raw word (code | site << 8 | block << 16).
  */
