@@ -752,15 +752,17 @@ def run_ours_fp8(args, spec):
     value = world * f_fwd * K / (total_ms / 1e3) / 1e12
     peaks, peak_src = load_peaks()
     peak8 = 2.0 * float(peaks["bf16_tflops"])
-    roofline = _roof("fa_fwd_kernel (e4m3)", f_fwd, fwd_ms, peak8, peak_src)
+    roofline = _roof("fa_fwd_kernel (e4m3)", f_fwd, fwd_ms, peak8, peak_src,
+                     recorded_traffic("fa_fwd_kernel (e4m3)", args.workload))
     roofline["peak_source"] = (f"{peak_src} bf16 dense (burst) x 2, the nominal e4m3 : bf16 dense "
                                "ratio (4.5 : 2.25 PFLOP/s)")
     q_bytes = 3 * (q.numel() * (2 + 1) + B * H * nt * 4)      # read bf16, write codes, descales
     q_gbs = q_bytes / (quant_ms / 1e3) / 1e9
     hbm = float(peaks["hbm_gbs"])
     roof_q = {"bound": "hbm", "kernel": "fa_quantize_e4m3 (Q, K, V)", "achieved": q_gbs,
-              "peak": hbm, "unit": "GB/s", "frac": q_gbs / hbm, "traffic": None,
-              "peak_source": f"{peak_src} HBM copy", "bytes_per_step": q_bytes}
+              "peak": hbm, "unit": "GB/s", "frac": q_gbs / hbm,
+              "traffic": recorded_traffic("fa_quantize_e4m3", args.workload),
+              "peak_source": f"{peak_src} HBM copy", "bytes_per_launch": q_bytes // 3}
 
     e2e = None
     if not args.no_e2e:
