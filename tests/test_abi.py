@@ -45,7 +45,7 @@ def test_binding_covers_every_declared_symbol():
 
 
 def test_status_strings_and_version(lib):
-    for code in range(0, 10):
+    for code in range(0, 12):
         s = lib.fa_status_string(code)
         assert isinstance(s, bytes) and len(s) > 0
     assert lib.fa_version() == 100
@@ -107,3 +107,35 @@ def test_missing_library_fails_loudly(tmp_path):
     from exact_io_aware_47_b200 import _lib
     with pytest.raises(RuntimeError, match="missing"):
         _lib.load(str(tmp_path / "nope.so"))
+
+
+def test_e4m3_rejections_before_any_cuda_call(lib):
+    from exact_io_aware_47_b200 import _lib
+    P = 1 << 20  # never dereferenced: every case below fails validation first
+    ok = dict(B=1, H=2, N=128, d=128, scale=0.125, dtype=0)
+
+    def fwd8(q=P, ds=P, o=P, **kw):
+        a = {**ok, **kw}
+        return lib.fa_fwd_e4m3(q, P, P, ds, ds, ds, o, P, a["B"], a["H"], a["N"], a["d"],
+                               a["scale"], 1, None, a["dtype"], None)
+    assert fwd8(q=None) == _lib.FA_ERR_INVALID_ARG
+    assert fwd8(ds=None) == _lib.FA_ERR_INVALID_ARG
+    assert fwd8(B=0) == _lib.FA_ERR_INVALID_ARG
+    assert fwd8(scale=-1.0) == _lib.FA_ERR_INVALID_ARG
+    assert fwd8(dtype=5) == _lib.FA_ERR_INVALID_ARG
+    assert fwd8(d=64) == _lib.FA_ERR_UNSUPPORTED                # 8-bit path: d = 128 only
+    assert fwd8(d=96) == _lib.FA_ERR_UNSUPPORTED
+    assert fwd8(ds=P + 2) == _lib.FA_ERR_ALIGNMENT              # descales: 4-byte aligned
+    assert fwd8(q=P + 8) == _lib.FA_ERR_ALIGNMENT               # codes: 16-byte aligned
+    assert fwd8(o=P + 4) == _lib.FA_ERR_ALIGNMENT
+
+    def quant(x=P, x8=P, ds=P, **kw):
+        a = {**ok, **kw}
+        return lib.fa_quantize_e4m3(x, x8, ds, a["B"], a["H"], a["N"], a["d"], a["dtype"], None)
+    assert quant(x=None) == _lib.FA_ERR_INVALID_ARG
+    assert quant(N=0) == _lib.FA_ERR_INVALID_ARG
+    assert quant(dtype=3) == _lib.FA_ERR_INVALID_ARG
+    assert quant(d=80) == _lib.FA_ERR_UNSUPPORTED
+    assert quant(x8=P + 8) == _lib.FA_ERR_ALIGNMENT
+    assert quant(ds=P + 1) == _lib.FA_ERR_ALIGNMENT
+    assert lib.fa_status_string(_lib.FA_ERR_DEVICE_SCALE) != b"unknown status"
