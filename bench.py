@@ -60,7 +60,7 @@ def flops_fwd(B, H, N, d, causal):
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="mid")
@@ -109,16 +109,58 @@ def recorded_traffic(kernel, workload):
     return e.get("dram_bytes_per_launch")
 
 
-class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+def summarise_clocks(text, t0=None, t1=None):
+    """Summary of nvidia-smi samples (ClockSampler.Q rows, CSV without units).
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    Keeps the samples whose timestamp lies in [t0, t1] (datetime, the timed
+    region); if none does, the samples nearest to the region's midpoint.
+    Returns the median SM clock, the max clock, the throttle reasons seen
+    active, and how many samples were used."""
+    import datetime
+    rows = []
+    for line in text.strip().splitlines():
+        r = [x.strip() for x in line.split(",")]
+        if len(r) < 10:
+            continue
+        try:
+            ts = datetime.datetime.strptime(r[0], "%Y/%m/%d %H:%M:%S.%f")
+        except ValueError:
+            continue
+        rows.append((ts, r[1:]))
+    if not rows:
+        return None
+    window = "timed region"
+    if t0 is not None and t1 is not None:
+        inside = [x for x in rows if t0 <= x[0] <= t1]
+        if not inside:
+            mid = t0 + (t1 - t0) / 2
+            best = min(abs((x[0] - mid).total_seconds()) for x in rows)
+            inside = [x for x in rows if abs((x[0] - mid).total_seconds()) <= best + 0.01]
+            window = "nearest to the timed region"
+        rows = inside
+    num = lambda v: float(v) if v.replace(".", "", 1).isdigit() else None
+    sm = [v for v in (num(r[1]) for _, r in rows) if v is not None]
+    mx = [v for v in (num(r[2]) for _, r in rows) if v is not None]
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    reasons = sorted({n for _, r in rows for n, v in zip(names, r[5:9])
+                      if "Active" in v and "Not" not in v})
+    return {"sm_mhz": statistics.median(sm) if sm else None,
+            "sm_max_mhz": max(mx) if mx else None,
+            "reasons": reasons, "samples": len(rows), "window": window}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms; mark()
+    brackets the timed region so that only its samples are summarised."""
+
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index):
         self.index = index
         self.proc = None
+        self.t0 = self.t1 = None
 
     def start(self):
         try:
@@ -129,26 +171,25 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
+    def mark(self, end=False):
+        import datetime
+        now = datetime.datetime.now()
+        if end:
+            self.t1 = now
+        else:
+            self.t0 = now
+
     def stop(self):
         if self.proc is None:
             return None
+        time.sleep(0.15)  # one more sample after the region
         self.proc.terminate()
         try:
             out, _ = self.proc.communicate(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
             out, _ = self.proc.communicate()
-        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
-        if not rows:
-            return None
-        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if "Active" in v
-                          and "Not" not in v})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        return summarise_clocks(out, self.t0, self.t1)
 
 
 def dist_setup():
@@ -269,11 +310,13 @@ def _timed_steps(torch, step, n_marks, args, world, dev, stream, lib):
     dist_barrier(world)
     torch.cuda.synchronize(dev)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks.mark()
     t0.record(stream)
     for i in range(K):
         step(evs[i])
     t1.record(stream)
     torch.cuda.synchronize(dev)
+    clocks.mark(end=True)
     dist_barrier(world)
     clk = None if args.no_clocks else clocks.stop()
     st, word = lib.fa_device_status(sh)
@@ -316,11 +359,17 @@ def _e2e(torch, dev_inputs, dev_outputs, api_step, K, world, dev, stream, step_f
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / ke}
 
 
-def _roof(kernel, flops, ms, peak, peak_src, traffic=None):
+def _roof(kernel, flops, ms, peak, peak_src, traffic=None, sustained=None):
+    """Tensor roofline against the burst peak (the stricter denominator);
+    the fraction of the sustained (power-capped) peak is given beside it."""
     tf = flops / (ms / 1e3) / 1e12
-    return {"bound": "tensor", "kernel": kernel, "achieved": tf, "peak": peak, "unit": "TFLOP/s",
-            "frac": tf / peak, "traffic": traffic, "peak_source": f"{peak_src} bf16 dense (burst)",
-            "flops_per_launch": flops}
+    r = {"bound": "tensor", "kernel": kernel, "achieved": tf, "peak": peak, "unit": "TFLOP/s",
+         "frac": tf / peak, "traffic": traffic, "peak_source": f"{peak_src} bf16 dense (burst)",
+         "flops_per_launch": flops}
+    if sustained:
+        r["frac_of_sustained"] = tf / sustained
+        r["peak_sustained"] = sustained
+    return r
 
 
 def _cpu_oracle(samples):
@@ -416,10 +465,11 @@ def run_ours(args, w):
     peaks, peak_src = load_peaks()
     peak = float(peaks["bf16_tflops"])
     dom = max(("fa_fwd_kernel", "fa_bwd_kernel"), key=lambda n: avg[n])
+    sus = float(peaks.get("bf16_tflops_sustained", 0.0)) or None
     roofline = _roof(dom, f_fwd if dom == "fa_fwd_kernel" else f_bwd, avg[dom], peak, peak_src,
-                     recorded_traffic(dom, w.name))
+                     recorded_traffic(dom, w.name), sus)
     roofline_fwd = _roof("fa_fwd_kernel", f_fwd, avg["fa_fwd_kernel"], peak, peak_src,
-                         recorded_traffic("fa_fwd_kernel", w.name))
+                         recorded_traffic("fa_fwd_kernel", w.name), sus)
     bwd_ms = avg["fa_bwd_pre"] + avg["fa_bwd_kernel"] + avg["fa_bwd_post"]
     fwd_tf = roofline_fwd["achieved"]
     bwd_tf = f_bwd / (bwd_ms / 1e3) / 1e12
