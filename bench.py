@@ -250,8 +250,15 @@ def run_reference(args, w):
     if int(os.environ.get("RANK", "0")) != 0:
         return 0
     n_rows = min(4096, w.N)
-    for _ in range(args.warmup):
-        oracle_sample(w, n_rows)
+    t_w = 0.0
+    for _ in range(max(1, args.warmup)):
+        t_w = oracle_sample(w, n_rows)[0]
+    # keep the timed steps near 90 s in all: the sample's cost grows with the
+    # square of its rows, so shrink the rows of every step together
+    budget = 90.0
+    if args.steps * t_w > budget:
+        shrink = math.sqrt(budget / (args.steps * t_w))
+        n_rows = max(256, int(n_rows * shrink) // 128 * 128)
     tot_t, tot_f, thr = 0.0, 0.0, 1
     for s in range(args.steps):
         dt, fl, thr = oracle_sample(w, n_rows, seed=s)
