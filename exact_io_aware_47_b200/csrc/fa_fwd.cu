@@ -33,6 +33,69 @@
 
 namespace fa {
 
+// Packed batches of at most this many sequences are scheduled longest
+// first (more fall back to the head-major order of work_item).
+constexpr int kRankMaxSeqs = 512;
+
+// Longest-first order of a packed batch's work.  The super-units of a
+// sequence (for each head, query-tile pair m with its mirror, as in
+// work_item) all cost about the same, so listing the sequences by length,
+// longest first, lists the super-units by cost; dealing them to the CTAs in
+// snake order (CTA c takes positions r G + c for even r and r G + G-1-c for
+// odd r) balances the CTAs where head-major order leaves those with short
+// sequences idle.  The table is built in shared memory by the whole CTA
+// before the roles split, and every role walks it with its own cursor.
+struct PackedOrder {
+  const int* len;   // [B] sequence lengths (as slice_info clamps them)
+  const int* seq;   // [B] sequence of each rank
+  const int* pre;   // [B + 1] super-units before each rank
+};
+
+__device__ __forceinline__ int fwd_pairs(int L) { return ((L + kBlockM - 1) / kBlockM + 1) / 2; }
+
+__device__ void packed_order_build(const FwdParams& p, int* len, int* seq, int* pre) {
+  for (int b = threadIdx.x; b < p.B; b += blockDim.x)
+    len[b] = slice_info<true>(b * p.H, p, kErrDeviceSeqlen).L;
+  __syncthreads();
+  for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
+    const int lb = len[b];
+    int rank = 0;
+    for (int o = 0; o < p.B; ++o) rank += (len[o] > lb) || (len[o] == lb && o < b);
+    seq[rank] = b;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int i = 0; i < p.B; ++i) {
+      pre[i] = acc;
+      acc += p.H * ((fwd_pairs(len[seq[i]]) + 1) / 2);
+    }
+    pre[p.B] = acc;
+  }
+}
+
+// Work item k of this CTA in the longest-first order; false past the end.
+// cursor (this role's, starting at 0) only moves forward.
+__device__ __forceinline__ bool packed_work_item(int k, const FwdParams& p, const PackedOrder& o,
+                                                 int& cursor, WorkItem& wi) {
+  const int r = k >> 1;
+  const long long pos = static_cast<long long>(r) * gridDim.x +
+                        ((r & 1) ? static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x)
+                                 : static_cast<int>(blockIdx.x));
+  if (pos >= o.pre[p.B]) return false;
+  while (o.pre[cursor + 1] <= pos) ++cursor;
+  const int b = o.seq[cursor];
+  const int pairs = fwd_pairs(o.len[b]);
+  const int half = (pairs + 1) / 2;
+  const int off = static_cast<int>(pos - o.pre[cursor]);
+  const int h = off / half;
+  const int m = off - h * half;
+  wi.bh = b * p.H + h;
+  const int a = pairs - 1 - m;
+  wi.idx = (k & 1) == 0 ? a : (m != a ? m : -1);
+  return true;
+}
+
 template <int D, int ESZ>
 struct FwdLayout {
   static constexpr int kRowBytes = D * ESZ;            // ESZ = element bytes (2, or 1 for e4m3)
@@ -45,7 +108,11 @@ struct FwdLayout {
   static constexpr int kSlot0 = 2 * kTileBytes;
   static constexpr int kBar = kSlot0 + kSlots * kTileBytes;
   static constexpr int kBarBytes = 512;
-  static constexpr int kSmemBytes = kBar + kBarBytes + 1024;  // + slack to align to 1024
+  // packed batches: sequence lengths, sequences ranked by length and the
+  // running count of super-units over the ranking (see PackedOrder)
+  static constexpr int kRank = kBar + kBarBytes;
+  static constexpr int kRankBytes = (3 * kRankMaxSeqs + 1) * 4;
+  static constexpr int kSmemBytes = kRank + kRankBytes + 1024;  // + slack to align to 1024
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColO = 256;
 };
@@ -165,9 +232,22 @@ __global__ void __launch_bounds__(384, 1)
     tmem_alloc(tmem_slot, Lay::kTmemCols);
     tmem_relinquish();
   }
+  PackedOrder order{nullptr, nullptr, nullptr};
+  const bool ranked = PACKED && p.B <= kRankMaxSeqs;
+  if (ranked) {
+    int* tab = reinterpret_cast<int*>(smem + Lay::kRank);
+    order = PackedOrder{tab, tab + kRankMaxSeqs, tab + 2 * kRankMaxSeqs};
+    packed_order_build(p, tab, tab + kRankMaxSeqs, tab + 2 * kRankMaxSeqs);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // this CTA's k-th work item, in the same order for every role
+  int cursor = 0;
+  auto next_item = [&](int k, WorkItem& wi) -> bool {
+    if (ranked) return packed_work_item(k, p, order, cursor, wi);
+    return work_item(k, p.n_pairs, p.B * p.H, wi);
+  };
   const uint32_t tmem = *tmem_slot;
 
   if (warp >= 8) {
@@ -183,7 +263,7 @@ __global__ void __launch_bounds__(384, 1)
       bool ok = true;
       for (int k = 0; ok; ++k) {
         WorkItem wi;
-        if (!work_item(k, p.n_pairs, p.B * p.H, wi)) break;
+        if (!next_item(k, wi)) break;
         if (wi.idx < 0) continue;
         const FwdUnit w = fwd_decode<PACKED, SPARSE>(wi.bh, wi.idx, p);
         const int je[2] = {w.jend0, w.jend1};
@@ -269,7 +349,7 @@ __global__ void __launch_bounds__(384, 1)
 
       for (int k = 0; ok; ++k) {
         WorkItem wi;
-        if (!work_item(k, p.n_pairs, p.B * p.H, wi)) break;
+        if (!next_item(k, wi)) break;
         if (wi.idx < 0) continue;
         const FwdUnit w = fwd_decode<PACKED, SPARSE>(wi.bh, wi.idx, p);
         const int je[2] = {w.jend0, w.jend1};
@@ -362,7 +442,7 @@ __global__ void __launch_bounds__(384, 1)
     bool ok = true;
     for (int k = 0; ok; ++k) {
       WorkItem wi;
-      if (!work_item(k, p.n_pairs, p.B * p.H, wi)) break;
+      if (!next_item(k, wi)) break;
       if (wi.idx < 0) continue;
       const FwdUnit w = fwd_decode<PACKED, SPARSE>(wi.bh, wi.idx, p);
       const int jend = t == 0 ? w.jend0 : w.jend1;
