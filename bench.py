@@ -79,32 +79,41 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
-# Files that hold device code (the kernels and the device helpers they use);
-# the host API in fa_api.cu does not change what a kernel moves.
-KERNEL_SOURCES = ("fa_bwd.cu", "fa_fwd.cu", "fa_internal.h", "fa_quant.cu", "sm100.cuh")
+# Device sources of each kernel (its own file and the device helpers it
+# includes); the host API in fa_api.cu does not change what a kernel moves.
+KERNEL_SOURCES = {
+    "fa_fwd_kernel": ("fa_fwd.cu", "fa_internal.h", "sm100.cuh"),
+    "fa_fwd_kernel (e4m3)": ("fa_fwd.cu", "fa_internal.h", "sm100.cuh"),
+    "fa_bwd_kernel": ("fa_bwd.cu", "fa_internal.h", "sm100.cuh"),
+    "fa_quantize_e4m3": ("fa_quant.cu", "fa_internal.h", "sm100.cuh"),
+}
 
 
-def kernel_source_sha():
-    """Hash of the kernels' sources: recorded DRAM traffic is reported only
-    while it matches (profiles/traffic.json)."""
-    h = hashlib.sha256()
+def kernel_source_sha(kernel, read=None):
+    """Hash of one kernel's device sources: its recorded DRAM traffic is
+    reported only while it matches (profiles/traffic.json).  ``read(name)``
+    returns a file's bytes (default: the working tree)."""
     csrc = os.path.join(ROOT, "exact_io_aware_47_b200", "csrc")
-    for fn in KERNEL_SOURCES:
-        with open(os.path.join(csrc, fn), "rb") as f:
-            h.update(fn.encode() + f.read())
+    if read is None:
+        def read(fn):
+            with open(os.path.join(csrc, fn), "rb") as f:
+                return f.read()
+    h = hashlib.sha256()
+    for fn in KERNEL_SOURCES[kernel]:
+        h.update(fn.encode() + read(fn))
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel, workload):
     """DRAM bytes per launch from the committed ncu summary, or None if the
-    kernel sources changed since it was captured."""
+    kernel's sources changed since it was captured."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
-    if not os.path.exists(p):
+    if not os.path.exists(p) or kernel not in KERNEL_SOURCES:
         return None
     with open(p) as f:
         d = json.load(f)
     e = d.get(kernel, {})
-    if e.get("workload") != workload or e.get("source_sha") != kernel_source_sha():
+    if e.get("workload") != workload or e.get("source_sha") != kernel_source_sha(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
