@@ -302,7 +302,9 @@ def quantize_e4m3(x, out=None, descale=None):
         out = torch.empty((B, H, N, d), dtype=torch.float8_e4m3fn, device=dev)
     if descale is None:
         descale = torch.empty((B, H, nt), dtype=torch.float32, device=dev)
-    _check_inputs({"out": out}, (B, H, N, d), out.dtype if out.dtype in _E4M3 else None, dev)
+    if out.dtype not in _E4M3:
+        raise ValueError(f"out has dtype {out.dtype}, expected float8_e4m3fn or uint8")
+    _check_inputs({"out": out}, (B, H, N, d), out.dtype, dev)
     _check_inputs({"descale": descale}, (B, H, nt), torch.float32, dev)
     with torch.cuda.device(dev):
         st = _lib.fa_quantize_e4m3(x.data_ptr(), out.data_ptr(), descale.data_ptr(), B, H, N, d,
