@@ -254,6 +254,142 @@ def oracle_sample(w, n_rows, n_slices=1, seed=0):
     return dt, fl, threads
 
 
+def oracle_samples_packed(q, k, v, do, cu, B, H, d, scale, causal, max_rows=None):
+    """(fn, flops) per (head, sequence) slice of a packed batch (any device),
+    sequences in order, head after head; slices cut to max_rows if given."""
+    from oracle import ref_bwd_slice, ref_fwd_slice
+    cuh = [int(x) for x in cu.cpu()]
+    for h in range(H):
+        for b in range(B):
+            s0, s1 = cuh[b], cuh[b + 1]
+            if max_rows is not None:
+                s1 = min(s1, s0 + max_rows)
+            if s1 == s0:
+                continue
+            qq, kk, vv, dd = (t[h, s0:s1].double().cpu().numpy() for t in (q, k, v, do))
+            yield ((lambda qq=qq, kk=kk, vv=vv, dd=dd: (
+                ref_fwd_slice(qq, kk, vv, scale, causal),
+                ref_bwd_slice(qq, kk, vv, dd, scale, causal))),
+                   3.5 * flops_fwd(1, 1, s1 - s0, d, causal))
+
+
+def oracle_samples_variant(kind, spec, q, k, v, do, mask_list, B, H, d, scale, causal, n_rows):
+    """(fn, flops) per (batch, head) slice cut to its first n_rows queries and
+    keys: block-sparse (mask_list) or dropout (spec's p_drop and seed)."""
+    import numpy as np
+    from oracle import (ref_bwd_dropout_slice, ref_bwd_slice, ref_fwd_dropout_slice,
+                        ref_fwd_slice)
+    nt_cut = (n_rows + 127) // 128
+    for b in range(B):
+        for h in range(H):
+            qq, kk, vv, dd = (t[b, h, :n_rows].double().cpu().numpy() for t in (q, k, v, do))
+            if kind == "sparse":
+                mnp = np.array(mask_list, dtype=bool)[:nt_cut, :nt_cut]
+                yield ((lambda qq=qq, kk=kk, vv=vv, dd=dd, mnp=mnp: (
+                    ref_fwd_slice(qq, kk, vv, scale, causal, block_mask=mnp),
+                    ref_bwd_slice(qq, kk, vv, dd, scale, causal, block_mask=mnp))),
+                       3.5 * flops_fwd_blocksparse(mnp.tolist(), 1, 1, d, causal))
+            else:
+                bh, p_drop, seed = b * H + h, spec["p_drop"], spec["seed"]
+                yield ((lambda qq=qq, kk=kk, vv=vv, dd=dd, bh=bh: (
+                    ref_fwd_dropout_slice(qq, kk, vv, scale, causal, p_drop, seed, 0, bh),
+                    ref_bwd_dropout_slice(qq, kk, vv, dd, scale, causal, p_drop, seed, 0, bh))),
+                       3.5 * flops_fwd(1, 1, n_rows, d, causal))
+
+
+def oracle_samples_fp8(q, k, v, B, H, d, scale, causal, n_rows):
+    """(fn, flops) per (batch, head) slice cut to its first n_rows: the
+    oracle's quantisation of Q, K, V and its e4m3 forward."""
+    from oracle.fp8 import quantize_tiles, ref_fwd_fp8_slice
+    for b in range(B):
+        for h in range(H):
+            xs = [t[b, h, :n_rows].float().cpu().numpy() for t in (q, k, v)]
+
+            def one(xs=xs):
+                (qc, qs), (kc, ks), (vc, vs) = (quantize_tiles(x) for x in xs)
+                return ref_fwd_fp8_slice(qc, kc, vc, qs, ks, vs, scale, causal)
+            yield one, flops_fwd(1, 1, n_rows, d, causal)
+
+
+def run_reference_workload(args):
+    """``--impl reference`` for the packed, block-sparse, dropout and 8-bit
+    workloads: the oracle of that workload on its synthetic inputs (drawn on
+    the host), one slice cut to a bounded number of rows per step, the slices
+    taken in turn."""
+    if int(os.environ.get("RANK", "0")) != 0:   # host-only: rank 0 runs it
+        return 0
+    import itertools
+    import torch
+    from exact_io_aware_47_b200.inputs import (BLOCKSPARSE_WORKLOADS, E4M3_WORKLOADS,
+                                               PACKED_WORKLOADS, WORKLOADS, make_inputs,
+                                               make_inputs_packed, window_block_mask)
+    name = args.workload
+
+    def gen(n_rows):
+        if name in PACKED_WORKLOADS:
+            w = PACKED_WORKLOADS[name]
+            inp = make_inputs_packed(name, seed=0, device="cpu")
+            return (w.description,
+                    oracle_samples_packed(inp["q"], inp["k"], inp["v"], inp["do"],
+                                          inp["cu_seqlens"], w.B, inp["q"].shape[0], w.d, w.scale,
+                                          w.causal, max_rows=n_rows))
+        spec = BLOCKSPARSE_WORKLOADS.get(name) or E4M3_WORKLOADS[name]
+        w = WORKLOADS[spec["base"]]
+        inp = make_inputs(w.name, dtype=w.dtypes[0], seed=0, with_do=name not in E4M3_WORKLOADS,
+                          device="cpu")
+        if name in E4M3_WORKLOADS:
+            return (spec["description"],
+                    oracle_samples_fp8(inp["q"], inp["k"], inp["v"], w.B, w.H, w.d, w.scale,
+                                       w.causal, n_rows))
+        mask = None
+        if spec["kind"] == "sparse":
+            mask = window_block_mask((w.N + 127) // 128, spec["window"], spec["n_global"]).tolist()
+        return (spec["description"],
+                oracle_samples_variant(spec["kind"], spec, inp["q"], inp["k"], inp["v"], inp["do"],
+                                       mask, w.B, w.H, w.d, w.scale, w.causal, n_rows))
+
+    torch.manual_seed(0)
+    n_rows = 1024
+    desc, it = gen(n_rows)
+    it = itertools.cycle(list(itertools.islice(it, 64)))
+    t_w = 0.0
+    for _ in range(max(1, args.warmup)):
+        fn, _ = next(it)
+        t0 = time.perf_counter()
+        fn()
+        t_w = time.perf_counter() - t0
+    budget = 90.0  # timed steps in all, as for the dense workloads
+    if args.steps * t_w > budget:
+        n_rows = max(256, int(n_rows * math.sqrt(budget / (args.steps * t_w))) // 128 * 128)
+        desc, it = gen(n_rows)
+        it = itertools.cycle(list(itertools.islice(it, 64)))
+    tot_t, tot_f = 0.0, 0.0
+    for _ in range(args.steps):
+        fn, fl = next(it)
+        t0 = time.perf_counter()
+        fn()
+        tot_t += time.perf_counter() - t0
+        tot_f += fl
+    from threadpoolctl import threadpool_info
+    thr = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    value = tot_f / tot_t / 1e12
+    sample = (f"per step: the float64 oracle of '{name}' on one slice cut to at most {n_rows} "
+              f"rows, slices in turn")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": desc, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_reference(args, w):
     # host-only program: rank 0 runs it, other ranks exit without work
     if int(os.environ.get("RANK", "0")) != 0:
@@ -583,21 +719,7 @@ def run_ours_packed(args, w):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        from oracle import ref_bwd_slice, ref_fwd_slice
-        cuh = [int(x) for x in cu.cpu()]
-        host = {n: t.double().cpu() for n, t in (("q", q), ("k", k), ("v", v), ("do", do))}
-
-        def samples():  # whole (head, sequence) slices, all sequences of the first heads
-            for h in range(H):
-                for b in range(B):
-                    s0, s1 = cuh[b], cuh[b + 1]
-                    if s1 == s0:
-                        continue
-                    qq, kk, vv, dd = (host[n][h, s0:s1].numpy() for n in ("q", "k", "v", "do"))
-                    yield ((lambda qq=qq, kk=kk, vv=vv, dd=dd: (
-                        ref_fwd_slice(qq, kk, vv, scale, causal),
-                        ref_bwd_slice(qq, kk, vv, dd, scale, causal))),
-                           3.5 * flops_fwd(1, 1, s1 - s0, d, causal))
+        samples = lambda: oracle_samples_packed(q, k, v, do, cu, B, H, d, scale, causal)
         val, thr, n_done, dt = _cpu_oracle(samples())
         cpu = {"value": val, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
                "sample": f"float64 oracle forward+backward of {n_done} whole (head, sequence) "
@@ -733,30 +855,10 @@ def run_ours_variant(args, spec):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        import numpy as np
-        from oracle import (ref_bwd_dropout_slice, ref_bwd_slice, ref_fwd_dropout_slice,
-                            ref_fwd_slice)
         n_rows = min(2048, N)  # slices cut to their first n_rows queries and keys
-        nt_cut = (n_rows + 127) // 128
-
-        def samples():
-            for b in range(B):
-                for h in range(H):
-                    qq, kk, vv, dd = (t[b, h, :n_rows].double().cpu().numpy()
-                                      for t in (q, k, v, do))
-                    if kind == "sparse":
-                        mnp = np.array(mask_list, dtype=bool)[:nt_cut, :nt_cut]
-                        yield ((lambda qq=qq, kk=kk, vv=vv, dd=dd, mnp=mnp: (
-                            ref_fwd_slice(qq, kk, vv, scale, causal, block_mask=mnp),
-                            ref_bwd_slice(qq, kk, vv, dd, scale, causal, block_mask=mnp))),
-                               3.5 * flops_fwd_blocksparse(mnp.tolist(), 1, 1, d, causal))
-                    else:
-                        bh = b * H + h
-                        yield ((lambda qq=qq, kk=kk, vv=vv, dd=dd, bh=bh: (
-                            ref_fwd_dropout_slice(qq, kk, vv, scale, causal, p_drop, seed, 0, bh),
-                            ref_bwd_dropout_slice(qq, kk, vv, dd, scale, causal, p_drop, seed, 0,
-                                                  bh))),
-                               3.5 * flops_fwd(1, 1, n_rows, d, causal))
+        samples = lambda: oracle_samples_variant(kind, spec, q, k, v, do,
+                                                 mask_list if kind == "sparse" else None,
+                                                 B, H, d, scale, causal, n_rows)
         val, thr, n_done, dt = _cpu_oracle(samples())
         cpu = {"value": val, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
                "sample": f"float64 oracle forward+backward ({kind}) of {n_done} (batch, head) "
@@ -840,18 +942,8 @@ def run_ours_fp8(args, spec):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        from oracle.fp8 import quantize_tiles, ref_fwd_fp8_slice
         n_rows = min(2048, N)  # slices cut to their first n_rows queries and keys
-
-        def samples():
-            for b in range(B):
-                for h in range(H):
-                    xs = [t[b, h, :n_rows].float().cpu().numpy() for t in (q, k, v)]
-
-                    def one(xs=xs):
-                        (qc, qs), (kc, ks), (vc, vs) = (quantize_tiles(x) for x in xs)
-                        return ref_fwd_fp8_slice(qc, kc, vc, qs, ks, vs, scale, causal)
-                    yield one, flops_fwd(1, 1, n_rows, d, causal)
+        samples = lambda: oracle_samples_fp8(q, k, v, B, H, d, scale, causal, n_rows)
         val, thr, n_done, dt = _cpu_oracle(samples())
         cpu = {"value": val, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
                "sample": f"oracle quantisation + e4m3 forward of {n_done} (batch, head) slices "
@@ -876,15 +968,15 @@ def main():
                                                PACKED_WORKLOADS, WORKLOADS)
     if args.workload in E4M3_WORKLOADS:
         if args.impl == "reference":
-            raise SystemExit("--impl reference times the dense workloads")
+            return run_reference_workload(args)
         return run_ours_fp8(args, E4M3_WORKLOADS[args.workload])
     if args.workload in BLOCKSPARSE_WORKLOADS:
         if args.impl == "reference":
-            raise SystemExit("--impl reference times the dense workloads")
+            return run_reference_workload(args)
         return run_ours_variant(args, BLOCKSPARSE_WORKLOADS[args.workload])
     if args.workload in PACKED_WORKLOADS:
         if args.impl == "reference":
-            raise SystemExit("--impl reference times the fixed-length workloads")
+            return run_reference_workload(args)
         return run_ours_packed(args, PACKED_WORKLOADS[args.workload])
     w = WORKLOADS[args.workload]
     if args.impl == "reference":

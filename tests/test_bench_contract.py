@@ -1,8 +1,8 @@
 """The JSON line of bench.py carries every key the harness reads.
 
-The reference arm runs on the host only, so it is run here for real (small
-workload, one step); the CUDA arm's line is assembled by the same helper
-the GPU runs use, from stand-in numbers."""
+The reference arm runs on the host only, so it is run here for real (every
+kind of workload, one step each); the CUDA arm's line is assembled by the
+same helper the GPU runs use, from stand-in numbers."""
 
 import json
 import os
@@ -18,9 +18,13 @@ TOP = {"metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "h
        "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"}
 
 
-def test_reference_arm_line():
+import pytest  # noqa: E402
+
+
+@pytest.mark.parametrize("workload", ["small", "varlen", "sparse", "dropout", "fp8"])
+def test_reference_arm_line(workload):
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                          "--workload", "small", "--steps", "1", "--warmup", "1"],
+                          "--workload", workload, "--steps", "1", "--warmup", "1"],
                          capture_output=True, text=True, timeout=300, cwd=ROOT)
     assert out.returncode == 0, out.stderr[-2000:]
     lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
