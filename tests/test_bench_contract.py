@@ -51,3 +51,13 @@ def test_cuda_arm_line_keys():
     assert line["gpu_launches"] == 80 and line["ms_per_step"] == 75.0 / 20
     assert line["higher_is_better"] is True and line["scaling"] == "weak"
     json.dumps(line)  # serialisable
+
+
+@pytest.mark.parametrize("workload", ["mid", "varlen"])
+def test_reference_arm_other_ranks_exit_without_work(workload):
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", workload, "--gpus", "2", "--steps", "1", "--warmup", "1"],
+                         capture_output=True, text=True, timeout=120, cwd=ROOT, env=env)
+    assert out.returncode == 0, out.stderr[-2000:]
+    assert not [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
