@@ -43,9 +43,18 @@ def _check_inputs(tensors, shape, dtype, device):
             raise ValueError(f"{name} must be contiguous [B, H, N, d]")
 
 
+def _on_device(name, t, device):
+    """Refuse a side tensor that lives on another accelerator: its pointer
+    would be read by the kernel as if it were memory of ``device``.  Host
+    tensors and lists are copied to ``device`` by the callers."""
+    if torch.is_tensor(t) and t.device.type != "cpu" and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device} (or a host tensor)")
+
+
 def _seqlens_arg(seqlens, B, device):
     if seqlens is None:
         return None, None
+    _on_device("seqlens", seqlens, device)
     sl = seqlens
     if not (torch.is_tensor(sl) and sl.is_cuda and sl.dtype == torch.int32 and sl.is_contiguous()):
         sl = torch.as_tensor(seqlens, dtype=torch.int32).to(device).contiguous()
@@ -162,6 +171,7 @@ def backward_dropout(q, k, v, o, lse, do, p_drop, seed, offset=0, scale=None, ca
 
 def _block_mask_arg(block_mask, N, device):
     nt = (N + 127) // 128
+    _on_device("block_mask", block_mask, device)
     bm = block_mask
     if not (torch.is_tensor(bm) and bm.is_cuda and bm.dtype == torch.uint8 and bm.is_contiguous()):
         bm = torch.as_tensor(block_mask).to(device=device, dtype=torch.uint8).contiguous()
@@ -223,6 +233,7 @@ def backward_blocksparse(q, k, v, o, lse, do, block_mask, scale=None, causal=Fal
 
 
 def _cu_seqlens_arg(cu_seqlens, T, device):
+    _on_device("cu_seqlens", cu_seqlens, device)
     cu = cu_seqlens
     if not (torch.is_tensor(cu) and cu.is_cuda and cu.dtype == torch.int32 and cu.is_contiguous()):
         cu = torch.as_tensor(cu_seqlens, dtype=torch.int32).to(device).contiguous()

@@ -139,3 +139,19 @@ def test_e4m3_rejections_before_any_cuda_call(lib):
     assert quant(x8=P + 8) == _lib.FA_ERR_ALIGNMENT
     assert quant(ds=P + 1) == _lib.FA_ERR_ALIGNMENT
     assert lib.fa_status_string(_lib.FA_ERR_DEVICE_SCALE) != b"unknown status"
+
+
+def test_side_tensors_on_another_device_are_refused():
+    """seqlens, block_mask and cu_seqlens are passed to the kernels as raw
+    pointers, so one that lives on another device must be refused on the host
+    (a meta tensor stands in for "another device": no GPU needed)."""
+    import torch
+    from exact_io_aware_47_b200 import attention as A
+    dev = torch.device("cuda", 0)
+    other = torch.device("meta")
+    with pytest.raises(ValueError, match="seqlens"):
+        A._seqlens_arg(torch.ones(2, dtype=torch.int32, device=other), 2, dev)
+    with pytest.raises(ValueError, match="block_mask"):
+        A._block_mask_arg(torch.ones((1, 1), dtype=torch.uint8, device=other), 128, dev)
+    with pytest.raises(ValueError, match="cu_seqlens"):
+        A._cu_seqlens_arg(torch.zeros(3, dtype=torch.int32, device=other), 10, dev)
