@@ -630,7 +630,7 @@ extern "C" const char* fa_status_string(int status) {
     case FA_ERR_DEVICE_LAYOUT: return "kernel refused: shared-memory window misaligned";
     case FA_ERR_SCRATCH_LIMIT:
       return "problem needs more backward scratch than fa_bwd_noalloc's static array holds";
-    case FA_ERR_DEVICE_SCALE: return "e4m3 descale factor not finite and positive, or infinite input";
+    case FA_ERR_DEVICE_SCALE: return "e4m3 descale factor not finite and positive, or infinite or NaN input";
     default: return "unknown status";
   }
 }

@@ -5,7 +5,8 @@
 // largest magnitude in the tile, descale = amax / 448 and inv = 448 / amax,
 // both fp32 divisions rounded to nearest; every element becomes
 // e4m3(x * inv) (fp32 product, then round to nearest even, saturating).  A
-// tile of zeros gets descale 1 and zero codes.  The format and the 448 bound
+// tile of zeros gets descale 1 and zero codes; a tile holding an infinite or
+// NaN value is reported as FA_ERR_DEVICE_SCALE.  The format and the 448 bound
 // are those of e4m3 in the OCP 8-bit floating-point specification; the pages
 // ("How Flash Attention Works", section "FlashAttention 2 and 3") only name
 // lower-precision paths.
@@ -23,6 +24,14 @@ namespace fa {
 
 constexpr int kQuantThreads = 256;
 
+// max that propagates NaN (the library max drops it), so that a NaN input
+// makes the tile's amax NaN and is reported like an infinite one
+__device__ __forceinline__ float max_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+
 __device__ __forceinline__ float abs_max8(const uint4& v, bool bf16, float m) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -36,7 +45,7 @@ __device__ __forceinline__ float abs_max8(const uint4& v, bool bf16, float m) {
       lo = __low2float(h);
       hi = __high2float(h);
     }
-    m = fmaxf(m, fmaxf(fabsf(lo), fabsf(hi)));
+    m = max_nan(m, max_nan(fabsf(lo), fabsf(hi)));
   }
   return m;
 }
@@ -92,19 +101,19 @@ __global__ void __launch_bounds__(kQuantThreads)
       }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    for (int o = 16; o > 0; o >>= 1) m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, o));
     if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = m;
     __syncthreads();
     float amax = warp_max[0];
 #pragma unroll
-    for (int i = 1; i < kQuantThreads / 32; ++i) amax = fmaxf(amax, warp_max[i]);
+    for (int i = 1; i < kQuantThreads / 32; ++i) amax = max_nan(amax, warp_max[i]);
     __syncthreads();  // warp_max is rewritten by the next tile
     float inv = 0.f, ds = 1.f;
     if (amax > 0.f) {
       inv = __fdiv_rn(448.f, amax);
       ds = __fdiv_rn(amax, 448.f);
     }
-    if (!(amax < INFINITY)) record_error(kErrDeviceScale, 2);   // an infinite input
+    if (!(amax < INFINITY)) record_error(kErrDeviceScale, 2);   // an infinite or NaN input
     if (threadIdx.x == 0) descale[tile] = ds;
 #pragma unroll
     for (int k = 0; k < kVecPerThread; ++k) {

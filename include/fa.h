@@ -68,8 +68,8 @@ typedef enum {
   FA_ERR_WORKSPACE = 8,       /* backward workspace missing or too small        */
   FA_ERR_DEVICE_LAYOUT = 9,   /* device: shared-memory window misaligned, kernel refused (fa_device_status) */
   FA_ERR_SCRATCH_LIMIT = 10,  /* fa_bwd_noalloc: workspace would exceed its static array */
-  FA_ERR_DEVICE_SCALE = 11    /* device: e4m3 descale not finite and > 0, or infinite input to
-                                 fa_quantize_e4m3 (fa_device_status) */
+  FA_ERR_DEVICE_SCALE = 11    /* device: e4m3 descale not finite and > 0, or infinite or NaN
+                                 input to fa_quantize_e4m3 (fa_device_status) */
 } fa_status;
 
 typedef enum { FA_BF16 = 0, FA_FP16 = 1 } fa_dtype;
@@ -173,7 +173,8 @@ int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o,
  *     descale = amax / 448 and each code = e4m3(x * (448 / amax)), both
  *     divisions and the product in fp32 rounded to nearest, the conversion
  *     round-to-nearest-even and saturating; a tile of zeros gets descale 1.
- *     d in {64, 128}.  An infinite input is reported as FA_ERR_DEVICE_SCALE.
+ *     d in {64, 128}.  An infinite or NaN input is reported as
+ *     FA_ERR_DEVICE_SCALE (that tile's descale and codes are then unspecified).
  *   fa_fwd_e4m3: forward attention of Q, K, V given as e4m3 codes
  *     [B, H, N, 128] with descales [B, H, ceil(N/128)] (any positive finite
  *     values; the quantiser's output is one choice): the tensors stand for
@@ -280,7 +281,10 @@ int fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* 
  *   everything the call reads, so no clearing is needed between calls.
  *   The first call on a device looks up the array's device address (once per
  *   device, with that device current); make that first call before any
- *   stream capture.
+ *   stream capture.  The address belongs to the device's primary context:
+ *   after cudaDeviceReset() (or anything else that destroys that context)
+ *   the looked-up address is stale, so do not call fa_bwd_noalloc again on
+ *   that device in the same process.
  */
 int fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
                    const void* dout, const float* lse, void* dq, void* dk, void* dv,

@@ -34,6 +34,18 @@ def sample_rows(N, n_random=96, seed=0, block=128):
     return np.array(sorted(r for r in rows if 0 <= r < N))
 
 
+def subset_slices(B, H):
+    """The fixed (batch, head) subset the large workloads are checked on:
+    (0, 0), (0, H-1), (B-1, H/2), (B-1, H-1), without repeats.  Slices are
+    independent problems, so checking some of them exactly is exact for
+    those slices."""
+    out = []
+    for s in ((0, 0), (0, H - 1), (B - 1, H // 2), (B - 1, H - 1)):
+        if s not in out:
+            out.append(s)
+    return out
+
+
 def assert_fwd_close(o_gpu, lse_gpu, o_ref, lse_ref, what=""):
     do = np.abs(o_gpu - o_ref)
     dl = np.abs(lse_gpu - lse_ref)

@@ -4,7 +4,7 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import assert_grad_close, f64, sample_rows
+from helpers import assert_grad_close, f64, sample_rows, subset_slices
 from oracle import ref_bwd_slice
 
 pytestmark = pytest.mark.gpu
@@ -36,8 +36,10 @@ def _check_full(fa, inp, causal, scale, what):
     for b in range(B):
         L = N if sl is None else int(sl[b])
         for h in range(H):
-            refs[b, h] = ref_bwd_slice(f64(q[b, h]), f64(k[b, h]), f64(v[b, h]), f64(do[b, h]),
-                                       scale, causal, L)
+            # kept in float32 (the tolerances are 5e-2 relative): the ragged
+            # workload's 128 slices would take 1.6 GB of float64
+            refs[b, h] = [g.astype(np.float32) for g in ref_bwd_slice(
+                f64(q[b, h]), f64(k[b, h]), f64(v[b, h]), f64(do[b, h]), scale, causal, L)]
     typical = [max(np.abs(g[n]).max() for g in refs.values()) for n in range(3)]
     for b in range(B):
         L = N if sl is None else int(sl[b])
@@ -105,23 +107,22 @@ def test_mid_context_sampled(fa, dtype):
     from exact_io_aware_47_b200.inputs import WORKLOADS, make_inputs
     w = WORKLOADS["mid"]
     inp = make_inputs("mid", dtype=dtype, device="cuda")
-    slices = [(0, 0), (w.B - 1, w.H - 1)]
-    _check_sampled(fa, inp, True, w.scale, slices, f"mid {dtype}")
+    _check_sampled(fa, inp, True, w.scale, subset_slices(w.B, w.H), f"mid {dtype}")
 
 
 def test_long_context_sampled(fa):
     from exact_io_aware_47_b200.inputs import WORKLOADS, make_inputs
     w = WORKLOADS["long"]
     inp = make_inputs("long", device="cuda")
-    _check_sampled(fa, inp, True, w.scale, [(0, w.H - 1)], "long", n_random=24)
+    _check_sampled(fa, inp, True, w.scale, subset_slices(w.B, w.H), "long", n_random=24)
 
 
-def test_ragged_padded_batch(fa):
+def test_ragged_padded_batch_every_slice(fa):
+    """B8 H16 N4099 d128 with key padding: dQ, dK and dV of every (batch,
+    head) slice, every row, against the oracle; padded keys exactly zero."""
     from exact_io_aware_47_b200.inputs import WORKLOADS, make_inputs
     w = WORKLOADS["ragged"]
-    inp = make_inputs("ragged", device="cuda")
-    slices = [(b, (3 * b + 1) % w.H) for b in range(w.B)]
-    _check_sampled(fa, inp, False, w.scale, slices, "ragged", n_random=32)
+    _check_full(fa, make_inputs("ragged", device="cuda"), False, w.scale, "ragged")
 
 
 def test_workspace_contents_do_not_matter_and_guards_hold(fa):

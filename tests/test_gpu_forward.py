@@ -4,7 +4,7 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import assert_fwd_close, f64, sample_rows
+from helpers import assert_fwd_close, f64, sample_rows, subset_slices
 from oracle import ref_fwd_slice
 
 pytestmark = pytest.mark.gpu
@@ -97,8 +97,7 @@ def test_mid_context_sampled(fa, dtype):
     from exact_io_aware_47_b200.inputs import WORKLOADS, make_inputs
     w = WORKLOADS["mid"]
     inp = make_inputs("mid", dtype=dtype, device="cuda", with_do=False)
-    slices = [(0, 0), (0, w.H - 1), (w.B - 1, w.H // 2), (w.B - 1, w.H - 1)]
-    _check_sampled(fa, inp, True, w.scale, slices, f"mid {dtype}")
+    _check_sampled(fa, inp, True, w.scale, subset_slices(w.B, w.H), f"mid {dtype}")
 
 
 def test_long_context_sampled_and_linear_memory(fa):
@@ -117,15 +116,26 @@ def test_long_context_sampled_and_linear_memory(fa):
     # one N x N fp16 score matrix of one head would be 2 GiB; the call allocates nothing
     assert extra < 64 * 2 ** 20, f"forward allocated {extra} bytes"
     inp2 = {"q": q, "k": k, "v": v, "seqlens": None}
-    _check_sampled(fa, inp2, True, w.scale, [(0, 0), (0, w.H - 1)], "long", n_random=48)
+    _check_sampled(fa, inp2, True, w.scale, subset_slices(w.B, w.H), "long", n_random=48)
 
 
-def test_ragged_padded_batch(fa):
+def test_ragged_padded_batch_every_slice(fa):
+    """B8 H16 N4099 d128, key padding, K growing along the sequence (the
+    workload built to stress the rescale): every (batch, head) slice, every
+    row, against the oracle."""
     from exact_io_aware_47_b200.inputs import WORKLOADS, make_inputs
     w = WORKLOADS["ragged"]
     inp = make_inputs("ragged", device="cuda", with_do=False)
-    slices = [(b, (5 * b) % w.H) for b in range(w.B)]
-    _check_sampled(fa, inp, False, w.scale, slices, "ragged", n_random=48)
+    q, k, v, sl = inp["q"], inp["k"], inp["v"], inp["seqlens"]
+    o, lse = fa.forward(q, k, v, scale=w.scale, causal=False, seqlens=sl)
+    st, word = fa.device_status()
+    assert st == 0, f"device status {st} word {word:#x}"
+    lens = sl.cpu().tolist()
+    for b in range(w.B):
+        for h in range(w.H):
+            ro, rl = ref_fwd_slice(f64(q[b, h]), f64(k[b, h]), f64(v[b, h]), w.scale, False,
+                                   lens[b])
+            assert_fwd_close(f64(o[b, h]), f64(lse[b, h]), ro, rl, f"ragged b{b} h{h} L{lens[b]}")
 
 
 def test_output_guard_regions_untouched(fa):

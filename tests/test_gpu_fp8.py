@@ -1,24 +1,28 @@
 """8-bit (e4m3) path on the GPU (fa_quantize_e4m3, fa_fwd_e4m3 through the C
-ABI) against the oracle of oracle/fp8.py.
+ABI) against the oracle.
 
 * The quantiser decides its integer codes in fp32 on both sides, so codes and
   descales must be identical, bit for bit.
-* The forward runs on codes the oracle produced.  LSE uses the unrounded
-  probabilities: the dense tolerance (1e-3).  O: the dense tolerances
-  (max 2e-2, mean 2e-3) plus, per element, one e4m3 step of the largest term
-  of its row (2^-3 p_ij |v_jc|): the kernel's fp32 scores and approximate
-  exp2 may round a probability that lies on an e4m3 rounding boundary to the
-  neighbouring code, which the fp64 oracle cannot reproduce; such elements
-  must stay rare.
+* The forward runs on codes the oracle produced and is compared with plain
+  softmax attention (oracle.attention, the definition) of the dequantised
+  inputs code x descale.  The one step of the 8-bit path that the definition
+  does not have is the rounding of the probabilities to e4m3 before the
+  product with V ("How Flash Attention Works", section "FlashAttention 2 and
+  3": lower-precision paths); oracle.fp8.fp8_error_bound bounds what that
+  rounding can change, element by element, from the format's precision alone.
+  So every O element must lie within the dense tolerance (2e-2) plus that
+  bound, the mean error within 2e-3 plus the mean bound, and LSE, which the
+  rounding does not touch, within the dense 1e-3.  No fraction of elements is
+  exempt.
 """
 
 import numpy as np
 import pytest
 import torch
 
-from helpers import f64, sample_rows
-from oracle import allowed_mask
-from oracle.fp8 import dequantize_tiles, quantize_tiles, ref_fwd_fp8_slice
+from helpers import LSE_MAX_ABS, O_MAX_ABS, O_MEAN_ABS, f64, sample_rows
+from oracle import ref_fwd_slice
+from oracle.fp8 import dequantize_tiles, fp8_error_bound, quantize_tiles
 
 pytestmark = pytest.mark.gpu
 
@@ -44,28 +48,24 @@ def _oracle_quantize(x):
     return codes, ds
 
 
-def _one_step_allowance(q8, k8, v8, sq, sk, sv, scale, causal, valid, rows):
+def _check_against_definition(o, lse, q8, k8, v8, sq, sk, sv, scale, causal, valid, rows, what):
+    """o, lse: the GPU's rows ``rows`` of one slice; the rest: that slice's
+    codes and descales.  Plain attention of the dequantised inputs, and the
+    element-wise bound of the 8-bit rounding of P."""
     qd, kd, vd = (dequantize_tiles(c, s) for c, s in ((q8, sq), (k8, sk), (v8, sv)))
-    s = scale * (qd[rows] @ kd.T)
-    s = np.where(allowed_mask(rows, kd.shape[0], valid, causal), s, -np.inf)
-    p = np.exp(s - s.max(axis=1, keepdims=True))
-    p /= p.sum(axis=1, keepdims=True)
-    # max_j p_ij |v_jc| for every (i, c), 32 rows at a time
-    av = np.abs(vd)
-    out = np.empty((len(rows), vd.shape[1]))
-    for r0 in range(0, len(rows), 32):
-        out[r0:r0 + 32] = np.max(p[r0:r0 + 32, :, None] * av[None, :, :], axis=1)
-    return 2.0 ** -3 * out
-
-
-def _check_fwd(o, lse, ro, rl, allow, what):
+    ro, rl = ref_fwd_slice(qd, kd, vd, scale, causal, valid, rows=rows)
+    bound = fp8_error_bound(q8, k8, v8, sq, sk, sv, scale, causal, valid, rows=rows)
+    assert np.isfinite(o).all() and np.isfinite(lse).all(), f"{what}: non-finite output"
     err = np.abs(o - ro)
-    assert np.abs(lse - rl).max() <= 1e-3, f"{what}: LSE max err {np.abs(lse - rl).max():.3e}"
-    assert err.mean() <= 2e-3, f"{what}: O mean err {err.mean():.3e}"
-    over = err > 2e-2 + allow
-    assert not over.any(), f"{what}: O err {err[over].max():.3e} beyond the allowance"
-    rare = (err > 2e-2).mean()
-    assert rare <= 1e-3, f"{what}: {rare:.2e} of O beyond 2e-2"
+    dl = np.abs(lse - rl).max()
+    assert dl <= LSE_MAX_ABS, f"{what}: LSE max err {dl:.3e}"
+    over = err > O_MAX_ABS + bound
+    assert not over.any(), \
+        f"{what}: {int(over.sum())} O elements beyond 2e-2 + bound (worst excess " \
+        f"{(err - O_MAX_ABS - bound).max():.3e})"
+    assert err.mean() <= O_MEAN_ABS + bound.mean(), \
+        f"{what}: O mean err {err.mean():.3e} vs {O_MEAN_ABS + bound.mean():.3e}"
+    return err.max(), err.mean(), bound.mean()
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
@@ -116,9 +116,8 @@ def test_forward_against_oracle(fa, N, causal):
     for b in range(B):
         for h in range(H):
             a = (qc[b, h], kc[b, h], vc[b, h], sq[b, h], sk[b, h], sv[b, h])
-            ro, rl = ref_fwd_fp8_slice(*a, scale, causal)
-            allow = _one_step_allowance(*a, scale, causal, N, np.arange(N))
-            _check_fwd(o[b, h], lse[b, h], ro, rl, allow, f"N{N} causal{causal} b{b} h{h}")
+            _check_against_definition(o[b, h], lse[b, h], *a, scale, causal, N, np.arange(N),
+                                      f"N{N} causal{causal} b{b} h{h}")
 
 
 def test_forward_key_padding_fp16_out_and_v_tile_scales(fa):
@@ -130,9 +129,8 @@ def test_forward_key_padding_fp16_out_and_v_tile_scales(fa):
     for b in range(B):
         for h in range(H):
             a = (qc[b, h], kc[b, h], vc[b, h], sq[b, h], sk[b, h], sv[b, h])
-            ro, rl = ref_fwd_fp8_slice(*a, scale, False, lens[b])
-            allow = _one_step_allowance(*a, scale, False, lens[b], np.arange(N))
-            _check_fwd(o[b, h], lse[b, h], ro, rl, allow, f"padded b{b} h{h}")
+            _check_against_definition(o[b, h], lse[b, h], *a, scale, False, lens[b],
+                                      np.arange(N), f"padded b{b} h{h}")
 
 
 def test_full_size_causal_sampled(fa):
@@ -156,9 +154,8 @@ def test_full_size_causal_sampled(fa):
             oracle_in += [codes, rds]
         a = (oracle_in[0], oracle_in[2], oracle_in[4], oracle_in[1], oracle_in[3], oracle_in[5])
         rows = sample_rows(N, n_random=24, seed=b + h)
-        ro, rl = ref_fwd_fp8_slice(*a, scale, True, rows=rows)
-        allow = _one_step_allowance(*a, scale, True, N, rows)
-        _check_fwd(f64(o[b, h])[rows], f64(lse[b, h])[rows], ro, rl, allow, f"full b{b} h{h}")
+        _check_against_definition(f64(o[b, h])[rows], f64(lse[b, h])[rows], *a, scale, True, N,
+                                  rows, f"full b{b} h{h}")
 
 
 def test_rejections_and_device_scale_status(fa):
@@ -180,6 +177,10 @@ def test_rejections_and_device_scale_status(fa):
     assert st == _lib.FA_ERR_DEVICE_SCALE
     x = torch.ones((1, 1, 128, 64), dtype=torch.bfloat16, device="cuda")
     x[0, 0, 5, 7] = float("inf")
+    fa.quantize_e4m3(x)
+    st, _ = _lib.fa_device_status(s)
+    assert st == _lib.FA_ERR_DEVICE_SCALE
+    x[0, 0, 5, 7] = float("nan")                               # NaN is reported too
     fa.quantize_e4m3(x)
     st, _ = _lib.fa_device_status(s)
     assert st == _lib.FA_ERR_DEVICE_SCALE

@@ -9,7 +9,8 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import GRAD_REL_MAX, f64
+from helpers import GRAD_REL_MAX, assert_grad_close, f64
+from oracle import ref_bwd_slice
 
 pytestmark = pytest.mark.gpu
 
@@ -49,6 +50,14 @@ def test_noalloc_matches_fa_bwd_on_two_calls(d, causal):
             assert err <= GRAD_REL_MAX * np.abs(r).max(), f"call {call} {name}: {err:.3e}"
         # dK and dV involve no atomics: identical to the allocating entry point
         assert torch.equal(dk, ref[1]) and torch.equal(dv, ref[2])
+        # and all three against the float64 oracle, on a full-length slice and
+        # on one of the batch whose keys are padded to 613
+        for b, h in ((0, 0), (1, H - 1)):
+            L = int(sl[b])
+            g = ref_bwd_slice(f64(q[b, h]), f64(k[b, h]), f64(v[b, h]), f64(do[b, h]), scale,
+                              causal, L)
+            for n, (name, got) in enumerate(zip(("dQ", "dK", "dV"), (dq, dk, dv))):
+                assert_grad_close(f64(got[b, h]), g[n], f"call {call} {name} b{b} h{h} (oracle)")
 
 
 def test_noalloc_refuses_problems_beyond_its_array():
