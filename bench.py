@@ -159,24 +159,76 @@ def summarise_clocks(text, t0=None, t1=None):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 100 ms; mark()
-    brackets the timed region so that only its samples are summarised."""
+    """SM clock, power and throttle reasons sampled during the run; mark()
+    brackets the timed region so that only its samples are summarised.
+
+    Samples come from NVML in a background thread every ``period_s`` (a few
+    ms, so that even a timed region of tens of ms holds several samples),
+    written as the rows ``nvidia-smi --query-gpu=<Q> --format=csv,noheader,
+    nounits`` would print; without NVML, nvidia-smi itself is run with its
+    shortest loop period."""
 
     Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits, in the order of the last four Q columns
+    REASON_BITS = (0x8, 0x40, 0x20, 0x4)
 
-    def __init__(self, index):
+    def __init__(self, index, uuid=None, period_s=0.003):
         self.index = index
+        self.uuid = uuid
+        self.period_s = period_s
         self.proc = None
+        self.thread = None
+        self.rows = []
+        self.source = None
         self.t0 = self.t1 = None
 
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        if self.uuid:
+            try:
+                u = self.uuid if self.uuid.startswith("GPU-") else "GPU-" + self.uuid
+                return pynvml, pynvml.nvmlDeviceGetHandleByUUID(u.encode())
+            except Exception:  # noqa: BLE001 - fall back to the index
+                pass
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.index)
+
+    def _nvml_loop(self, nv, h, stop):
+        import datetime
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+            except Exception:  # noqa: BLE001 - a failed read ends sampling
+                break
+            flags = ["Active" if rs & b else "Not Active" for b in self.REASON_BITS]
+            ts = datetime.datetime.now().strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+            self.rows.append(", ".join([ts, str(self.index), str(sm), str(mx), f"{pw:.2f}",
+                                        f"0x{rs:016x}", *flags]))
+            stop.wait(self.period_s)
+
     def start(self):
+        import threading
+        try:
+            nv, h = self._nvml_handle()
+            self._stop = threading.Event()
+            self.thread = threading.Thread(target=self._nvml_loop, args=(nv, h, self._stop),
+                                           daemon=True)
+            self.thread.start()
+            self.source = f"NVML every {self.period_s * 1e3:.0f} ms"
+            return
+        except Exception:  # noqa: BLE001 - no NVML: use nvidia-smi
+            self.thread = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.source = "nvidia-smi every 100 ms"
         except OSError:
             self.proc = None
 
@@ -189,16 +241,25 @@ class ClockSampler:
             self.t0 = now
 
     def stop(self):
-        if self.proc is None:
+        if self.thread is not None:
+            time.sleep(2 * self.period_s)  # one more sample after the region
+            self._stop.set()
+            self.thread.join(timeout=5)
+            out = "\n".join(self.rows)
+        elif self.proc is not None:
+            time.sleep(0.15)  # one more sample after the region
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+        else:
             return None
-        time.sleep(0.15)  # one more sample after the region
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        return summarise_clocks(out, self.t0, self.t1)
+        s = summarise_clocks(out, self.t0, self.t1)
+        if s is not None:
+            s["source"] = self.source
+        return s
 
 
 def dist_setup():
@@ -455,7 +516,11 @@ def _timed_steps(torch, step, n_marks, args, world, dev, stream, lib):
         raise RuntimeError(f"device status {st} ({word:#x}) after warm-up")
     K = args.steps
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_marks)] for _ in range(K)]
-    clocks = ClockSampler(dev.index if dev.index is not None else 0)
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:  # noqa: BLE001 - older torch: match by index
+        uuid = None
+    clocks = ClockSampler(dev.index if dev.index is not None else 0, uuid)
     if not args.no_clocks:
         clocks.start()
         time.sleep(0.3)

@@ -42,3 +42,32 @@ def test_short_region_falls_back_to_the_nearest_samples():
 def test_unparseable_output_gives_none():
     assert bench.summarise_clocks("", None, None) is None
     assert bench.summarise_clocks("garbage\n1,2,3", None, None) is None
+
+
+def test_nvml_sampler_gives_several_samples_in_a_short_region(monkeypatch):
+    """The NVML sampler (here a fake module: no GPU needed) records every few
+    ms, so a timed region of tens of ms still holds several samples; the
+    reason bits map to the named throttle reasons."""
+    import time
+    import types
+    fake = types.SimpleNamespace(
+        NVML_CLOCK_SM=1,
+        nvmlInit=lambda: None,
+        nvmlDeviceGetHandleByIndex=lambda i: ("h", i),
+        nvmlDeviceGetHandleByUUID=lambda u: ("h", u),
+        nvmlDeviceGetMaxClockInfo=lambda h, c: 1965,
+        nvmlDeviceGetClockInfo=lambda h, c: 1800,
+        nvmlDeviceGetPowerUsage=lambda h: 812000,
+        nvmlDeviceGetCurrentClocksEventReasons=lambda h: 0x4,   # sw_power_cap
+    )
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    c = bench.ClockSampler(0, "GPU-fake", period_s=0.002)
+    c.start()
+    time.sleep(0.02)
+    c.mark()
+    time.sleep(0.06)
+    c.mark(end=True)
+    s = c.stop()
+    assert s["samples"] >= 5 and s["window"] == "timed region"
+    assert s["sm_mhz"] == 1800 and s["sm_max_mhz"] == 1965
+    assert s["reasons"] == ["sw_power_cap"] and s["source"].startswith("NVML")
