@@ -55,6 +55,7 @@ SIGNATURES = {
     "fa_quantize_e4m3": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP]),
     "fa_fwd_e4m3": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _VP, _I,
                          _VP]),
+    "fa_set_wait_limit_ns": (ctypes.c_ulonglong, [ctypes.c_ulonglong]),
     "fa_device_status": (_I, [_VP, ctypes.POINTER(ctypes.c_uint32)]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_version": (_I, []),
@@ -183,6 +184,12 @@ def fa_fwd_e4m3(q8, k8, v8, q_descale, k_descale, v_descale, o, lse, B, H, N, d,
 
 def fa_bwd_noalloc_max_bytes():
     return load().fa_bwd_noalloc_max_bytes()
+
+
+def fa_set_wait_limit_ns(ns):
+    """Bound of every pipeline wait of later launches (0: the 2 s default);
+    returns the previous bound."""
+    return load().fa_set_wait_limit_ns(ns)
 
 
 def fa_device_status(stream):

@@ -2,6 +2,7 @@
 //
 // Every check here runs on the host before anything is enqueued, so a bad
 // call returns a status and leaves the device untouched.
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -32,6 +33,10 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn g_encode = nullptr;
+
+// Bound of every pipeline wait of the kernels launched from now on
+// (fa_set_wait_limit_ns).
+std::atomic<unsigned long long> g_wait_ns{kWaitTimeoutNs};
 
 int current_device_info(DeviceInfo* out) {
   int dev = -1;
@@ -187,6 +192,7 @@ int fwd_core(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.n_qtiles = (p.max_seqlen + kBlockM - 1) / kBlockM;
   p.n_pairs = (p.n_qtiles + 1) / 2;
   p.n_units = B * H * ((p.n_pairs + 1) / 2);
+  p.wait_ns = g_wait_ns.load(std::memory_order_relaxed);
   const cudaError_t e =
       e4m3 ? launch_fwd_e4m3(dtype == FA_BF16, tq, tk, tv, p, di.num_sms,
                              static_cast<cudaStream_t>(stream))
@@ -343,6 +349,7 @@ int bwd_common(void* workspace, size_t workspace_bytes, int B, int H, int N, int
   p->scale_log2 = scale * 1.4426950408889634f;
   p->n_ktiles = (p->max_seqlen + kBlockN - 1) / kBlockN;
   p->n_units = B * H * ((p->n_ktiles + 1) / 2);
+  p->wait_ns = g_wait_ns.load(std::memory_order_relaxed);
   return FA_OK;
 }
 
@@ -598,6 +605,10 @@ extern "C" int fa_bwd_noalloc(const void* q, const void* k, const void* v, const
   // so whatever an earlier call left in the array does not matter.
   return fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, scratch, kStaticScratchBytes, B, H, N, d,
                 scale, causal, seqlens, dtype, stream);
+}
+
+extern "C" unsigned long long fa_set_wait_limit_ns(unsigned long long ns) {
+  return g_wait_ns.exchange(ns == 0 ? kWaitTimeoutNs : ns);
 }
 
 extern "C" int fa_device_status(void* stream, uint32_t* detail) {

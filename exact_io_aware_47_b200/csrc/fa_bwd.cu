@@ -168,6 +168,7 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* ds_full = bars + 21;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const WaitCtl wc{abort_flag, p.wait_ns};  // every pipeline wait of this CTA
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -215,6 +216,7 @@ __global__ void __launch_bounds__(512, 1)
       tma_prefetch_desc(&tmv);
       tma_prefetch_desc(&tmdo);
       int nunit = 0, lt = 0;  // lt: query tiles loaded (Q_lt -> slot lt & 1, dO_lt -> slot 2)
+      int issued[3] = {0, 0, 0};  // loads issued into each Q/dO slot (for the drain)
       bool ok = true;
       for (int k = 0; ok; ++k) {
         WorkItem wi;
@@ -222,7 +224,7 @@ __global__ void __launch_bounds__(512, 1)
         if (wi.idx < 0) continue;
         const BwdUnit w = bwd_decode<PACKED, SPARSE>(wi.bh, wi.idx, p);
         if (w.skip) continue;
-        ok = mbar_wait(kv_empty, (nunit & 1) ^ 1, abort_flag, 20);
+        ok = mbar_wait(kv_empty, (nunit & 1) ^ 1, wc, 20);
         if (!ok) break;
         mbar_arrive_expect_tx(kv_full, 2 * Lay::kTileBytes);
 #pragma unroll
@@ -239,7 +241,7 @@ __global__ void __launch_bounds__(512, 1)
           for (int t = 0; t < 2 && ok; ++t) {  // Q_i, then dO_i
             const int slot = t == 0 ? (lt & 1) : 2;
             const int use = t == 0 ? (lt >> 1) : lt;  // earlier loads into this slot
-            ok = mbar_wait(&slot_empty[slot], (use & 1) ^ 1, abort_flag, 21);
+            ok = mbar_wait(&slot_empty[slot], (use & 1) ^ 1, wc, 21);
             if (!ok) break;
             mbar_arrive_expect_tx(&slot_full[slot], Lay::kTileBytes);
 #pragma unroll
@@ -247,18 +249,17 @@ __global__ void __launch_bounds__(512, 1)
               tma_load_3d(sSlot + slot * Lay::kTileBytes + pn * Lay::kPanelBytes,
                           t == 0 ? &tmq : &tmdo, &slot_full[slot], pn * 64,
                           w.row0 + i * kBlockM, w.z);
+            ++issued[slot];
           }
           ++lt;
         }
       }
+      // Never leave with copies in flight: wait for the last load issued into
+      // every barrier (the n-th use of a slot completes its phase n & 1;
+      // already complete on the normal path).
       if (nunit > 0) mbar_wait_drain(kv_full, (nunit - 1) & 1, 200000000ull);
-      for (int s = 0; s < 2; ++s) {
-        if (lt > s) {
-          const int last = lt - 1 - ((lt - 1 - s) & 1);
-          mbar_wait_drain(&slot_full[s], (last >> 1) & 1, 200000000ull);
-        }
-      }
-      if (lt > 0) mbar_wait_drain(&slot_full[2], (lt - 1) & 1, 200000000ull);
+      for (int s = 0; s < 3; ++s)
+        if (issued[s] > 0) mbar_wait_drain(&slot_full[s], (issued[s] - 1) & 1, 200000000ull);
     }
     __syncwarp();
   } else if (warp == 14) {
@@ -277,7 +278,7 @@ __global__ void __launch_bounds__(512, 1)
       for (int idx = 0; idx < w.ni && ok; ++idx) {
         i = bwd_next_i<SPARSE>(p, w, i + 1);
         const int st = seq & 1;
-        ok = mbar_wait_warp(&ld_empty[st], ((seq >> 1) & 1) ^ 1, abort_flag, 22);
+        ok = mbar_wait_warp(&ld_empty[st], ((seq >> 1) & 1) ^ 1, wc, 22);
         if (!ok) break;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -322,7 +323,7 @@ __global__ void __launch_bounds__(512, 1)
         if (wi.idx < 0) continue;
         const BwdUnit w = bwd_decode<PACKED, SPARSE>(wi.bh, wi.idx, p);
         if (w.skip) continue;
-        ok = mbar_wait(kv_full, nunit & 1, abort_flag, 23);
+        ok = mbar_wait(kv_full, nunit & 1, wc, 23);
         if (!ok) break;
         tc_fence_after();
         // The epilogue of the previous unit must have read dV/dK before this
@@ -341,7 +342,7 @@ __global__ void __launch_bounds__(512, 1)
           umma_commit(s_full);
         };
         if (w.ni > 0) {
-          ok = mbar_wait(&slot_full[it & 1], (it >> 1) & 1, abort_flag, 24);
+          ok = mbar_wait(&slot_full[it & 1], (it >> 1) & 1, wc, 24);
           if (!ok) break;
           tc_fence_after();
           issue_s(it);
@@ -350,10 +351,10 @@ __global__ void __launch_bounds__(512, 1)
           FA_TRACE_AT(it, 0);
           // d = 128: dQ^T of the previous tile lives in the dP^T columns
           if (D == 128 && it > 0) {
-            ok = mbar_wait(dq_empty, (it - 1) & 1, abort_flag, 25);
+            ok = mbar_wait(dq_empty, (it - 1) & 1, wc, 25);
             if (!ok) break;
           }
-          ok = mbar_wait(&slot_full[2], it & 1, abort_flag, 35);
+          ok = mbar_wait(&slot_full[2], it & 1, wc, 35);
           if (!ok) break;
           tc_fence_after();
           FA_TRACE_AT(it, 1);
@@ -361,12 +362,12 @@ __global__ void __launch_bounds__(512, 1)
           umma_ss_group<D / 16, false, false>(tmem + Lay::kColDP, lV_k, lO_k, kIdS, 0u);
           umma_commit(dp_full);
           // dV_j += P^T dO_i once the first softmax phase wrote P^T
-          ok = mbar_wait(p_full, it & 1, abort_flag, 26);
+          ok = mbar_wait(p_full, it & 1, wc, 26);
           if (!ok) break;
           tc_fence_after();
           FA_TRACE_AT(it, 2);
           if (!dkv_free) {
-            ok = mbar_wait(dkv_empty, (nunit - 1) & 1, abort_flag, 27);
+            ok = mbar_wait(dkv_empty, (nunit - 1) & 1, wc, 27);
             if (!ok) break;
             tc_fence_after();
             dkv_free = true;
@@ -380,14 +381,14 @@ __global__ void __launch_bounds__(512, 1)
           // S^T of the next tile: its MMA runs after dV (in order), which has
           // read P^T out of these columns
           if (idx + 1 < w.ni) {
-            ok = mbar_wait(&slot_full[(it + 1) & 1], ((it + 1) >> 1) & 1, abort_flag, 24);
+            ok = mbar_wait(&slot_full[(it + 1) & 1], ((it + 1) >> 1) & 1, wc, 24);
             if (!ok) break;
             tc_fence_after();
             issue_s(it + 1);
           }
           FA_TRACE_AT(it, 14);
           // dQ and dK_j += dS^T Q_i once the second phase wrote dS^T
-          ok = mbar_wait(ds_full, it & 1, abort_flag, 36);
+          ok = mbar_wait(ds_full, it & 1, wc, 36);
           if (!ok) break;
           tc_fence_after();
           FA_TRACE_AT(it, 8);
@@ -410,7 +411,7 @@ __global__ void __launch_bounds__(512, 1)
           } else {
             issue_dk();
             if (it > 0) {
-              ok = mbar_wait(dq_empty, (it - 1) & 1, abort_flag, 25);
+              ok = mbar_wait(dq_empty, (it - 1) & 1, wc, 25);
               if (!ok) break;
               tc_fence_after();
             }
@@ -422,7 +423,7 @@ __global__ void __launch_bounds__(512, 1)
         }
         if (!ok) break;
         if (!dkv_free) {
-          ok = mbar_wait(dkv_empty, (nunit - 1) & 1, abort_flag, 34);
+          ok = mbar_wait(dkv_empty, (nunit - 1) & 1, wc, 34);
           if (!ok) break;
         }
         umma_commit(dkv_full);
@@ -513,8 +514,8 @@ __global__ void __launch_bounds__(512, 1)
           }
         }
         // ---- phase 1: P^T = 2^(c S^T - LSE_i log2 e) from S^T, back to TMEM
-        ok = mbar_wait_warp(&ld_full[st], (it >> 1) & 1, abort_flag, 28) &&
-             mbar_wait_warp(s_full, it & 1, abort_flag, 29);
+        ok = mbar_wait_warp(&ld_full[st], (it >> 1) & 1, wc, 28) &&
+             mbar_wait_warp(s_full, it & 1, wc, 29);
         if (!ok) break;
         tc_fence_after();
         if (threadIdx.x == 0) FA_TRACE_AT(it, 4);
@@ -561,8 +562,8 @@ __global__ void __launch_bounds__(512, 1)
         mbar_arrive(p_full);
         if (threadIdx.x == 0) FA_TRACE_AT(it, 15);
         // ---- phase 2: dS^T = P^T * (dP^T - D_i) from dP^T, to shared memory
-        ok = mbar_wait_warp(dp_full, it & 1, abort_flag, 30);
-        if (ok && it > 0) ok = mbar_wait_warp(ds_empty, (it - 1) & 1, abort_flag, 31);
+        ok = mbar_wait_warp(dp_full, it & 1, wc, 30);
+        if (ok && it > 0) ok = mbar_wait_warp(ds_empty, (it - 1) & 1, wc, 31);
         if (!ok) break;
         tc_fence_after();
         if (threadIdx.x == 0) FA_TRACE_AT(it, 11);
@@ -633,7 +634,8 @@ __global__ void __launch_bounds__(512, 1)
       int i = w.i0 - 1;  // walks the unit's query tiles
       for (int idx = 0; idx < w.ni && ok; ++idx) {
         i = bwd_next_i<SPARSE>(p, w, i + 1);
-        ok = mbar_wait_warp(dq_full, it & 1, abort_flag, 32);
+        // the four warps share named barrier 1 below: they go on or stop together
+        ok = named_bar_and(1, 128, mbar_wait_warp(dq_full, it & 1, wc, 32));
         if (!ok) break;
         tc_fence_after();
         if (threadIdx.x == 256) FA_TRACE_AT(it, 6);
@@ -680,7 +682,7 @@ __global__ void __launch_bounds__(512, 1)
         ++it;
       }
       if (!ok) break;
-      ok = mbar_wait_warp(dkv_full, nunit & 1, abort_flag, 33);
+      ok = named_bar_and(1, 128, mbar_wait_warp(dkv_full, nunit & 1, wc, 33));
       if (!ok) break;
       tc_fence_after();
       const int key = w.j * kBlockN + r;

@@ -208,6 +208,7 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* drain = o_full + 2;         // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const WaitCtl wc{abort_flag, p.wait_ns};  // every pipeline wait of this CTA
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -270,7 +271,7 @@ __global__ void __launch_bounds__(384, 1)
         const int jl[2] = {w.jlast0, w.jlast1};
         for (int t = 0; t < 2 && ok; ++t) {
           if (jl[t] < 0) continue;
-          ok = mbar_wait(&q_empty[t], (qload[t] & 1) ^ 1, abort_flag, 1);
+          ok = mbar_wait(&q_empty[t], (qload[t] & 1) ^ 1, wc, 1);
           if (!ok) break;
           mbar_arrive_expect_tx(&q_full[t], Lay::kTileBytes);
 #pragma unroll
@@ -284,7 +285,7 @@ __global__ void __launch_bounds__(384, 1)
           for (int kv = 0; kv < 2; ++kv) {
             const int slot = kv_seq % kSlots;
             const int round = kv_seq / kSlots;
-            ok = mbar_wait(&kv_empty[slot], (round & 1) ^ 1, abort_flag, 2);
+            ok = mbar_wait(&kv_empty[slot], (round & 1) ^ 1, wc, 2);
             if (!ok) break;
             mbar_arrive_expect_tx(&kv_full[slot], Lay::kTileBytes);
             uint8_t* dst = skv + slot * Lay::kTileBytes;
@@ -360,7 +361,7 @@ __global__ void __launch_bounds__(384, 1)
         if ((PACKED || SPARSE) && j0 >= jmax) continue;
         for (int t = 0; t < 2 && ok; ++t) {
           if (jl[t] < 0) continue;
-          ok = mbar_wait(&q_full[t], qload[t] & 1, abort_flag, 3);
+          ok = mbar_wait(&q_full[t], qload[t] & 1, wc, 3);
           ++qload[t];
         }
         if (!ok) break;
@@ -368,7 +369,7 @@ __global__ void __launch_bounds__(384, 1)
         // first K tile
         {
           const int slot = kv_seq % kSlots;
-          ok = mbar_wait(&kv_full[slot], (kv_seq / kSlots) & 1, abort_flag, 4);
+          ok = mbar_wait(&kv_full[slot], (kv_seq / kSlots) & 1, wc, 4);
           if (!ok) break;
           tc_fence_after();
           for (int t = 0; t < 2; ++t) {
@@ -383,7 +384,7 @@ __global__ void __launch_bounds__(384, 1)
         int npv[2] = {0, 0};  // P.V issued per query tile in this unit
         for (int j = j0; j < jmax && ok;) {
           const int vslot = kv_seq % kSlots;
-          ok = mbar_wait(&kv_full[vslot], (kv_seq / kSlots) & 1, abort_flag, 5);
+          ok = mbar_wait(&kv_full[vslot], (kv_seq / kSlots) & 1, wc, 5);
           if (!ok) break;
           tc_fence_after();
           ++kv_seq;
@@ -392,7 +393,7 @@ __global__ void __launch_bounds__(384, 1)
           bool k_ready = false;
           for (int t = 0; t < 2 && ok; ++t) {
             if (fwd_need<SPARSE>(p, w, t, j)) {
-              ok = mbar_wait(&p_full[t], pcnt[t] & 1, abort_flag, 6);
+              ok = mbar_wait(&p_full[t], pcnt[t] & 1, wc, 6);
               if (!ok) break;
               FA_TRACE_AT(pcnt[t], t);
               ++pcnt[t];
@@ -403,7 +404,7 @@ __global__ void __launch_bounds__(384, 1)
             }
             if (jn < jmax && fwd_need<SPARSE>(p, w, t, jn)) {
               if (!k_ready) {
-                ok = mbar_wait(&kv_full[kslot], (kv_seq / kSlots) & 1, abort_flag, 7);
+                ok = mbar_wait(&kv_full[kslot], (kv_seq / kSlots) & 1, wc, 7);
                 if (!ok) break;
                 tc_fence_after();
                 k_ready = true;
@@ -506,7 +507,7 @@ __global__ void __launch_bounds__(384, 1)
           cj = c * sq_t * skj;
           rho = svj / sv_max;
         }
-        ok = mbar_wait_warp(&s_full[t], scnt & 1, abort_flag, 8);
+        ok = mbar_wait_warp(&s_full[t], scnt & 1, wc, 8);
         if (!ok) break;
         if (r == 0) FA_TRACE_AT(scnt, 2 + 2 * t);
         ++scnt;
@@ -598,7 +599,7 @@ __global__ void __launch_bounds__(384, 1)
       }
       if (!ok) break;
       // epilogue: O / l -> 16-bit, LSE
-      ok = mbar_wait_warp(&o_full[t], ocnt & 1, abort_flag, 9);
+      ok = mbar_wait_warp(&o_full[t], ocnt & 1, wc, 9);
       if (!ok) break;
       ++ocnt;
       tc_fence_after();

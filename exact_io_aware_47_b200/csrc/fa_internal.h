@@ -46,6 +46,7 @@ struct FwdParams {
   int n_qtiles;             // ceil(N / 128)
   int n_pairs;              // ceil(n_qtiles / 2): a work unit is two query tiles
   int n_units;              // B * H * ceil(n_pairs / 2) super-units (see work_item)
+  unsigned long long wait_ns;  // bound of one pipeline wait (kErrDeviceTimeout past it)
 };
 
 struct BwdParams {
@@ -72,6 +73,7 @@ struct BwdParams {
   int causal;
   int n_ktiles;             // ceil(N / 128)
   int n_units;              // B * H * ceil(n_ktiles / 2) super-units (see work_item)
+  unsigned long long wait_ns;  // bound of one pipeline wait (kErrDeviceTimeout past it)
 };
 
 // Work order of the persistent kernels.  A head's units (query-tile pairs in

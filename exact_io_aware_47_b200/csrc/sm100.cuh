@@ -48,8 +48,9 @@ __device__ unsigned long long g_trace[kTraceSlots];
   } while (0)
 #endif
 
-// A wait gives up after this long and reports kErrDeviceTimeout.  No wait in
-// a correct pipeline lasts more than microseconds.
+// Default bound of a pipeline wait: it gives up after this long and reports
+// kErrDeviceTimeout.  No wait in a correct pipeline lasts more than
+// microseconds.  The host may set another bound per launch (WaitCtl).
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
@@ -96,20 +97,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// What a pipeline wait needs besides its barrier: the CTA-wide abort flag
+// (in shared memory) and the bound of one wait in nanoseconds.
+struct WaitCtl {
+  volatile int* abort;
+  unsigned long long limit_ns;
+};
+
 // Wait until the phase with the given parity has completed.  Returns false if
-// the CTA-wide abort flag is raised or the wait runs past kWaitTimeoutNs (in
+// the CTA-wide abort flag is raised or the wait runs past wc.limit_ns (in
 // which case it records the error and raises the flag itself).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtl& wc,
                                           unsigned site) {
   const uint32_t a = smem_addr(bar);
   if (mbar_try_wait(a, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(a, parity)) return true;
-    if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+    if (*wc.abort) return false;
+    if (globaltimer_ns() - t0 > wc.limit_ns) {
       record_error(kErrDeviceTimeout, site);
-      *abort_flag = 1;
+      *wc.abort = 1;
       return false;
     }
   }
@@ -118,10 +126,27 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 // Warp-uniform wait: every lane polls, and the warp proceeds only if all
 // lanes saw the phase complete, so .sync.aligned tcgen05 ops that follow are
 // reached by the whole warp or by none of it.
-__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
-                                               volatile int* abort_flag, unsigned site) {
-  const bool ok = mbar_wait(bar, parity, abort_flag, site);
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, const WaitCtl& wc,
+                                               unsigned site) {
+  const bool ok = mbar_wait(bar, parity, wc, site);
   return __all_sync(0xffffffffu, ok);
+}
+
+// Agreement of `threads` threads (whole warps) that meet at named barrier
+// `id`: true only if every one of them passes true.  Warps that share a
+// named barrier later on decide together whether to go on, so that none of
+// them waits there for a warp that has left.
+__device__ __forceinline__ bool named_bar_and(int id, int threads, bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(ok ? 1u : 0u), "r"(id), "r"(threads)
+      : "memory");
+  return r != 0;
 }
 
 // Same, with an explicit (short) limit and no error report: used only while

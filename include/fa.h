@@ -36,7 +36,8 @@
  *   Scale.  finite and > 0 (typically 1/sqrt(d)).
  *   Memory.  All pointers are device pointers owned by the caller, 16-byte
  *     aligned.  The library allocates no device memory and keeps no state
- *     other than cached driver entry points and per-device properties.
+ *     other than cached driver entry points, per-device properties and the
+ *     wait bound of fa_set_wait_limit_ns().
  *   Streams.  stream is a cudaStream_t (NULL = legacy default stream).  Work
  *     is enqueued asynchronously; no entry point synchronises except
  *     fa_device_status().
@@ -302,6 +303,23 @@ size_t fa_bwd_noalloc_max_bytes(void);
  * receives the raw word (code | site << 8 | block << 16).
  */
 int fa_device_status(void* stream, uint32_t* detail);
+
+/*
+ * Bound, in nanoseconds, of every pipeline wait inside the kernels launched
+ * after this call, from any host thread (default 2e9 = 2 s; 0 restores the
+ * default).  Returns the previous bound.
+ *   Every wait of a kernel's producer/consumer pipeline (a warp waiting for
+ *   a tile load, a tensor-core result or another warp's data) gives up after
+ *   this long: it records FA_ERR_DEVICE_TIMEOUT, with the site of the wait,
+ *   in the device status word, the CTA's other roles stop at their next
+ *   wait, copies and tensor-core work already in flight are waited for, and
+ *   the kernel returns, so the device stays usable; that call's outputs are
+ *   unspecified.  In a correct pipeline no wait lasts more than microseconds,
+ *   so the default only fires on a hang.  A bound far below a kernel's
+ *   ordinary waits (say 1 ns) makes ordinary waits give up: that is how the
+ *   timeout path is exercised without a fault.
+ */
+unsigned long long fa_set_wait_limit_ns(unsigned long long ns);
 
 /* Static description of a status code.  Never NULL. */
 const char* fa_status_string(int status);

@@ -155,3 +155,14 @@ def test_side_tensors_on_another_device_are_refused():
         A._block_mask_arg(torch.ones((1, 1), dtype=torch.uint8, device=other), 128, dev)
     with pytest.raises(ValueError, match="cu_seqlens"):
         A._cu_seqlens_arg(torch.zeros(3, dtype=torch.int32, device=other), 10, dev)
+
+
+def test_wait_limit_setting_is_host_state(lib):
+    """fa_set_wait_limit_ns returns the previous bound; 0 restores the 2 s
+    default (no GPU needed: the bound is passed to later launches)."""
+    lib.fa_set_wait_limit_ns.restype = ctypes.c_ulonglong
+    lib.fa_set_wait_limit_ns.argtypes = [ctypes.c_ulonglong]
+    first = lib.fa_set_wait_limit_ns(12345)
+    assert first == 2_000_000_000
+    assert lib.fa_set_wait_limit_ns(0) == 12345
+    assert lib.fa_set_wait_limit_ns(0) == 2_000_000_000
