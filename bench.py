@@ -49,6 +49,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "attention fwd/bwd TFLOP/s on 1 B200 and fraction of bf16 tensor-core peak"
+L2_BYTES = 126 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -64,6 +65,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="mid")
+    ap.add_argument("--dtype", choices=("bf16", "fp16"), default=None,
+                    help="16-bit type of a dense workload (default: its first)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -302,17 +305,66 @@ def oracle_sample(w, n_rows, n_slices=1, seed=0):
     from threadpoolctl import threadpool_info
     from exact_io_aware_47_b200.inputs import make_inputs_shape
     from oracle import ref_bwd_slice, ref_fwd_slice
-    dt = 0.0
+    dt, fl = 0.0, 0.0
     for s_ in range(n_slices):
-        inp = make_inputs_shape(1, 1, n_rows, w.d, w.dtypes[0], seed=seed + s_, ragged=False)
+        # the key-padded workload's recipe (drawn valid length, growing K)
+        # applies to the cut slice too
+        inp = make_inputs_shape(1, 1, n_rows, w.d, w.dtypes[0], seed=seed + s_, ragged=w.ragged)
         q, k, v, do = (inp[n][0, 0].double().numpy() for n in ("q", "k", "v", "do"))
+        L = n_rows if inp["seqlens"] is None else int(inp["seqlens"][0])
         t0 = time.perf_counter()
-        ref_fwd_slice(q, k, v, w.scale, w.causal)
-        ref_bwd_slice(q, k, v, do, w.scale, w.causal)
+        ref_fwd_slice(q, k, v, w.scale, w.causal, L)
+        ref_bwd_slice(q, k, v, do, w.scale, w.causal, L)
         dt += time.perf_counter() - t0
-    fl = n_slices * 3.5 * flops_fwd(1, 1, n_rows, w.d, w.causal)
+        fl += 3.5 * (flops_fwd(1, 1, n_rows, w.d, w.causal) if inp["seqlens"] is None else
+                     flops_fwd_keys([L], 1, n_rows, w.d, w.causal))
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     return dt, fl, threads
+
+
+def flops_fwd_keys(lengths, H, N, d, causal):
+    """Forward FLOPs with key padding: every one of the N query rows of batch
+    b meets its L_b valid keys (non-causal), 4 d FLOPs per score."""
+    if causal:
+        raise ValueError("key-padded FLOPs are defined for the non-causal workload")
+    return sum(4.0 * H * N * L * d for L in lengths)
+
+
+def cpu_baseline_slices(w, q, k, v, do, lengths, budget_s=20.0, threads=None):
+    """The float64 oracle (forward + backward) on whole (batch, head) slices of
+    the workload's own inputs (copied from the device), slices in order,
+    until all are done or about budget_s of CPU work.  threads=1 pins the
+    BLAS pool to one core.  Returns the cpu_baseline dict."""
+    from threadpoolctl import threadpool_info, threadpool_limits
+    from oracle import ref_bwd_slice, ref_fwd_slice
+    B, H, N = w.B, w.H, w.N
+    dt, fl, n_done = 0.0, 0.0, 0
+    limit = threadpool_limits(threads) if threads else None
+    try:
+        for b in range(B):
+            L = N if lengths is None else int(lengths[b])
+            for h in range(H):
+                qq, kk, vv, dd = (t[b, h].double().cpu().numpy() for t in (q, k, v, do))
+                tc = time.perf_counter()
+                ref_fwd_slice(qq, kk, vv, w.scale, w.causal, L)
+                ref_bwd_slice(qq, kk, vv, dd, w.scale, w.causal, L)
+                dt += time.perf_counter() - tc
+                f = flops_fwd(1, 1, N, w.d, w.causal) if lengths is None else \
+                    flops_fwd_keys([L], 1, N, w.d, w.causal)
+                fl += 3.5 * f
+                n_done += 1
+                if dt >= budget_s:
+                    break
+            if dt >= budget_s:
+                break
+        thr = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    finally:
+        if limit is not None:
+            limit.unregister()
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+            "sample": f"float64 oracle forward+backward of {n_done} of the {B * H} whole (batch, "
+                      f"head) slices of '{w.name}', the workload's own inputs, in order "
+                      f"({dt:.1f} s)"}
 
 
 def oracle_samples_packed(q, k, v, do, cu, B, H, d, scale, causal, max_rows=None):
@@ -634,6 +686,10 @@ def run_ours(args, w):
 
     B, H, N, d = w.B, w.H, w.N, w.d
     dtype = w.dtypes[0]
+    if args.dtype is not None:
+        dtype = torch.bfloat16 if args.dtype == "bf16" else torch.float16
+        if dtype not in w.dtypes:
+            raise SystemExit(f"workload {w.name} is defined for {w.dtypes}, not {args.dtype}")
     causal, scale = w.causal, w.scale
     inp = make_inputs(w.name, dtype=dtype, seed=rank, device=dev)
     q, k, v, do = inp["q"], inp["k"], inp["v"], inp["do"]
@@ -648,7 +704,16 @@ def run_ours(args, w):
     dt_code = _lib.FA_BF16 if dtype == torch.bfloat16 else _lib.FA_FP16
     slp = sl.data_ptr() if sl is not None else None
 
+    # Inputs and outputs of a step that fit in L2 with room to spare would be
+    # served from it on the next step: those workloads write a 256 MiB buffer
+    # before every step (outside the step's own events).
+    step_bytes = 8 * q.numel() * q.element_size()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if step_bytes < 2 * L2_BYTES \
+        else None
+
     def step(ev=None):
+        if flush is not None:
+            flush.fill_(1)
         if ev is not None:
             ev[0].record(stream)
         _lib.check("fa_fwd", _lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
@@ -673,8 +738,16 @@ def run_ours(args, w):
 
     warmup, total_ms, seg, clk = _timed_steps(torch, step, 5, args, world, dev, stream, _lib)
     K = args.steps
+    if flush is not None:
+        # the time of the K steps is their own events' spans (the flushes
+        # between them excluded), max over ranks
+        total_ms = dist_max(K * sum(seg), world)
     avg = dict(zip(("fa_fwd_kernel", "fa_bwd_pre", "fa_bwd_kernel", "fa_bwd_post"), seg))
-    f_fwd = flops_fwd(B, H, N, d, causal)
+    lengths = sl.cpu().tolist() if sl is not None else None
+    f_nominal = flops_fwd(B, H, N, d, causal)
+    # key padding: the work done is that of the valid keys (the primary
+    # figure); the N^2 count is reported beside it
+    f_fwd = f_nominal if lengths is None else flops_fwd_keys(lengths, H, N, d, causal)
     f_bwd = 2.5 * f_fwd
     step_flops = f_fwd + f_bwd
     ms_per_step = total_ms / K
@@ -702,16 +775,22 @@ def run_ours(args, w):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n_slices = 3
-        dt, fl, thr = oracle_sample(w, w.N, n_slices=n_slices)
-        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
-               "sample": f"float64 oracle forward+backward of {n_slices} whole (batch, head) "
-                         f"slices of '{w.name}' ({dt:.1f} s)"}
+        cpu = cpu_baseline_slices(w, q, k, v, do, lengths)
+        if w.name == "tiny":  # the smallest workload is also timed on one core
+            cpu["one_core"] = cpu_baseline_slices(w, q, k, v, do, lengths, threads=1)
 
+    mib = q.numel() * q.element_size() / 2 ** 20
     config = {"workload": w.description, "B": B, "H": H, "N": N, "d": d, "causal": causal,
+              "dtype": "bf16" if dtype == torch.bfloat16 else "fp16",
               "step": "fa_fwd + fa_bwd_preprocess + fa_bwd_main + fa_bwd_postprocess",
               "flops_per_step": step_flops, "parallelism": f"replicas x{world}",
-              "l2": "inputs larger than L2 (4 x 128 MiB per step), no flush"}
+              "l2": (f"inputs {mib:.1f} MiB per tensor: a 256 MiB buffer is written before "
+                     "every step, outside the step's events") if flush is not None else
+                    f"inputs larger than L2 ({mib:.0f} MiB per tensor), no flush"}
+    if lengths is not None:
+        config["flops"] = "valid keys only (4 d per score of a valid key)"
+        config["flops_per_step_nominal"] = 3.5 * f_nominal
+        config["seqlens"] = lengths
     line = _base_line(value, K, warmup, total_ms, world,
                       "bf16" if dtype == torch.bfloat16 else "f16", config,
                       {"ms": avg["fa_fwd_kernel"], "tflops": fwd_tf, "frac": fwd_tf / peak},

@@ -565,7 +565,7 @@ __global__ void __launch_bounds__(384, 1)
             const uint32_t h = pack_e4m3x2(p0 * rho, p1 * rho);
             pk[i >> 1] = (i & 1) ? (pk[i >> 1] | (h << 16)) : h;
           } else {
-            pk[i] = pack2<BF16>(p0, p1);
+            pk[i] = pack_op2<BF16>(p0, p1);
           }
         }
         {
