@@ -818,7 +818,7 @@ def run_ours_packed(args, w):
     B, causal, scale = w.B, w.causal, w.scale
     o, lse = torch.empty_like(q), torch.empty((H, T), dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws_bytes = fa.workspace_bytes(1, H, T, d)
+    ws_bytes = _lib.fa_bwd_varlen_workspace_size(B, H, T, d)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     sh = stream.cuda_stream

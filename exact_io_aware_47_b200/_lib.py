@@ -50,6 +50,7 @@ SIGNATURES = {
     "fa_bwd_blocksparse": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP,
                                 _I, _I, _I, _I, _F, _I, _VP, _I, _VP]),
     "fa_fwd_varlen": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _F, _I, _I, _VP]),
+    "fa_bwd_varlen_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "fa_bwd_varlen": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP,
                            _I, _I, _I, _I, _I, _F, _I, _I, _VP]),
     "fa_quantize_e4m3": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _VP]),
@@ -164,6 +165,10 @@ def fa_fwd_varlen(q, k, v, o, lse, cu_seqlens, B, H, T, max_seqlen, d, scale, ca
                   stream):
     return load().fa_fwd_varlen(q, k, v, o, lse, cu_seqlens, B, H, T, max_seqlen, d, scale, causal,
                                 dtype, stream)
+
+
+def fa_bwd_varlen_workspace_size(B, H, T, d):
+    return load().fa_bwd_varlen_workspace_size(B, H, T, d)
 
 
 def fa_bwd_varlen(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, cu_seqlens, B, H,

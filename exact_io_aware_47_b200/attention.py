@@ -280,7 +280,8 @@ def backward_varlen(q, k, v, o, lse, do, cu_seqlens, max_seqlen, scale=None, cau
     dv = torch.empty_like(v) if dv is None else dv
     _check_inputs({"dq": dq, "dk": dk, "dv": dv}, (H, T, d), q.dtype, dev)
     if workspace is None:
-        workspace = torch.empty(workspace_bytes(1, H, T, d), dtype=torch.uint8, device=dev)
+        workspace = torch.empty(_lib.fa_bwd_varlen_workspace_size(B, H, T, d), dtype=torch.uint8,
+                                device=dev)
     with torch.cuda.device(dev):
         st = _lib.fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                                 do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),

@@ -312,6 +312,16 @@ extern "C" size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   return round256(rows * sizeof(float)) + round256(rows * d * sizeof(float));
 }
 
+extern "C" size_t fa_bwd_varlen_workspace_size(int B, int H, int T, int d) {
+  if (B < 1) return 0;
+  const size_t base = fa_bwd_workspace_size(1, H, T, d);
+  if (base == 0) return 0;
+  // the longest-first order table: 3 B + 1 ints (batches of up to
+  // kBwdRankMaxSeqs sequences; larger ones run in head-major order)
+  const size_t table = B <= kBwdRankMaxSeqs ? round256((3ull * B + 1) * sizeof(int)) : 0;
+  return base + table;
+}
+
 namespace fa {
 namespace {
 
@@ -327,7 +337,8 @@ int bwd_common(void* workspace, size_t workspace_bytes, int B, int H, int N, int
   if ((seqlens && (reinterpret_cast<uintptr_t>(seqlens) & 3u)) ||
       (cu_seqlens && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)))
     return FA_ERR_ALIGNMENT;
-  const size_t need = cu_seqlens ? fa_bwd_workspace_size(1, H, N, d) : fa_bwd_workspace_size(B, H, N, d);
+  const size_t need = cu_seqlens ? fa_bwd_varlen_workspace_size(B, H, N, d)
+                                 : fa_bwd_workspace_size(B, H, N, d);
   if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) & 255u) return FA_ERR_ALIGNMENT;
   st = current_device_info(di);
@@ -339,6 +350,12 @@ int bwd_common(void* workspace, size_t workspace_bytes, int B, int H, int N, int
   p->dsum = static_cast<float*>(workspace);
   p->dq_acc =
       reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round256(rows * sizeof(float)));
+  // packed batches: the longest-first table after the accumulator
+  p->rank = (cu_seqlens && B <= kBwdRankMaxSeqs)
+                ? reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) +
+                                         round256(rows * sizeof(float)) +
+                                         round256(rows * d * sizeof(float)))
+                : nullptr;
   p->seqlens = seqlens;
   p->cu_seqlens = cu_seqlens;
   p->max_seqlen = cu_seqlens ? max_seqlen : N;
@@ -470,6 +487,7 @@ int bwd_variant_run(BwdParams& p, const DeviceInfo& di, const void* q, const voi
   const bool bf16 = dtype == FA_BF16;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (launch_bwd_pre(d, bf16, p, di.num_sms, s) != cudaSuccess) return FA_ERR_CUDA;
+  if (p.rank != nullptr && launch_bwd_rank(p, s) != cudaSuccess) return FA_ERR_CUDA;
   if (launch_bwd_main(d, bf16, tq, tk, tv, tdo, tdq, p, di.num_sms, s) != cudaSuccess)
     return FA_ERR_CUDA;
   return launch_bwd_post(d, bf16, p, di.num_sms, s) == cudaSuccess ? FA_OK : FA_ERR_CUDA;

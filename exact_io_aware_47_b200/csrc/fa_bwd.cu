@@ -128,6 +128,42 @@ __device__ __forceinline__ int bwd_next_i(const BwdParams& p, const BwdUnit& w, 
   return i;
 }
 
+// Longest-first order of a packed batch's backward work (the table is built
+// once per call by fa_bwd_rank into the workspace).  A sequence of L rows has
+// n = ceil(L / 128) key tiles; for each head its key tiles are paired with
+// their mirror (tile m with tile n-1-m, equal cost under a causal mask, and
+// every key tile costs the same without one), so listing the sequences by
+// length, longest first, lists the super-units by cost.  Dealing them to the
+// CTAs in snake order (CTA c takes positions r G + c for even r and
+// r G + G-1-c for odd r) keeps CTAs busy where the head-major order over
+// max_seqlen would leave those with short sequences idle.  cursor (this
+// role's, starting at 0) only moves forward.
+__device__ __forceinline__ bool packed_bwd_item(int k, const BwdParams& p, int& cursor,
+                                                WorkItem& wi) {
+  const int* len = p.rank;
+  const int* seq = p.rank + p.B;
+  const int* pre = p.rank + 2 * p.B;
+  const int r = k >> 1;
+  const long long pos = static_cast<long long>(r) * gridDim.x +
+                        ((r & 1) ? static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x)
+                                 : static_cast<int>(blockIdx.x));
+  if (pos >= pre[p.B]) return false;
+  while (pre[cursor + 1] <= pos) ++cursor;
+  const int b = seq[cursor];
+  const int n = (len[b] + kBlockN - 1) / kBlockN;
+  const int half = (n + 1) / 2;
+  const int off = static_cast<int>(pos - pre[cursor]);
+  const int h = off / half;
+  const int m = off - h * half;
+  wi.bh = b * p.H + h;
+  const int a = n - 1 - m;
+  // first half: key tile m (the longer one under a causal mask); second: its
+  // mirror.  bwd_decode takes the unit index n_ktiles - 1 - j of key tile j.
+  const int j = (k & 1) == 0 ? m : (m != a ? a : -1);
+  wi.idx = j < 0 ? -1 : p.n_ktiles - 1 - j;
+  return true;
+}
+
 template <int D, bool BF16, bool PACKED, bool SPARSE, bool DROPOUT>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
@@ -205,6 +241,12 @@ __global__ void __launch_bounds__(512, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // this CTA's k-th work item, in the same order for every role
+  int cursor = 0;
+  auto next_item = [&](int k, WorkItem& wi) -> bool {
+    if (PACKED && p.rank != nullptr) return packed_bwd_item(k, p, cursor, wi);
+    return work_item(k, p.n_ktiles, p.B * p.H, wi);
+  };
 
   if (warp >= 12) {
   regs_decrease<kBwdOtherRegs>();
@@ -220,7 +262,7 @@ __global__ void __launch_bounds__(512, 1)
       bool ok = true;
       for (int k = 0; ok; ++k) {
         WorkItem wi;
-        if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
+        if (!next_item(k, wi)) break;
         if (wi.idx < 0) continue;
         const BwdUnit w = bwd_decode<PACKED, SPARSE>(wi.bh, wi.idx, p);
         if (w.skip) continue;
@@ -269,7 +311,7 @@ __global__ void __launch_bounds__(512, 1)
     const float log2e = 1.4426950408889634f;
     for (int k = 0; ok; ++k) {
       WorkItem wi;
-      if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
+      if (!next_item(k, wi)) break;
       if (wi.idx < 0) continue;
       const BwdUnit w = bwd_decode<PACKED, SPARSE>(wi.bh, wi.idx, p);
       if (w.skip) continue;
@@ -319,7 +361,7 @@ __global__ void __launch_bounds__(512, 1)
       bool ok = true;
       for (int k = 0; ok; ++k) {
         WorkItem wi;
-        if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
+        if (!next_item(k, wi)) break;
         if (wi.idx < 0) continue;
         const BwdUnit w = bwd_decode<PACKED, SPARSE>(wi.bh, wi.idx, p);
         if (w.skip) continue;
@@ -354,6 +396,7 @@ __global__ void __launch_bounds__(512, 1)
             ok = mbar_wait(dq_empty, (it - 1) & 1, wc, 25);
             if (!ok) break;
           }
+          FA_TRACE_AT(it, 30);
           ok = mbar_wait(&slot_full[2], it & 1, wc, 35);
           if (!ok) break;
           tc_fence_after();
@@ -450,7 +493,7 @@ __global__ void __launch_bounds__(512, 1)
     bool ok = true;
     for (int k = 0; ok; ++k) {
       WorkItem wi;
-      if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
+      if (!next_item(k, wi)) break;
       if (wi.idx < 0) continue;
       const BwdUnit w = bwd_decode<PACKED, SPARSE>(wi.bh, wi.idx, p);
       if (w.skip) continue;
@@ -491,7 +534,7 @@ __global__ void __launch_bounds__(512, 1)
     bool ok = true;
     for (int k = 0; ok; ++k) {
       WorkItem wi;
-      if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
+      if (!next_item(k, wi)) break;
       if (wi.idx < 0) continue;
       const BwdUnit w = bwd_decode<PACKED, SPARSE>(wi.bh, wi.idx, p);
       if (w.skip) continue;
@@ -518,7 +561,7 @@ __global__ void __launch_bounds__(512, 1)
              mbar_wait_warp(s_full, it & 1, wc, 29);
         if (!ok) break;
         tc_fence_after();
-        if (threadIdx.x == 0) FA_TRACE_AT(it, 4);
+        if (threadIdx.x == FA_TRACE_SM_THREAD) FA_TRACE_AT(it, 4);
         // a query tile on the causal diagonal hides keys above the query
         const int diag_lim = (p.causal && i == w.j) ? r : -1;  // visible iff q_local >= r
         const float* lse2 = sLSE + st * 128;
@@ -528,9 +571,9 @@ __global__ void __launch_bounds__(512, 1)
         for (int cc = 0; cc < 2; ++cc) {
           const int c = half * 2 + cc;  // 32-query chunk
           uint32_t sr[32];
-          if (threadIdx.x == 0 && cc == 1) FA_TRACE_AT(it, 27);
+          if (threadIdx.x == FA_TRACE_SM_THREAD && cc == 1) FA_TRACE_AT(it, 27);
           tmem_ld32(tS + c * 32, sr);
-          if (threadIdx.x == 0) FA_TRACE_AT(it, cc == 0 ? 10 : 24);
+          if (threadIdx.x == FA_TRACE_SM_THREAD) FA_TRACE_AT(it, cc == 0 ? 10 : 24);
           uint32_t pp[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 4) {
@@ -555,25 +598,25 @@ __global__ void __launch_bounds__(512, 1)
           // half's
           tmem_st16(tS + half * 64 + (c & 1) * 16, pp);
         }
-        if (threadIdx.x == 0) FA_TRACE_AT(it, 25);
+        if (threadIdx.x == FA_TRACE_SM_THREAD) FA_TRACE_AT(it, 25);
         tmem_st_wait();
-        if (threadIdx.x == 0) FA_TRACE_AT(it, 26);
+        if (threadIdx.x == FA_TRACE_SM_THREAD) FA_TRACE_AT(it, 26);
         tc_fence_before();
         mbar_arrive(p_full);
-        if (threadIdx.x == 0) FA_TRACE_AT(it, 15);
+        if (threadIdx.x == FA_TRACE_SM_THREAD) FA_TRACE_AT(it, 15);
         // ---- phase 2: dS^T = P^T * (dP^T - D_i) from dP^T, to shared memory
         ok = mbar_wait_warp(dp_full, it & 1, wc, 30);
         if (ok && it > 0) ok = mbar_wait_warp(ds_empty, (it - 1) & 1, wc, 31);
         if (!ok) break;
         tc_fence_after();
-        if (threadIdx.x == 0) FA_TRACE_AT(it, 11);
+        if (threadIdx.x == FA_TRACE_SM_THREAD) FA_TRACE_AT(it, 11);
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           const int c = half * 2 + cc;
           uint32_t dr[32];
-          if (threadIdx.x == 0 && cc == 1) FA_TRACE_AT(it, 28);
+          if (threadIdx.x == FA_TRACE_SM_THREAD && cc == 1) FA_TRACE_AT(it, 28);
           tmem_ld32(tDP + c * 32, dr);
-          if (threadIdx.x == 0) FA_TRACE_AT(it, cc == 0 ? 12 : 21);
+          if (threadIdx.x == FA_TRACE_SM_THREAD) FA_TRACE_AT(it, cc == 0 ? 12 : 21);
           uint32_t dd[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 4) {
@@ -607,13 +650,13 @@ __global__ void __launch_bounds__(512, 1)
                          dd[4 * w4 + 3]);
           }
         }
-        if (threadIdx.x == 0) FA_TRACE_AT(it, 22);
+        if (threadIdx.x == FA_TRACE_SM_THREAD) FA_TRACE_AT(it, 22);
         fence_proxy_async_smem();
-        if (threadIdx.x == 0) FA_TRACE_AT(it, 23);
+        if (threadIdx.x == FA_TRACE_SM_THREAD) FA_TRACE_AT(it, 23);
         tc_fence_before();
         mbar_arrive(ds_full);
         mbar_arrive(&ld_empty[st]);
-        if (threadIdx.x == 0) FA_TRACE_AT(it, 5);
+        if (threadIdx.x == FA_TRACE_SM_THREAD) FA_TRACE_AT(it, 5);
         ++it;
       }
     }
@@ -626,7 +669,7 @@ __global__ void __launch_bounds__(512, 1)
     bool ok = true;
     for (int k = 0; ok; ++k) {
       WorkItem wi;
-      if (!work_item(k, p.n_ktiles, p.B * p.H, wi)) break;
+      if (!next_item(k, wi)) break;
       if (wi.idx < 0) continue;
       const BwdUnit w = bwd_decode<PACKED, SPARSE>(wi.bh, wi.idx, p);
       if (w.skip) continue;
@@ -653,6 +696,7 @@ __global__ void __launch_bounds__(512, 1)
           uint32_t v[D];
           if constexpr (D == 128) tmem_ld64x2(tmem + lane_off + Lay::kColDQ, v);
           else tmem_ld64(tmem + lane_off + Lay::kColDQ, v);
+          if (threadIdx.x == 256) FA_TRACE_AT(it, 29);
           tc_fence_before();
           mbar_arrive(dq_empty);
 #pragma unroll
@@ -796,6 +840,38 @@ __global__ void __launch_bounds__(256) fa_bwd_post(const float4* __restrict__ ac
     r.w = pack2<BF16>(b.z * scale, b.w * scale);
     dq[g] = r;
   }
+}
+
+// The longest-first table of a packed batch (see packed_bwd_item): lengths
+// as slice_info clamps them, sequences ranked by length (ties by index), and
+// the running count of super-units over the ranking.  One block.
+__global__ void __launch_bounds__(1024) fa_bwd_rank(const BwdParams p) {
+  int* len = p.rank;
+  int* seq = p.rank + p.B;
+  int* pre = p.rank + 2 * p.B;
+  for (int b = threadIdx.x; b < p.B; b += blockDim.x)
+    len[b] = slice_info<true>(b * p.H, p, kErrDeviceSeqlen).L;
+  __syncthreads();
+  for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
+    const int lb = len[b];
+    int rank = 0;
+    for (int o = 0; o < p.B; ++o) rank += (len[o] > lb) || (len[o] == lb && o < b);
+    seq[rank] = b;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int i = 0; i < p.B; ++i) {
+      pre[i] = acc;
+      acc += p.H * (((len[seq[i]] + kBlockN - 1) / kBlockN + 1) / 2);
+    }
+    pre[p.B] = acc;
+  }
+}
+
+cudaError_t launch_bwd_rank(const BwdParams& p, cudaStream_t stream) {
+  fa_bwd_rank<<<1, 1024, 0, stream>>>(p);
+  return cudaGetLastError();
 }
 
 static int elementwise_grid(long long n8, int num_sms) {

@@ -120,6 +120,14 @@ struct FwdLayout {
 // Register split: 384 threads launched at 168 registers (launch bounds 384,1);
 // the two softmax warpgroups take 184, the MMA/TMA warpgroup keeps 136:
 // 2 * 184 + 136 = 3 * 168 (no spills at this split).
+#ifndef FA_FWD_POLY_EVERY
+#define FA_FWD_POLY_EVERY 0
+#endif
+constexpr int kFwdPolyEvery = FA_FWD_POLY_EVERY;
+#ifndef FA_FWD_ST_CHUNKS
+#define FA_FWD_ST_CHUNKS 1
+#endif
+constexpr int kFwdStoreChunks = FA_FWD_ST_CHUNKS;
 constexpr int kFwdLaunchRegs = 168;
 constexpr int kFwdSoftmaxRegs = 184;
 constexpr int kFwdOtherRegs = 136;
@@ -553,7 +561,11 @@ __global__ void __launch_bounds__(384, 1)
               ffma2(f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), c2, nm2);
           float x0, x1;
           f2unpack(x2, x0, x1);
-          const unsigned long long p2 = f2pack(ex2_approx(x0), ex2_approx(x1));
+          // every FA_FWD_POLY_EVERY-th pair on the FMA pipe, the rest on the
+          // special-function unit, which is what bounds this loop
+          const bool poly = kFwdPolyEvery > 0 && !FP8 && (i % (kFwdPolyEvery > 0 ? kFwdPolyEvery : 1)) == kFwdPolyEvery - 1;
+          const unsigned long long p2 =
+              poly ? exp2_poly2(x0, x1) : f2pack(ex2_approx(x0), ex2_approx(x1));
           acc[i & 3] = fadd2(acc[i & 3], p2);
           float p0, p1;
           f2unpack(p2, p0, p1);
@@ -566,6 +578,12 @@ __global__ void __launch_bounds__(384, 1)
             pk[i >> 1] = (i & 1) ? (pk[i >> 1] | (h << 16)) : h;
           } else {
             pk[i] = pack_op2<BF16>(p0, p1);
+            // P goes back to TMEM in chunks as it is made, so the stores
+            // overlap the rest of the loop
+            if constexpr (kFwdStoreChunks > 1) {
+              constexpr int kC = 64 / kFwdStoreChunks;
+              if ((i % kC) == kC - 1) tmem_st_n<kC>(tS + (i + 1 - kC), pk + (i + 1 - kC));
+            }
           }
         }
         {
@@ -577,7 +595,7 @@ __global__ void __launch_bounds__(384, 1)
           l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
         }
         if constexpr (FP8) tmem_st32(tS, pk);
-        else tmem_st64(tS, pk);
+        else if (kFwdStoreChunks == 1) tmem_st64(tS, pk);
         if (jj > 0 && __any_sync(0xffffffffu, moved)) {
           // O_t holds the sum up to the previous key tile (its MMA completed
           // before S_t(j) was committed) and PV_t(j) waits for p_full:

@@ -65,6 +65,10 @@ struct BwdParams {
   const int32_t* cu_seqlens;  // as in FwdParams
   int max_seqlen;
   const uint8_t* block_mask;  // as in FwdParams ([n_ktiles][n_ktiles])
+  // packed batches: longest-first work order (workspace, built by
+  // fa_bwd_rank): lengths [B], sequences by rank [B], super-units before each
+  // rank [B + 1]; nullptr: head-major order
+  int* rank;
   uint32_t seed_lo, seed_hi, drop_offset, keep_t;  // as in FwdParams
   float inv_keep;
   int B, H, N;
@@ -212,5 +216,9 @@ cudaError_t launch_bwd_main(int d, bool bf16, const CUtensorMap& tmq, const CUte
                             cudaStream_t stream);
 cudaError_t launch_bwd_post(int d, bool bf16, const BwdParams& p, int num_sms,
                             cudaStream_t stream);
+// Packed batches of at most this many sequences get the longest-first
+// backward order; the table takes 3 B + 1 ints of the workspace.
+constexpr int kBwdRankMaxSeqs = 4096;
+cudaError_t launch_bwd_rank(const BwdParams& p, cudaStream_t stream);
 
 }  // namespace fa

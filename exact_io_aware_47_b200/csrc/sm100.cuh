@@ -34,6 +34,9 @@ __device__ __forceinline__ void record_error(unsigned code, unsigned site) {
 // Optional device timeline (build with -DFA_TRACE): SM clock stamps of
 // pipeline events of CTA 0, slot = iteration * 32 + event.  Compiled out by
 // default.
+#ifndef FA_TRACE_SM_THREAD
+#define FA_TRACE_SM_THREAD 0  // the softmax thread whose events are recorded
+#endif
 #ifdef FA_TRACE
 constexpr int kTraceSlots = 1 << 16;
 __device__ unsigned long long g_trace[kTraceSlots];
@@ -87,6 +90,15 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
+#ifdef FA_WAIT_HINT_NS
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "n"(FA_WAIT_HINT_NS)
+      : "memory");
+#else
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
@@ -94,6 +106,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "=r"(ok)
       : "r"(bar), "r"(parity)
       : "memory");
+#endif
   return ok != 0;
 }
 
@@ -474,6 +487,34 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 
+// N (16 or 32) consecutive columns from a register array, by pointer (the
+// caller's indices are compile-time after unrolling).
+template <int N>
+__device__ __forceinline__ void tmem_st_n(uint32_t taddr, const uint32_t* r) {
+  static_assert(N == 16 || N == 32, "16 or 32 columns");
+  if constexpr (N == 16) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+        : "memory");
+  } else {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+        "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+        "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+        "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+  }
+}
+
 // Wide TMEM moves (generated): 64 or 128 consecutive columns per thread.
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
   asm volatile(
@@ -621,6 +662,34 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x for a pair of fp32 values on the FMA and integer pipes (no
+// special-function unit), written from the textbook method: range reduction
+// x = n + f with n = round(x) (adding 1.5 * 2^23 + 127 rounds x to an integer
+// under round-to-nearest and leaves n + 127, the biased exponent of 2^n, in
+// the low mantissa bits) and f in [-1/2, 1/2]; 2^f from a cubic
+// c0 + f (c1 + f (c2 + f c3)) whose coefficients minimise the largest
+// relative error over [-1/2, 1/2] (fitted here as a linear program over a
+// dense grid; the fp32 evaluation stays within 7.5e-5 of 2^f); then the
+// product with 2^n, built from the biased exponent.  x is clamped to >= -127,
+// where 2^n is +0, so very negative inputs give exactly 0 (as the flushing
+// ex2.approx.ftz does below 2^-126); x must stay below 127.
+__device__ __forceinline__ unsigned long long exp2_poly2(float x0, float x1) {
+  constexpr float kShift = 12583039.f;  // 1.5 * 2^23 + 127, exact in fp32
+  const unsigned long long x = f2pack(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
+  const unsigned long long t = fadd2(x, f2pack(kShift, kShift));
+  const unsigned long long n = fadd2(t, f2pack(-kShift, -kShift));        // round(x)
+  const unsigned long long f = ffma2(n, f2pack(-1.f, -1.f), x);           // x - n
+  unsigned long long p = f2pack(0.05517222f, 0.05517222f);
+  p = ffma2(p, f, f2pack(0.24261116f, 0.24261116f));
+  p = ffma2(p, f, f2pack(0.69326086f, 0.69326086f));
+  p = ffma2(p, f, f2pack(0.99992808f, 0.99992808f));
+  float t0, t1;
+  f2unpack(t, t0, t1);
+  const unsigned long long e = f2pack(__uint_as_float(__float_as_uint(t0) << 23),
+                                      __uint_as_float(__float_as_uint(t1) << 23));  // 2^n
+  return fmul2(p, e);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -225,12 +225,17 @@ int fa_fwd_e4m3(const void* q8, const void* k8, const void* v8, const float* q_d
  *     that is out of range (decreasing, past T, a sequence longer than
  *     max_seqlen) is clamped on the device and reported by
  *     fa_device_status() as FA_ERR_DEVICE_SEQLEN.
- *   fa_bwd_varlen's workspace: fa_bwd_workspace_size(1, H, T, d) bytes,
- *     256-byte aligned; it runs the three backward stages on `stream`.
+ *   fa_bwd_varlen's workspace: fa_bwd_varlen_workspace_size(B, H, T, d)
+ *     bytes, 256-byte aligned: the row dots and dQ accumulator of
+ *     fa_bwd_workspace_size(1, H, T, d), then (for B <= 4096) the table of
+ *     the longest-first work order.  It runs the three backward stages on
+ *     `stream`, with a one-block kernel that ranks the sequences by length
+ *     before the main kernel (B > 4096: head-major order, no table).
  */
 int fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
                   const int32_t* cu_seqlens, int B, int H, int T, int max_seqlen,
                   int d, float scale, int causal, int dtype, void* stream);
+size_t fa_bwd_varlen_workspace_size(int B, int H, int T, int d);
 int fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
                   const void* dout, const float* lse, void* dq, void* dk, void* dv,
                   void* workspace, size_t workspace_bytes, const int32_t* cu_seqlens,

@@ -93,6 +93,18 @@ def test_rejections_before_any_cuda_call(lib):
     assert bwd(H=0) == _lib.FA_ERR_INVALID_ARG
 
 
+def test_varlen_workspace_size(lib):
+    """The packed backward's workspace: the dense one for [H, T, d], then the
+    longest-first table (3 B + 1 ints, 256-byte padded) for B <= 4096."""
+    H, T, d = 3, 1000, 64
+    base = lib.fa_bwd_workspace_size(1, H, T, d)
+    assert lib.fa_bwd_varlen_workspace_size(1, H, T, d) == base + 256
+    assert lib.fa_bwd_varlen_workspace_size(100, H, T, d) == base + (301 * 4 + 255) // 256 * 256
+    assert lib.fa_bwd_varlen_workspace_size(5000, H, T, d) == base
+    assert lib.fa_bwd_varlen_workspace_size(0, H, T, d) == 0
+    assert lib.fa_bwd_varlen_workspace_size(2, H, T, 96) == 0
+
+
 def test_noalloc_size_limit_checked_on_the_host(lib):
     from exact_io_aware_47_b200 import _lib
     P = 1 << 20

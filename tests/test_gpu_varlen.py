@@ -207,7 +207,7 @@ def test_host_side_rejections(fa):
                                 lse.data_ptr(), args["cu"], args["B"], 1, args["T"], args["ms"],
                                 args["d"], 0.125, 0, _lib.FA_BF16, s)
         assert st in (_lib.FA_ERR_INVALID_ARG, _lib.FA_ERR_UNSUPPORTED), (kw, st)
-    ws = torch.empty(_lib.fa_bwd_workspace_size(1, 1, 128, 64) - 256, dtype=torch.uint8,
+    ws = torch.empty(_lib.fa_bwd_varlen_workspace_size(1, 1, 128, 64) - 256, dtype=torch.uint8,
                      device="cuda")
     st = _lib.fa_bwd_varlen(q.data_ptr(), q.data_ptr(), q.data_ptr(), q.data_ptr(), q.data_ptr(),
                             lse.data_ptr(), q.data_ptr(), q.data_ptr(), q.data_ptr(),
