@@ -590,8 +590,8 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4)
               pd[k4] = DROPOUT && !((drop_keep[cc] >> (e + k4)) & 1u) ? 0.f : pv[cc * 32 + e + k4];
-            pp[(e >> 1)] = pack_op2<BF16>(pd[0], pd[1]);
-            pp[(e >> 1) + 1] = pack_op2<BF16>(pd[2], pd[3]);
+            pp[(e >> 1)] = pack2<BF16>(pd[0], pd[1]);
+            pp[(e >> 1) + 1] = pack2<BF16>(pd[2], pd[3]);
           }
           // P^T of queries [32c, 32c+32) goes to columns 64 half + 16 (c & 1): only
           // over S^T columns this thread has already read, never the other
@@ -638,8 +638,8 @@ __global__ void __launch_bounds__(512, 1)
             float gv[4];
             f2unpack(fmul2(f2pack(pv[b0], pv[b0 + 1]), x01), gv[0], gv[1]);
             f2unpack(fmul2(f2pack(pv[b0 + 2], pv[b0 + 3]), x23), gv[2], gv[3]);
-            dd[(e >> 1)] = pack_op2<BF16>(gv[0], gv[1]);
-            dd[(e >> 1) + 1] = pack_op2<BF16>(gv[2], gv[3]);
+            dd[(e >> 1)] = pack2<BF16>(gv[0], gv[1]);
+            dd[(e >> 1) + 1] = pack2<BF16>(gv[2], gv[3]);
           }
           // four 16-byte units of the 128-byte swizzled row (chunk c = units
           // 4 (c & 1) .. 4 (c & 1) + 3 of panel `half`)

@@ -522,6 +522,7 @@ __global__ void __launch_bounds__(384, 1)
         tc_fence_after();
         uint32_t sr[128];  // raw scores q.k of this row, one TMEM load
         tmem_ld128(tS, sr);
+        if (r == 0 && t == 0) FA_TRACE_AT(scnt - 1, 6);
         const int kbase = j * kBlockN;
         const bool need_mask = (p.causal && j == qt) || (kbase + kBlockN > w.L);
         if (need_mask) {
@@ -545,6 +546,7 @@ __global__ void __launch_bounds__(384, 1)
         const float mx = fmax3(mc[0], mc[1], fmaxf(mc[2], mc[3])) * cj;  // log2 units (cj > 0)
         const float m_new = (mx > m + kRescaleThreshold) ? mx : m;
         const bool moved = m_new != m;
+        if (r == 0 && t == 0) FA_TRACE_AT(scnt - 1, 7);
         const float alpha = moved ? ex2_approx(m - m_new) : 1.f;  // 0 when m was -inf
         l *= alpha;
         m = m_new;
@@ -577,7 +579,8 @@ __global__ void __launch_bounds__(384, 1)
             const uint32_t h = pack_e4m3x2(p0 * rho, p1 * rho);
             pk[i >> 1] = (i & 1) ? (pk[i >> 1] | (h << 16)) : h;
           } else {
-            pk[i] = pack_op2<BF16>(p0, p1);
+            pk[i] = pack2<BF16>(p0, p1);
+            if (r == 0 && t == 0 && (i & 15) == 15) FA_TRACE_AT(scnt - 1, 8 + (i >> 4));
             // P goes back to TMEM in chunks as it is made, so the stores
             // overlap the rest of the loop
             if constexpr (kFwdStoreChunks > 1) {
@@ -596,6 +599,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         if constexpr (FP8) tmem_st32(tS, pk);
         else if (kFwdStoreChunks == 1) tmem_st64(tS, pk);
+        if (r == 0 && t == 0) FA_TRACE_AT(scnt - 1, 12);
         if (jj > 0 && __any_sync(0xffffffffu, moved)) {
           // O_t holds the sum up to the previous key tile (its MMA completed
           // before S_t(j) was committed) and PV_t(j) waits for p_full:
@@ -609,7 +613,9 @@ __global__ void __launch_bounds__(384, 1)
             tmem_st32(tO + cc * 32, ro);
           }
         }
+        if (r == 0 && t == 0) FA_TRACE_AT(scnt - 1, 13);
         tmem_st_wait();
+        if (r == 0 && t == 0) FA_TRACE_AT(scnt - 1, 14);
         tc_fence_before();
         mbar_arrive(&p_full[t]);
         if (r == 0) FA_TRACE_AT(scnt - 1, 3 + 2 * t);

@@ -708,30 +708,6 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   else return pack_f16x2(lo, hi);
 }
 
-// Two finite fp32 values to bf16x2 on the integer pipe: round to nearest,
-// ties away from zero (adding half a bf16 unit to the magnitude bits, then
-// keeping the high halves).  It differs from round-to-nearest-even only on
-// exact ties.  Used for tensor-core operands made in the softmax loops, where
-// the conversion instruction would compete with ex2 for the
-// special-function pipe.
-__device__ __forceinline__ uint32_t pack_bf16x2_int(float lo, float hi) {
-  const uint32_t a = __float_as_uint(lo) + 0x8000u;
-  const uint32_t b = __float_as_uint(hi) + 0x8000u;
-  return __byte_perm(a, b, 0x7632);
-}
-
-// Tensor-core operand pack (P, P^T, dS^T): bf16 on the integer pipe, fp16
-// with the conversion instruction.
-template <bool BF16>
-__device__ __forceinline__ uint32_t pack_op2(float lo, float hi) {
-#ifdef FA_PACK_CVT
-  return pack2<BF16>(lo, hi);
-#else
-  if constexpr (BF16) return pack_bf16x2_int(lo, hi);
-  else return pack_f16x2(lo, hi);
-#endif
-}
-
 // Two fp32 values to two e4m3 bytes (round to nearest even, saturating to
 // +-448): lo in bits 0..7, hi in bits 8..15.
 __device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
