@@ -15,26 +15,26 @@
 //  2. fa_bwd_kernel (persistent, one CTA per SM, 512 threads): a work unit is
 //     (batch*head, 128-key tile j).  K_j and V_j stay in shared memory while
 //     the query tiles i (i >= j when causal) stream past:
-//       S^T  = K_j Q_i^T      (tcgen05, TMEM, keys on lanes)
-//       dP^T = V_j dO_i^T     (tcgen05, TMEM)
-//       P^T  = exp2(c S^T - LSE_i log2 e), dS^T = P^T * (dP^T - D_i)
-//                              (warps 0-7, one key row and half the queries
-//                              per thread; P^T goes back to TMEM over S^T as
-//                              16-bit, dS^T to a swizzled shared-memory tile)
-//       dQ_i  = dS K_j     (issued first; d = 128 computes dQ_i^T = K_j^T dS^T
-//                           so each warp's reduce-add is one contiguous row
-//                           segment; warps 8-11 add it into the fp32
-//                           accumulator in global memory)
+//       S^T  = K_j Q_i^T      (tcgen05, TMEM region A, keys on lanes)
+//       P^T  = exp2(c S^T - LSE_i log2 e)  (warps 0-7, one key row and half
+//                              the queries per thread; to region B as 16-bit)
+//       dP^T = V_j dO_i^T     (region A, once S^T has been loaded out of it)
+//       dS^T = P^T * (dP^T - D_i)  (warps 0-7, from dP^T and the 16-bit P^T;
+//                              to a swizzled shared-memory tile)
 //       dV_j += P^T dO_i,  dK_j += dS^T Q_i   (TMEM accumulators)
+//       dQ_i  = dS K_j     (region B, once dV has read P^T out of it; warps
+//                           8-11 add it into the fp32 accumulator in global
+//                           memory with TMA reduce-adds)
 //     warp 12 issues the MMAs, warp 13 the TMA loads, warp 14 stages LSE_i
 //     and D_i in shared memory; warps 8-11 also write dK_j (times scale) and
 //     dV_j at the end of the unit;
 //  3. fa_bwd_post: dQ = scale * accumulator, rounded to 16-bit.
 //
-// TMEM columns: S^T [0,128) with P^T (16-bit) over [0,32) and [64,96),
-// dP^T [128,256), dV [256,256+d),
-// dK [256+d,256+2d); dQ_i reuses the dP^T columns when d = 128 (the 512
-// columns are all taken) and [384,448) when d = 64.
+// TMEM columns: region A [0,128) holds S^T(i), then dP^T(i); region B
+// [128,256) holds P^T(i) (16-bit, columns 0-31 and 64-95 of the region; with
+// dropout the unmasked copy in 32-63 and 96-127), then dQ(i); dV [256,256+d),
+// dK [256+d,256+2d).  Each region is handed on as soon as its contents have
+// been read, so no MMA waits for work that does not produce its operands.
 #include <algorithm>
 
 #include <cuda_bf16.h>
@@ -64,11 +64,10 @@ struct BwdLayout {
   static constexpr int kSmemMax = 232448;              // sm_100 per-block opt-in maximum
   static constexpr int kSmemBytes = (kUsed + 1024 <= kSmemMax) ? kUsed + 1024 : kSmemMax;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kColS = 0;
-  static constexpr uint32_t kColDP = 128;
+  static constexpr uint32_t kColA = 0;    // S^T(i), then dP^T(i)
+  static constexpr uint32_t kColB = 128;  // P^T(i) (16-bit), then dQ(i)
   static constexpr uint32_t kColDV = 256;
   static constexpr uint32_t kColDK = 256 + D;
-  static constexpr uint32_t kColDQ = (D == 128) ? 128 : 256 + 2 * D;
 };
 
 struct BwdUnit {
@@ -77,6 +76,15 @@ struct BwdUnit {
   int z, row0, rows;  // slice placement (SliceInfo)
   bool skip;          // packed key tile past its sequence: no role does anything
 };
+
+// dQ_i leaves the SM by per-thread fp32 reduce-adds from registers (d = 128,
+// dQ computed transposed) instead of a shared-memory staging tile and TMA
+// reduce-adds; a build option while the two are compared.
+#ifndef FA_BWD_DQ_RED
+#define FA_BWD_DQ_RED 0
+#endif
+template <int D>
+constexpr bool kDqRed = FA_BWD_DQ_RED != 0 && D == 128;
 
 // Register split: 512 threads launched at 128 registers (launch bounds 512,1);
 // the softmax warpgroups keep their P^T values between the two phases and the
@@ -202,7 +210,9 @@ __global__ void __launch_bounds__(512, 1)
   uint64_t* dkv_empty = bars + 19;
   uint64_t* drain = bars + 20;
   uint64_t* ds_full = bars + 21;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 22);
+  uint64_t* s_read = bars + 22;   // the first softmax phase has loaded S^T out of region A
+  uint64_t* dp_read = bars + 23;  // the second phase has loaded dP^T out of region A
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const WaitCtl wc{abort_flag, p.wait_ns};  // every pipeline wait of this CTA
 
@@ -230,6 +240,8 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(dkv_full, 1);
     mbar_init(dkv_empty, 128);
     mbar_init(drain, 1);
+    mbar_init(s_read, 256);
+    mbar_init(dp_read, 256);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -346,6 +358,8 @@ __global__ void __launch_bounds__(512, 1)
       constexpr uint32_t kIdTS = idesc_f16(BF16, 128, D, false, true);    // dV, dK (B MN-major)
       // dQ = dS K_j (M = queries, N = d): a TMEM lane holds one query row
       constexpr uint32_t kIdDQ = idesc_f16(BF16, 128, D, true, true);
+      // dQ^T = K_j^T dS^T (M = d, N = queries): a TMEM lane holds one d index
+      constexpr uint32_t kIdDQT = idesc_f16(BF16, 128, 128, true, true);
       // Low descriptor words of every operand tile, K-major (_k) or MN-major
       // (_m) view; the grouped MMAs derive the K steps from them.
       const uint32_t aSlot = smem_addr(sSlot);
@@ -373,36 +387,35 @@ __global__ void __launch_bounds__(512, 1)
         // barrier never runs two phases ahead of its waiter, also for units
         // with no query tiles).
         bool dkv_free = nunit == 0;
-        // Software pipeline over the query tiles of the unit:
-        //   S(0) | dP(i), dV(i), S(i+1), dK(i), dQ(i) | ...
-        // so the softmax of tile i+1 (first phase, from S) runs while the
-        // tensor core does dK(i) and dQ(i), and its second phase (from dP)
-        // while it does dV(i+1).
-        auto issue_s = [&](int t) {  // S^T(t) = K_j Q_t^T, Q_t in slot t & 1
-          umma_ss_group<D / 16, false, false>(tmem + Lay::kColS, lK_k, (t & 1) ? lQ1_k : lQ0_k,
+        // Software pipeline over the query tiles of the unit.  TMEM region A
+        // holds S^T(i), then dP^T(i); region B holds P^T(i), then dQ(i):
+        //   dP(i) once the first softmax phase has loaded S^T(i) out of A,
+        //   dV(i) once it has written P^T(i) into B,
+        //   S(i+1) once the second phase has loaded dP^T(i) out of A,
+        //   dQ(i) into B (dV(i), issued before it, has read P^T(i)) and dK(i)
+        //   once dS^T(i) is in shared memory.
+        // No MMA waits for the exponentials of the tile it overwrites, nor for
+        // the read-out of dQ (the first phase of the next tile waits for that
+        // before it writes P^T into B).
+        auto issue_s = [&](int t) -> bool {  // S^T(t) = K_j Q_t^T, Q_t in slot t & 1
+          if (t > 0 && !mbar_wait(dp_read, (t - 1) & 1, wc, 37)) return false;
+          if (!mbar_wait(&slot_full[t & 1], (t >> 1) & 1, wc, 24)) return false;
+          tc_fence_after();
+          umma_ss_group<D / 16, false, false>(tmem + Lay::kColA, lK_k, (t & 1) ? lQ1_k : lQ0_k,
                                               kIdS, 0u);
           umma_commit(s_full);
+          return true;
         };
-        if (w.ni > 0) {
-          ok = mbar_wait(&slot_full[it & 1], (it >> 1) & 1, wc, 24);
-          if (!ok) break;
-          tc_fence_after();
-          issue_s(it);
-        }
+        if (w.ni > 0) ok = issue_s(it);
         for (int idx = 0; idx < w.ni && ok; ++idx) {
           FA_TRACE_AT(it, 0);
-          // d = 128: dQ^T of the previous tile lives in the dP^T columns
-          if (D == 128 && it > 0) {
-            ok = mbar_wait(dq_empty, (it - 1) & 1, wc, 25);
-            if (!ok) break;
-          }
-          FA_TRACE_AT(it, 30);
-          ok = mbar_wait(&slot_full[2], it & 1, wc, 35);
+          // dP^T = V_j dO_i^T into region A
+          ok = mbar_wait(s_read, it & 1, wc, 25);
+          if (ok) ok = mbar_wait(&slot_full[2], it & 1, wc, 35);
           if (!ok) break;
           tc_fence_after();
           FA_TRACE_AT(it, 1);
-          // dP^T = V_j dO_i^T
-          umma_ss_group<D / 16, false, false>(tmem + Lay::kColDP, lV_k, lO_k, kIdS, 0u);
+          umma_ss_group<D / 16, false, false>(tmem + Lay::kColA, lV_k, lO_k, kIdS, 0u);
           umma_commit(dp_full);
           // dV_j += P^T dO_i once the first softmax phase wrote P^T
           ok = mbar_wait(p_full, it & 1, wc, 26);
@@ -415,19 +428,15 @@ __global__ void __launch_bounds__(512, 1)
             tc_fence_after();
             dkv_free = true;
           }
-          // (A = P^T in TMEM, 16 queries = 8 columns; queries 64..127 sit 64
-          // columns further, in the second half's S^T columns)
-          umma_ts_group8<true, true>(tmem + Lay::kColDV, tmem + Lay::kColS, lO_m, kIdTS,
+          // (A = P^T in TMEM region B, 16 queries = 8 columns; queries 64..127
+          // sit 64 columns further)
+          umma_ts_group8<true, true>(tmem + Lay::kColDV, tmem + Lay::kColB, lO_m, kIdTS,
                                      idx > 0 ? 1u : 0u);
           umma_commit(&slot_empty[2]);  // dO_i: dP and dV done
           FA_TRACE_AT(it, 13);
-          // S^T of the next tile: its MMA runs after dV (in order), which has
-          // read P^T out of these columns
           if (idx + 1 < w.ni) {
-            ok = mbar_wait(&slot_full[(it + 1) & 1], ((it + 1) >> 1) & 1, wc, 24);
+            ok = issue_s(it + 1);
             if (!ok) break;
-            tc_fence_after();
-            issue_s(it + 1);
           }
           FA_TRACE_AT(it, 14);
           // dQ and dK_j += dS^T Q_i once the second phase wrote dS^T
@@ -435,32 +444,22 @@ __global__ void __launch_bounds__(512, 1)
           if (!ok) break;
           tc_fence_after();
           FA_TRACE_AT(it, 8);
-          auto issue_dk = [&]() {  // A = dS^T K-major, B = Q_i MN-major
-            umma_ss_group<8, false, true>(tmem + Lay::kColDK, lS_k, (it & 1) ? lQ1_m : lQ0_m,
-                                          kIdTS, idx > 0 ? 1u : 0u);
-            umma_commit(&slot_empty[it & 1]);  // Q_i: S and dK done
-          };
-          // dQ = dS K_j: A = dS^T read MN-major (queries contiguous), B = K_j
-          // read MN-major (d contiguous)
-          auto issue_dq = [&]() {
-            umma_ss_group<8, true, true>(tmem + Lay::kColDQ, lS_m, lK_m, kIdDQ, 0u);
-            umma_commit(dq_full);
-          };
-          if constexpr (D == 128) {
-            // dQ lives in the dP^T columns: issued before dK, so that the dQ
-            // warps release them for the next tile's dP^T while dK runs
-            issue_dq();
-            issue_dk();
+          if constexpr (kDqRed<D>) {
+            // dQ^T = K_j^T dS^T into region B (a TMEM lane per d index): A =
+            // K_j read MN-major (d contiguous), B = dS^T read MN-major
+            // (queries contiguous)
+            umma_ss_group<8, true, true>(tmem + Lay::kColB, lK_m, lS_m, kIdDQT, 0u);
           } else {
-            issue_dk();
-            if (it > 0) {
-              ok = mbar_wait(dq_empty, (it - 1) & 1, wc, 25);
-              if (!ok) break;
-              tc_fence_after();
-            }
-            issue_dq();
+            // dQ = dS K_j into region B: A = dS^T read MN-major (queries
+            // contiguous), B = K_j read MN-major (d contiguous)
+            umma_ss_group<8, true, true>(tmem + Lay::kColB, lS_m, lK_m, kIdDQ, 0u);
           }
-          umma_commit(ds_empty);  // dK and dQ have read dS^T
+          umma_commit(dq_full);
+          // dK_j += dS^T Q_i: A = dS^T K-major, B = Q_i MN-major
+          umma_ss_group<8, false, true>(tmem + Lay::kColDK, lS_k, (it & 1) ? lQ1_m : lQ0_m, kIdTS,
+                                        idx > 0 ? 1u : 0u);
+          umma_commit(&slot_empty[it & 1]);  // Q_i: S and dK done
+          umma_commit(ds_empty);             // dK and dQ have read dS^T
           FA_TRACE_AT(it, 3);
           ++it;
         }
@@ -525,8 +524,8 @@ __global__ void __launch_bounds__(512, 1)
     const int half = warp >> 2;              // queries [64 half, 64 half + 64)
     const int r = ((warp & 3) << 5) | lane;  // key row in the tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_off + Lay::kColS;
-    const uint32_t tDP = tmem + lane_off + Lay::kColDP;
+    const uint32_t tA = tmem + lane_off + Lay::kColA;  // S^T, then dP^T
+    const uint32_t tB = tmem + lane_off + Lay::kColB;  // P^T (16-bit), then dQ
     // dS^T row r, queries of this half: panel `half` of the swizzled tile
     const uint32_t ds_row = smem_addr(sDS) + half * 16384 + r * 128;
     const float cl = p.scale_log2;
@@ -556,7 +555,8 @@ __global__ void __launch_bounds__(512, 1)
             drop_keep[g >> 1] = (g & 1) ? (drop_keep[g >> 1] & 0xFFFFu) | (m16 << 16) : m16;
           }
         }
-        // ---- phase 1: P^T = 2^(c S^T - LSE_i log2 e) from S^T, back to TMEM
+        // ---- phase 1: P^T = 2^(c S^T - LSE_i log2 e) from S^T (region A),
+        // to region B as 16-bit for the dV product
         ok = mbar_wait_warp(&ld_full[st], (it >> 1) & 1, wc, 28) &&
              mbar_wait_warp(s_full, it & 1, wc, 29);
         if (!ok) break;
@@ -566,93 +566,105 @@ __global__ void __launch_bounds__(512, 1)
         const int diag_lim = (p.causal && i == w.j) ? r : -1;  // visible iff q_local >= r
         const float* lse2 = sLSE + st * 128;
         const float* dsm = sDSUM + st * 128;
-        float pv[64];  // this thread's P^T values, kept for the second phase
+        uint32_t pp[32];               // P^T as dV sees it (dropped scores zero), 16-bit pairs
+        uint32_t pu[DROPOUT ? 32 : 1];  // dropout: P^T before the mask, for the second phase
+        {
+          uint32_t sr[64];  // S^T of this key row, the half's 64 queries
+          tmem_ld64(tA + 64 * half, sr);
+          // region A may now take dP^T(i)
+          tc_fence_before();
+          mbar_arrive(s_read);
+          if (threadIdx.x == FA_TRACE_SM_THREAD) FA_TRACE_AT(it, 10);
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int c = half * 2 + cc;  // 32-query chunk
-          uint32_t sr[32];
-          if (threadIdx.x == FA_TRACE_SM_THREAD && cc == 1) FA_TRACE_AT(it, 27);
-          tmem_ld32(tS + c * 32, sr);
-          if (threadIdx.x == FA_TRACE_SM_THREAD) FA_TRACE_AT(it, cc == 0 ? 10 : 24);
-          uint32_t pp[16];
-#pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            const int q0 = c * 32 + e;
+          for (int e = 0; e < 64; e += 4) {
+            const int q0 = 64 * half + e;  // query inside the tile
             const float4 l4 = *reinterpret_cast<const float4*>(lse2 + q0);
             const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+            float pv[4], pd[4];
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
               const bool vis = key_ok && (q0 + k4 >= diag_lim);
               const float x = fmaf(__uint_as_float(sr[e + k4]), cl, -lv[k4]);
-              pv[cc * 32 + e + k4] = vis ? ex2_approx(x) : 0.f;
+              pv[k4] = vis ? ex2_approx(x) : 0.f;
+              // P^T as dV sees it: dropped scores are zero
+              pd[k4] = DROPOUT && !((drop_keep[e >> 5] >> ((e & 31) + k4)) & 1u) ? 0.f : pv[k4];
             }
-            float pd[4];  // P^T as dV sees it: dropped scores are zero
-#pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4)
-              pd[k4] = DROPOUT && !((drop_keep[cc] >> (e + k4)) & 1u) ? 0.f : pv[cc * 32 + e + k4];
-            pp[(e >> 1)] = pack2<BF16>(pd[0], pd[1]);
+            pp[e >> 1] = pack2<BF16>(pd[0], pd[1]);
             pp[(e >> 1) + 1] = pack2<BF16>(pd[2], pd[3]);
+            if constexpr (DROPOUT) {
+              pu[e >> 1] = pack2<BF16>(pv[0], pv[1]);
+              pu[(e >> 1) + 1] = pack2<BF16>(pv[2], pv[3]);
+            }
           }
-          // P^T of queries [32c, 32c+32) goes to columns 64 half + 16 (c & 1): only
-          // over S^T columns this thread has already read, never the other
-          // half's
-          tmem_st16(tS + half * 64 + (c & 1) * 16, pp);
         }
-        if (threadIdx.x == FA_TRACE_SM_THREAD) FA_TRACE_AT(it, 25);
+        // region B still holds dQ(i-1) until the dQ warps have read it
+        if (it > 0) {
+          ok = mbar_wait_warp(dq_empty, (it - 1) & 1, wc, 38);
+          if (!ok) break;
+        }
+        tc_fence_after();
+        // P^T of the half's queries [64 half, 64 half + 64): columns 64 half ..
+        // 64 half + 31 of region B (16 queries per 8 columns); with dropout the
+        // unmasked copy goes to the next 32 columns
+        tmem_st_n<32>(tB + 64 * half, pp);
+        if constexpr (DROPOUT) tmem_st_n<32>(tB + 64 * half + 32, pu);
         tmem_st_wait();
-        if (threadIdx.x == FA_TRACE_SM_THREAD) FA_TRACE_AT(it, 26);
         tc_fence_before();
         mbar_arrive(p_full);
         if (threadIdx.x == FA_TRACE_SM_THREAD) FA_TRACE_AT(it, 15);
-        // ---- phase 2: dS^T = P^T * (dP^T - D_i) from dP^T, to shared memory
+        // ---- phase 2: dS^T = P^T * (dP^T - D_i) from dP^T (region A) and the
+        // 16-bit P^T (region B), to shared memory
         ok = mbar_wait_warp(dp_full, it & 1, wc, 30);
         if (ok && it > 0) ok = mbar_wait_warp(ds_empty, (it - 1) & 1, wc, 31);
         if (!ok) break;
         tc_fence_after();
         if (threadIdx.x == FA_TRACE_SM_THREAD) FA_TRACE_AT(it, 11);
+        uint32_t dr[64];  // dP^T of this key row, the half's 64 queries
+        tmem_ld64(tA + 64 * half, dr);
+        uint32_t pq[32];  // P^T, 16-bit pairs (unmasked with dropout)
+        tmem_ld32(tB + 64 * half + (DROPOUT ? 32 : 0), pq);
+        // region A may now take S^T(i+1)
+        tc_fence_before();
+        mbar_arrive(dp_read);
+        if (threadIdx.x == FA_TRACE_SM_THREAD) FA_TRACE_AT(it, 12);
+        uint32_t dd[16];
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int c = half * 2 + cc;
-          uint32_t dr[32];
-          if (threadIdx.x == FA_TRACE_SM_THREAD && cc == 1) FA_TRACE_AT(it, 28);
-          tmem_ld32(tDP + c * 32, dr);
-          if (threadIdx.x == FA_TRACE_SM_THREAD) FA_TRACE_AT(it, cc == 0 ? 12 : 21);
-          uint32_t dd[16];
+        for (int e = 0; e < 64; e += 4) {
+          const int q0 = 64 * half + e;
+          const float4 nd = *reinterpret_cast<const float4*>(dsm + q0);  // -D
+          if constexpr (DROPOUT) {  // dP of the kept scores, scaled by 256 / t
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            const int q0 = c * 32 + e;
-            const float4 nd = *reinterpret_cast<const float4*>(dsm + q0);  // -D
-            if constexpr (DROPOUT) {  // dP of the kept scores, scaled by 256 / t
-#pragma unroll
-              for (int k4 = 0; k4 < 4; ++k4)
-                dr[e + k4] = (drop_keep[cc] >> (e + k4)) & 1u
-                                 ? __float_as_uint(__uint_as_float(dr[e + k4]) * p.inv_keep)
-                                 : 0u;
-            }
-            // packed pairs: (dP - D) then P (dP - D)
-            const int b0 = cc * 32 + e;
-            const auto x01 = fadd2(f2pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])),
-                                   f2pack(nd.x, nd.y));
-            const auto x23 = fadd2(f2pack(__uint_as_float(dr[e + 2]), __uint_as_float(dr[e + 3])),
-                                   f2pack(nd.z, nd.w));
-            float gv[4];
-            f2unpack(fmul2(f2pack(pv[b0], pv[b0 + 1]), x01), gv[0], gv[1]);
-            f2unpack(fmul2(f2pack(pv[b0 + 2], pv[b0 + 3]), x23), gv[2], gv[3]);
-            dd[(e >> 1)] = pack2<BF16>(gv[0], gv[1]);
-            dd[(e >> 1) + 1] = pack2<BF16>(gv[2], gv[3]);
+            for (int k4 = 0; k4 < 4; ++k4)
+              dr[e + k4] = (drop_keep[e >> 5] >> ((e & 31) + k4)) & 1u
+                               ? __float_as_uint(__uint_as_float(dr[e + k4]) * p.inv_keep)
+                               : 0u;
           }
-          // four 16-byte units of the 128-byte swizzled row (chunk c = units
-          // 4 (c & 1) .. 4 (c & 1) + 3 of panel `half`)
+          float pf[4];
+          unpack2<BF16>(pq[e >> 1], pf[0], pf[1]);
+          unpack2<BF16>(pq[(e >> 1) + 1], pf[2], pf[3]);
+          // packed pairs: (dP - D) then P (dP - D)
+          const auto x01 = fadd2(f2pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])),
+                                 f2pack(nd.x, nd.y));
+          const auto x23 = fadd2(f2pack(__uint_as_float(dr[e + 2]), __uint_as_float(dr[e + 3])),
+                                 f2pack(nd.z, nd.w));
+          float gv[4];
+          f2unpack(fmul2(f2pack(pf[0], pf[1]), x01), gv[0], gv[1]);
+          f2unpack(fmul2(f2pack(pf[2], pf[3]), x23), gv[2], gv[3]);
+          dd[(e & 31) >> 1] = pack2<BF16>(gv[0], gv[1]);
+          dd[((e & 31) >> 1) + 1] = pack2<BF16>(gv[2], gv[3]);
+          if ((e & 31) == 28) {
+            // 32 queries done: four 16-byte units of the 128-byte swizzled row
+            // (units 4 cc .. 4 cc + 3 of panel `half`, cc = e / 32)
 #pragma unroll
-          for (int w4 = 0; w4 < 4; ++w4) {
-            const uint32_t unit = ((c & 1) * 4 + w4) ^ (r & 7);
-            st_shared_v4(ds_row + unit * 16, dd[4 * w4], dd[4 * w4 + 1], dd[4 * w4 + 2],
-                         dd[4 * w4 + 3]);
+            for (int w4 = 0; w4 < 4; ++w4) {
+              const uint32_t unit = ((e >> 5) * 4 + w4) ^ (r & 7);
+              st_shared_v4(ds_row + unit * 16, dd[4 * w4], dd[4 * w4 + 1], dd[4 * w4 + 2],
+                           dd[4 * w4 + 3]);
+            }
           }
         }
         if (threadIdx.x == FA_TRACE_SM_THREAD) FA_TRACE_AT(it, 22);
         fence_proxy_async_smem();
-        if (threadIdx.x == FA_TRACE_SM_THREAD) FA_TRACE_AT(it, 23);
         tc_fence_before();
         mbar_arrive(ds_full);
         mbar_arrive(&ld_empty[st]);
@@ -691,11 +703,27 @@ __global__ void __launch_bounds__(512, 1)
         // transfer (the TMA path sustains more reduce bandwidth per SM than
         // per-thread reds); staging a round overlaps the previous transfer.
         // Rows past N are clipped by the transfer.
-        {
+        if constexpr (kDqRed<D>) {
+          // Lane r holds d index r of dQ_i^T for the tile's 128 queries: read
+          // them, release the TMEM columns, and add them into the fp32
+          // accumulator from registers; the 32 lanes of a warp cover 32
+          // consecutive d of one query row, so every reduce of a warp is one
+          // 128-byte line.  Rows past the slice's computed rows are skipped.
+          uint32_t v[128];
+          tmem_ld64x2(tmem + lane_off + Lay::kColB, v);
+          if (threadIdx.x == 256) FA_TRACE_AT(it, 29);
+          tc_fence_before();
+          mbar_arrive(dq_empty);
+          const int qn = min(kBlockM, w.rows - i * kBlockM);
+          float* acc = p.dq_acc + (base + static_cast<size_t>(i) * kBlockM) * D + r;
+#pragma unroll
+          for (int q = 0; q < 128; ++q)
+            if (q < qn) red_add_f32(acc + static_cast<size_t>(q) * D, __uint_as_float(v[q]));
+        } else {
           const bool leader = warp == 8 && lane == 0;
           uint32_t v[D];
-          if constexpr (D == 128) tmem_ld64x2(tmem + lane_off + Lay::kColDQ, v);
-          else tmem_ld64(tmem + lane_off + Lay::kColDQ, v);
+          if constexpr (D == 128) tmem_ld64x2(tmem + lane_off + Lay::kColB, v);
+          else tmem_ld64(tmem + lane_off + Lay::kColB, v);
           if (threadIdx.x == 256) FA_TRACE_AT(it, 29);
           tc_fence_before();
           mbar_arrive(dq_empty);

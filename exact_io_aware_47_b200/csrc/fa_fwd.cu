@@ -124,10 +124,15 @@ struct FwdLayout {
 #define FA_FWD_POLY_EVERY 0
 #endif
 constexpr int kFwdPolyEvery = FA_FWD_POLY_EVERY;
-#ifndef FA_FWD_ST_CHUNKS
-#define FA_FWD_ST_CHUNKS 1
+// P of a key tile is handed to the tensor core in this many parts (keys
+// 128 / parts each): part q is stored and signalled while the exponentials
+// of part q + 1 are computed, and P V runs part by part, so only the last
+// part's share of P V lies between the end of the softmax and the next S.
+#ifndef FA_FWD_P_PARTS
+#define FA_FWD_P_PARTS 1
 #endif
-constexpr int kFwdStoreChunks = FA_FWD_ST_CHUNKS;
+constexpr int kPParts = FA_FWD_P_PARTS;
+static_assert(kPParts == 1 || kPParts == 2 || kPParts == 4, "P parts");
 constexpr int kFwdLaunchRegs = 168;
 constexpr int kFwdSoftmaxRegs = 184;
 constexpr int kFwdOtherRegs = 136;
@@ -211,8 +216,8 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* kv_full = bars + 4;         // [kSlots]
   uint64_t* kv_empty = kv_full + kSlots;
   uint64_t* s_full = kv_empty + kSlots; // [2]
-  uint64_t* p_full = s_full + 2;        // [2]
-  uint64_t* o_full = p_full + 2;        // [2]
+  uint64_t* p_full = s_full + 2;        // [2][kPParts]: part q of P_t written
+  uint64_t* o_full = p_full + 2 * kPParts;  // [2]
   uint64_t* drain = o_full + 2;         // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -226,7 +231,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&q_full[t], 1);
       mbar_init(&q_empty[t], 1);
       mbar_init(&s_full[t], 1);
-      mbar_init(&p_full[t], 128);
+      for (int q = 0; q < kPParts; ++q) mbar_init(&p_full[t * kPParts + q], 128);
       mbar_init(&o_full[t], 1);
     }
     for (int s = 0; s < kSlots; ++s) {
@@ -355,6 +360,23 @@ __global__ void __launch_bounds__(384, 1)
           umma_ts_group8<true, false>(tmem + Lay::kColO + t * D, tmem + t * 128,
                                       lKV_m + vslot * kTileLo, kIdescPV, acc ? 1u : 0u);
       };
+      // Part q of O_t += P_t V: the K steps of keys [128 q / parts, 128 (q + 1)
+      // / parts); P_t's columns for them sit 8 per step (16-bit) or 8 per
+      // step of 32 keys (e4m3) after the tile's first column.
+      auto issue_pv_part = [&](int t, int vslot, int q, bool acc) {
+        if constexpr (kPParts == 1) {
+          issue_pv(t, vslot, acc);
+        } else {
+          constexpr int kSteps = (FP8 ? 4 : 8) / kPParts;
+#pragma unroll
+          for (int u = 0; u < kSteps; ++u) {
+            const int kk = q * kSteps + u;
+            const uint32_t b = lKV_m + vslot * kTileLo + (FP8 ? sw128_step8(true, kk) : sw128_step(true, kk));
+            umma_ts_one<FP8>(tmem + Lay::kColO + t * D, tmem + t * 128 + kk * 8, b, kIdescPV,
+                             (acc || u > 0) ? 1u : 0u);
+          }
+        }
+      };
 
       for (int k = 0; ok; ++k) {
         WorkItem wi;
@@ -401,12 +423,16 @@ __global__ void __launch_bounds__(384, 1)
           bool k_ready = false;
           for (int t = 0; t < 2 && ok; ++t) {
             if (fwd_need<SPARSE>(p, w, t, j)) {
-              ok = mbar_wait(&p_full[t], pcnt[t] & 1, wc, 6);
+#pragma unroll
+              for (int q = 0; q < kPParts; ++q) {
+                ok = mbar_wait(&p_full[t * kPParts + q], pcnt[t] & 1, wc, 6);
+                if (!ok) break;
+                tc_fence_after();
+                issue_pv_part(t, vslot, q, npv[t] > 0 || q > 0);
+              }
               if (!ok) break;
               FA_TRACE_AT(pcnt[t], t);
               ++pcnt[t];
-              tc_fence_after();
-              issue_pv(t, vslot, npv[t] > 0);
               ++npv[t];
               if (j == jl[t]) umma_commit(&o_full[t]);
             }
@@ -531,25 +557,46 @@ __global__ void __launch_bounds__(384, 1)
           for (int i = 0; i < 128; ++i)
             if (kbase + i >= lim) sr[i] = __float_as_uint(-INFINITY);
         }
-        // row max of the raw scores: four independent 3-input max chains,
-        // chain q4 takes elements 8k + 2 q4 and 8k + 2 q4 + 1
-        float mc[4];
+        // row max of the raw scores as a tree of 3-input maxima (depth 5, so
+        // the max instruction's latency is paid 5 times, not once per element)
+        float mx;
+        {
+          float t1[43];
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
-          mc[q4] = fmaxf(__uint_as_float(sr[2 * q4]), __uint_as_float(sr[2 * q4 + 1]));
+          for (int u = 0; u < 42; ++u)
+            t1[u] = fmax3(__uint_as_float(sr[3 * u]), __uint_as_float(sr[3 * u + 1]),
+                          __uint_as_float(sr[3 * u + 2]));
+          t1[42] = fmaxf(__uint_as_float(sr[126]), __uint_as_float(sr[127]));
+          float t2[15];
 #pragma unroll
-        for (int i = 8; i < 128; i += 8) {
+          for (int u = 0; u < 14; ++u) t2[u] = fmax3(t1[3 * u], t1[3 * u + 1], t1[3 * u + 2]);
+          t2[14] = t1[42];
+          float t3[5];
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4)
-            mc[q4] = fmax3(mc[q4], __uint_as_float(sr[i + 2 * q4]), __uint_as_float(sr[i + 2 * q4 + 1]));
+          for (int u = 0; u < 5; ++u) t3[u] = fmax3(t2[3 * u], t2[3 * u + 1], t2[3 * u + 2]);
+          mx = fmaxf(fmax3(t3[0], t3[1], t3[2]), fmaxf(t3[3], t3[4])) * cj;  // log2 units (cj > 0)
         }
-        const float mx = fmax3(mc[0], mc[1], fmaxf(mc[2], mc[3])) * cj;  // log2 units (cj > 0)
         const float m_new = (mx > m + kRescaleThreshold) ? mx : m;
         const bool moved = m_new != m;
         if (r == 0 && t == 0) FA_TRACE_AT(scnt - 1, 7);
         const float alpha = moved ? ex2_approx(m - m_new) : 1.f;  // 0 when m was -inf
         l *= alpha;
         m = m_new;
+        // O_t holds the sum up to the previous key tile (its MMA completed
+        // before S_t(j) was committed) and no part of PV_t(j) is issued
+        // before the first part of P is signalled: when a row's max moved,
+        // rescale O_t before that signal; rows that did not move multiply by 1
+        const bool rescale = jj > 0 && __any_sync(0xffffffffu, moved);
+        auto rescale_o = [&]() {
+#pragma unroll 1
+          for (int cc = 0; cc < D / 16; ++cc) {
+            uint32_t ro[16];
+            tmem_ld16(tO + cc * 16, ro);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) ro[e] = __float_as_uint(__uint_as_float(ro[e]) * alpha);
+            tmem_st_n<16>(tO + cc * 16, ro);
+          }
+        };
         // p = 2^(c s - m): packed FMA on pairs, then ex2; row sum in fp32 over
         // four packed accumulators
         const float mu = (m == -INFINITY) ? 0.f : m;
@@ -580,12 +627,22 @@ __global__ void __launch_bounds__(384, 1)
             pk[i >> 1] = (i & 1) ? (pk[i >> 1] | (h << 16)) : h;
           } else {
             pk[i] = pack2<BF16>(p0, p1);
-            if (r == 0 && t == 0 && (i & 15) == 15) FA_TRACE_AT(scnt - 1, 8 + (i >> 4));
-            // P goes back to TMEM in chunks as it is made, so the stores
-            // overlap the rest of the loop
-            if constexpr (kFwdStoreChunks > 1) {
-              constexpr int kC = 64 / kFwdStoreChunks;
-              if ((i % kC) == kC - 1) tmem_st_n<kC>(tS + (i + 1 - kC), pk + (i + 1 - kC));
+          }
+          if (r == 0 && t == 0 && (i & 15) == 15) FA_TRACE_AT(scnt - 1, 8 + (i >> 4));
+          if constexpr (kPParts > 1) {
+            // part q of P is complete: signal part q - 1 (its store has had
+            // this part's exponentials to finish), then store part q
+            constexpr int kPairs = 64 / kPParts;           // score pairs per part
+            constexpr int kCols = FP8 ? kPairs / 2 : kPairs;  // TMEM columns per part
+            if ((i % kPairs) == kPairs - 1) {
+              const int q = i / kPairs;
+              if (q == 1 && rescale) rescale_o();
+              if (q > 0) {
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(&p_full[t * kPParts + q - 1]);
+              }
+              tmem_st_n<kCols>(tS + q * kCols, pk + q * kCols);
             }
           }
         }
@@ -597,27 +654,16 @@ __global__ void __launch_bounds__(384, 1)
           f2unpack(acc[3], d0, d1);
           l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
         }
-        if constexpr (FP8) tmem_st32(tS, pk);
-        else if (kFwdStoreChunks == 1) tmem_st64(tS, pk);
-        if (r == 0 && t == 0) FA_TRACE_AT(scnt - 1, 12);
-        if (jj > 0 && __any_sync(0xffffffffu, moved)) {
-          // O_t holds the sum up to the previous key tile (its MMA completed
-          // before S_t(j) was committed) and PV_t(j) waits for p_full:
-          // rescale it now; rows that did not move multiply by 1.
-          uint32_t ro[32];
-#pragma unroll
-          for (int cc = 0; cc < D / 32; ++cc) {
-            tmem_ld32(tO + cc * 32, ro);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) ro[i] = __float_as_uint(__uint_as_float(ro[i]) * alpha);
-            tmem_st32(tO + cc * 32, ro);
-          }
+        if constexpr (kPParts == 1) {
+          if constexpr (FP8) tmem_st32(tS, pk);
+          else tmem_st64(tS, pk);
+          if (rescale) rescale_o();
         }
-        if (r == 0 && t == 0) FA_TRACE_AT(scnt - 1, 13);
+        if (r == 0 && t == 0) FA_TRACE_AT(scnt - 1, 12);
         tmem_st_wait();
         if (r == 0 && t == 0) FA_TRACE_AT(scnt - 1, 14);
         tc_fence_before();
-        mbar_arrive(&p_full[t]);
+        mbar_arrive(&p_full[t * kPParts + kPParts - 1]);
         if (r == 0) FA_TRACE_AT(scnt - 1, 3 + 2 * t);
         ++jj;
       }

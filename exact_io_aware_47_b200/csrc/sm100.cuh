@@ -431,6 +431,28 @@ __device__ __forceinline__ void umma_ts_group4_e4m3(uint32_t d_tmem, uint32_t a_
                "n"(sw128_step8(true, 1)), "n"(sw128_step8(true, 2)), "n"(sw128_step8(true, 3))
                : "memory");
 }
+// One tcgen05.mma with A in TMEM and B in shared memory (low descriptor
+// word b_lo), kind::f16 or kind::f8f6f4.
+template <bool F8>
+__device__ __forceinline__ void umma_ts_one(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
+                                            uint32_t idesc, uint32_t accumulate) {
+  if constexpr (F8) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "mov.b64 db, {%2, %5};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], db, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(accumulate), "n"(kSdescHi)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "mov.b64 db, {%2, %5};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(accumulate), "n"(kSdescHi)
+        : "memory");
+  }
+}
+
 #undef FA_MMA8_SS_FIRST
 #undef FA_MMA8_SS_STEP
 #undef FA_MMA8_TS_FIRST
@@ -463,6 +485,18 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -487,12 +521,18 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 
-// N (16 or 32) consecutive columns from a register array, by pointer (the
-// caller's indices are compile-time after unrolling).
+// N (8, 16 or 32) consecutive columns from a register array, by pointer
+// (the caller's indices are compile-time after unrolling).
 template <int N>
 __device__ __forceinline__ void tmem_st_n(uint32_t taddr, const uint32_t* r) {
-  static_assert(N == 16 || N == 32, "16 or 32 columns");
-  if constexpr (N == 16) {
+  static_assert(N == 8 || N == 16 || N == 32, "8, 16 or 32 columns");
+  if constexpr (N == 8) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+        : "memory");
+  } else if constexpr (N == 16) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
         "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
@@ -708,6 +748,19 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   else return pack_f16x2(lo, hi);
 }
 
+// The two 16-bit values of a pair back to fp32 (exact).
+template <bool BF16>
+__device__ __forceinline__ void unpack2(uint32_t w, float& lo, float& hi) {
+  if constexpr (BF16) {
+    lo = __uint_as_float(w << 16);
+    hi = __uint_as_float(w & 0xFFFF0000u);
+  } else {
+    uint16_t a = static_cast<uint16_t>(w), b = static_cast<uint16_t>(w >> 16);
+    asm("cvt.f32.f16 %0, %1;" : "=f"(lo) : "h"(a));
+    asm("cvt.f32.f16 %0, %1;" : "=f"(hi) : "h"(b));
+  }
+}
+
 // Two fp32 values to two e4m3 bytes (round to nearest even, saturating to
 // +-448): lo in bits 0..7, hi in bits 8..15.
 __device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
@@ -731,6 +784,11 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
                "r"(d)
                : "memory");
+}
+
+// Relaxed fp32 add into global memory (no return value: a reduction in L2).
+__device__ __forceinline__ void red_add_f32(float* p, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
 }
 
 __device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, uint32_t c,

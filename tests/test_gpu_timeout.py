@@ -20,7 +20,7 @@ from oracle import ref_bwd_slice, ref_fwd_slice
 pytestmark = pytest.mark.gpu
 
 FWD_SITES = set(range(1, 10))      # the forward kernel's waits
-BWD_SITES = set(range(20, 37))     # the backward kernel's waits
+BWD_SITES = set(range(20, 40))     # the backward kernel's waits
 
 
 @pytest.fixture(scope="module")
