@@ -85,6 +85,14 @@ struct BwdUnit {
 #endif
 template <int D>
 constexpr bool kDqRed = FA_BWD_DQ_RED != 0 && D == 128;
+// dS^T also goes to TMEM (region B, beside P^T), so dK reads it from there
+// instead of shared memory; a build option while the two are compared (not
+// with dropout, whose unmasked P^T copy takes those columns).
+#ifndef FA_BWD_DS_TMEM
+#define FA_BWD_DS_TMEM 0
+#endif
+template <bool DROPOUT>
+constexpr bool kDsTmem = FA_BWD_DS_TMEM != 0 && !DROPOUT;
 
 // Register split: 512 threads launched at 128 registers (launch bounds 512,1);
 // the softmax warpgroups keep their P^T values between the two phases and the
@@ -92,9 +100,15 @@ constexpr bool kDqRed = FA_BWD_DQ_RED != 0 && D == 128;
 // take 144 each; the MMA/TMA/LSE warpgroup keeps 80: 2 * 144 + 144 + 80 =
 // 4 * 128.
 constexpr int kBwdLaunchRegs = 128;
-constexpr int kBwdSoftmaxRegs = 144;
-constexpr int kBwdDqRegs = 144;
+#ifndef FA_BWD_SM_REGS
+#define FA_BWD_SM_REGS 144
+#endif
+constexpr int kBwdSoftmaxRegs = FA_BWD_SM_REGS;
 constexpr int kBwdOtherRegs = 80;
+constexpr int kBwdDqRegs = 4 * kBwdLaunchRegs - 2 * kBwdSoftmaxRegs - kBwdOtherRegs;
+// With fewer than 144 registers the dQ warps read dQ_i in two halves of
+// d / 2 columns (staging the first half before reading the second).
+constexpr bool kDqHalves = kBwdDqRegs < 144;
 static_assert(2 * kBwdSoftmaxRegs + kBwdDqRegs + kBwdOtherRegs <= 4 * kBwdLaunchRegs,
               "register split");
 
@@ -444,6 +458,12 @@ __global__ void __launch_bounds__(512, 1)
           if (!ok) break;
           tc_fence_after();
           FA_TRACE_AT(it, 8);
+          if constexpr (kDsTmem<DROPOUT>) {
+            // dK_j += dS^T Q_i with dS^T from region B; issued before dQ, which
+            // overwrites region B
+            umma_ts_group8<true, true>(tmem + Lay::kColDK, tmem + Lay::kColB + 32,
+                                       (it & 1) ? lQ1_m : lQ0_m, kIdTS, idx > 0 ? 1u : 0u);
+          }
           if constexpr (kDqRed<D>) {
             // dQ^T = K_j^T dS^T into region B (a TMEM lane per d index): A =
             // K_j read MN-major (d contiguous), B = dS^T read MN-major
@@ -456,8 +476,9 @@ __global__ void __launch_bounds__(512, 1)
           }
           umma_commit(dq_full);
           // dK_j += dS^T Q_i: A = dS^T K-major, B = Q_i MN-major
-          umma_ss_group<8, false, true>(tmem + Lay::kColDK, lS_k, (it & 1) ? lQ1_m : lQ0_m, kIdTS,
-                                        idx > 0 ? 1u : 0u);
+          if constexpr (!kDsTmem<DROPOUT>)
+            umma_ss_group<8, false, true>(tmem + Lay::kColDK, lS_k, (it & 1) ? lQ1_m : lQ0_m,
+                                          kIdTS, idx > 0 ? 1u : 0u);
           umma_commit(&slot_empty[it & 1]);  // Q_i: S and dK done
           umma_commit(ds_empty);             // dK and dQ have read dS^T
           FA_TRACE_AT(it, 3);
@@ -661,8 +682,11 @@ __global__ void __launch_bounds__(512, 1)
               st_shared_v4(ds_row + unit * 16, dd[4 * w4], dd[4 * w4 + 1], dd[4 * w4 + 2],
                            dd[4 * w4 + 3]);
             }
+            // and to region B beside P^T, for the dK product
+            if constexpr (kDsTmem<DROPOUT>) tmem_st_n<16>(tB + 64 * half + 32 + 16 * (e >> 5), dd);
           }
         }
+        if constexpr (kDsTmem<DROPOUT>) tmem_st_wait();
         if (threadIdx.x == FA_TRACE_SM_THREAD) FA_TRACE_AT(it, 22);
         fence_proxy_async_smem();
         tc_fence_before();
@@ -673,7 +697,7 @@ __global__ void __launch_bounds__(512, 1)
       }
     }
   } else {
-    regs_increase<kBwdDqRegs>();
+    regs_set<kBwdDqRegs, kBwdLaunchRegs>();
     // --------------------------- dQ read-out and reduce-add; dK_j, dV_j epilogue
     const int r = ((warp & 3) << 5) | lane;  // TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -721,14 +745,26 @@ __global__ void __launch_bounds__(512, 1)
             if (q < qn) red_add_f32(acc + static_cast<size_t>(q) * D, __uint_as_float(v[q]));
         } else {
           const bool leader = warp == 8 && lane == 0;
-          uint32_t v[D];
-          if constexpr (D == 128) tmem_ld64x2(tmem + lane_off + Lay::kColB, v);
+          constexpr int kV = (kDqHalves && D == 128) ? 64 : D;  // columns held at a time
+          uint32_t v[kV];
+          if constexpr (kV == 128) tmem_ld64x2(tmem + lane_off + Lay::kColB, v);
           else tmem_ld64(tmem + lane_off + Lay::kColB, v);
-          if (threadIdx.x == 256) FA_TRACE_AT(it, 29);
-          tc_fence_before();
-          mbar_arrive(dq_empty);
+          if constexpr (kV == D) {
+            if (threadIdx.x == 256) FA_TRACE_AT(it, 29);
+            tc_fence_before();
+            mbar_arrive(dq_empty);
+          }
 #pragma unroll
           for (int rd = 0; rd < D / 32; ++rd) {
+            if constexpr (kV < D) {
+              if (rd == kV / 32) {
+                // second half: read it, then release the TMEM columns
+                tmem_ld64(tmem + lane_off + Lay::kColB + kV, v);
+                if (threadIdx.x == 256) FA_TRACE_AT(it, 29);
+                tc_fence_before();
+                mbar_arrive(dq_empty);
+              }
+            }
             uint8_t* stg = sSTG + (stage_round & 1) * 16384;
             if (stage_round >= 2) {
               // the transfer that used this buffer two rounds ago must have
@@ -739,8 +775,9 @@ __global__ void __launch_bounds__(512, 1)
             const uint32_t row = smem_addr(stg) + r * 128;
 #pragma unroll
             for (int u = 0; u < 8; ++u)
-              st_shared_v4(row + ((u ^ (r & 7)) << 4), v[rd * 32 + 4 * u], v[rd * 32 + 4 * u + 1],
-                           v[rd * 32 + 4 * u + 2], v[rd * 32 + 4 * u + 3]);
+              st_shared_v4(row + ((u ^ (r & 7)) << 4), v[(rd * 32) % kV + 4 * u],
+                           v[(rd * 32) % kV + 4 * u + 1], v[(rd * 32) % kV + 4 * u + 2],
+                           v[(rd * 32) % kV + 4 * u + 3]);
             fence_proxy_async_smem();
             named_bar_sync(1, 128);
             if (leader) {

@@ -134,8 +134,11 @@ constexpr int kFwdPolyEvery = FA_FWD_POLY_EVERY;
 constexpr int kPParts = FA_FWD_P_PARTS;
 static_assert(kPParts == 1 || kPParts == 2 || kPParts == 4, "P parts");
 constexpr int kFwdLaunchRegs = 168;
-constexpr int kFwdSoftmaxRegs = 184;
-constexpr int kFwdOtherRegs = 136;
+#ifndef FA_FWD_SM_REGS
+#define FA_FWD_SM_REGS 184
+#endif
+constexpr int kFwdSoftmaxRegs = FA_FWD_SM_REGS;
+constexpr int kFwdOtherRegs = 3 * kFwdLaunchRegs - 2 * kFwdSoftmaxRegs;
 static_assert(2 * kFwdSoftmaxRegs + kFwdOtherRegs <= 3 * kFwdLaunchRegs, "register split");
 
 struct FwdUnit {
@@ -557,25 +560,19 @@ __global__ void __launch_bounds__(384, 1)
           for (int i = 0; i < 128; ++i)
             if (kbase + i >= lim) sr[i] = __float_as_uint(-INFINITY);
         }
-        // row max of the raw scores as a tree of 3-input maxima (depth 5, so
-        // the max instruction's latency is paid 5 times, not once per element)
-        float mx;
-        {
-          float t1[43];
+        // row max of the raw scores: four independent 3-input max chains,
+        // chain q4 takes elements 8k + 2 q4 and 8k + 2 q4 + 1
+        float mc[4];
 #pragma unroll
-          for (int u = 0; u < 42; ++u)
-            t1[u] = fmax3(__uint_as_float(sr[3 * u]), __uint_as_float(sr[3 * u + 1]),
-                          __uint_as_float(sr[3 * u + 2]));
-          t1[42] = fmaxf(__uint_as_float(sr[126]), __uint_as_float(sr[127]));
-          float t2[15];
+        for (int q4 = 0; q4 < 4; ++q4)
+          mc[q4] = fmaxf(__uint_as_float(sr[2 * q4]), __uint_as_float(sr[2 * q4 + 1]));
 #pragma unroll
-          for (int u = 0; u < 14; ++u) t2[u] = fmax3(t1[3 * u], t1[3 * u + 1], t1[3 * u + 2]);
-          t2[14] = t1[42];
-          float t3[5];
+        for (int i = 8; i < 128; i += 8) {
 #pragma unroll
-          for (int u = 0; u < 5; ++u) t3[u] = fmax3(t2[3 * u], t2[3 * u + 1], t2[3 * u + 2]);
-          mx = fmaxf(fmax3(t3[0], t3[1], t3[2]), fmaxf(t3[3], t3[4])) * cj;  // log2 units (cj > 0)
+          for (int q4 = 0; q4 < 4; ++q4)
+            mc[q4] = fmax3(mc[q4], __uint_as_float(sr[i + 2 * q4]), __uint_as_float(sr[i + 2 * q4 + 1]));
         }
+        const float mx = fmax3(mc[0], mc[1], fmaxf(mc[2], mc[3])) * cj;  // log2 units (cj > 0)
         const float m_new = (mx > m + kRescaleThreshold) ? mx : m;
         const bool moved = m_new != m;
         if (r == 0 && t == 0) FA_TRACE_AT(scnt - 1, 7);

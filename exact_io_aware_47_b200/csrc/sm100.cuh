@@ -90,7 +90,15 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
-#ifdef FA_WAIT_HINT_NS
+#if defined(FA_WAIT_SPIN)
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+#elif defined(FA_WAIT_HINT_NS)
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
@@ -245,6 +253,12 @@ __device__ __forceinline__ void regs_increase() {
 template <int N>
 __device__ __forceinline__ void regs_decrease() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+// A warpgroup's share moved from the launch allocation L to N (either way).
+template <int N, int L>
+__device__ __forceinline__ void regs_set() {
+  if constexpr (N > L) regs_increase<N>();
+  else if constexpr (N < L) regs_decrease<N>();
 }
 
 __device__ __forceinline__ void tc_fence_before() {
