@@ -77,38 +77,15 @@ struct BwdUnit {
   bool skip;          // packed key tile past its sequence: no role does anything
 };
 
-// dQ_i leaves the SM by per-thread fp32 reduce-adds from registers (d = 128,
-// dQ computed transposed) instead of a shared-memory staging tile and TMA
-// reduce-adds; a build option while the two are compared.
-#ifndef FA_BWD_DQ_RED
-#define FA_BWD_DQ_RED 0
-#endif
-template <int D>
-constexpr bool kDqRed = FA_BWD_DQ_RED != 0 && D == 128;
-// dS^T also goes to TMEM (region B, beside P^T), so dK reads it from there
-// instead of shared memory; a build option while the two are compared (not
-// with dropout, whose unmasked P^T copy takes those columns).
-#ifndef FA_BWD_DS_TMEM
-#define FA_BWD_DS_TMEM 0
-#endif
-template <bool DROPOUT>
-constexpr bool kDsTmem = FA_BWD_DS_TMEM != 0 && !DROPOUT;
-
 // Register split: 512 threads launched at 128 registers (launch bounds 512,1);
 // the softmax warpgroups keep their P^T values between the two phases and the
 // dQ warpgroup holds a whole dQ^T row (128 fp32) before staging it, so they
 // take 144 each; the MMA/TMA/LSE warpgroup keeps 80: 2 * 144 + 144 + 80 =
 // 4 * 128.
 constexpr int kBwdLaunchRegs = 128;
-#ifndef FA_BWD_SM_REGS
-#define FA_BWD_SM_REGS 144
-#endif
-constexpr int kBwdSoftmaxRegs = FA_BWD_SM_REGS;
+constexpr int kBwdSoftmaxRegs = 144;
+constexpr int kBwdDqRegs = 144;
 constexpr int kBwdOtherRegs = 80;
-constexpr int kBwdDqRegs = 4 * kBwdLaunchRegs - 2 * kBwdSoftmaxRegs - kBwdOtherRegs;
-// With fewer than 144 registers the dQ warps read dQ_i in two halves of
-// d / 2 columns (staging the first half before reading the second).
-constexpr bool kDqHalves = kBwdDqRegs < 144;
 static_assert(2 * kBwdSoftmaxRegs + kBwdDqRegs + kBwdOtherRegs <= 4 * kBwdLaunchRegs,
               "register split");
 
@@ -193,8 +170,9 @@ __global__ void __launch_bounds__(512, 1)
                   const __grid_constant__ CUtensorMap tmdq, const BwdParams p) {
   using Lay = BwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned base, derived from smem_raw by pointer arithmetic so
+  // that the compiler keeps every derived pointer in the shared space
+  uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   if (smem + Lay::kUsed > smem_raw + Lay::kSmemBytes) {
     // the dynamic shared-memory window is not aligned well enough: refuse
     if (threadIdx.x == 0) record_error(kErrDeviceLayout, 0);
@@ -372,8 +350,6 @@ __global__ void __launch_bounds__(512, 1)
       constexpr uint32_t kIdTS = idesc_f16(BF16, 128, D, false, true);    // dV, dK (B MN-major)
       // dQ = dS K_j (M = queries, N = d): a TMEM lane holds one query row
       constexpr uint32_t kIdDQ = idesc_f16(BF16, 128, D, true, true);
-      // dQ^T = K_j^T dS^T (M = d, N = queries): a TMEM lane holds one d index
-      constexpr uint32_t kIdDQT = idesc_f16(BF16, 128, 128, true, true);
       // Low descriptor words of every operand tile, K-major (_k) or MN-major
       // (_m) view; the grouped MMAs derive the K steps from them.
       const uint32_t aSlot = smem_addr(sSlot);
@@ -458,27 +434,13 @@ __global__ void __launch_bounds__(512, 1)
           if (!ok) break;
           tc_fence_after();
           FA_TRACE_AT(it, 8);
-          if constexpr (kDsTmem<DROPOUT>) {
-            // dK_j += dS^T Q_i with dS^T from region B; issued before dQ, which
-            // overwrites region B
-            umma_ts_group8<true, true>(tmem + Lay::kColDK, tmem + Lay::kColB + 32,
-                                       (it & 1) ? lQ1_m : lQ0_m, kIdTS, idx > 0 ? 1u : 0u);
-          }
-          if constexpr (kDqRed<D>) {
-            // dQ^T = K_j^T dS^T into region B (a TMEM lane per d index): A =
-            // K_j read MN-major (d contiguous), B = dS^T read MN-major
-            // (queries contiguous)
-            umma_ss_group<8, true, true>(tmem + Lay::kColB, lK_m, lS_m, kIdDQT, 0u);
-          } else {
-            // dQ = dS K_j into region B: A = dS^T read MN-major (queries
-            // contiguous), B = K_j read MN-major (d contiguous)
-            umma_ss_group<8, true, true>(tmem + Lay::kColB, lS_m, lK_m, kIdDQ, 0u);
-          }
+          // dQ = dS K_j into region B: A = dS^T read MN-major (queries
+          // contiguous), B = K_j read MN-major (d contiguous)
+          umma_ss_group<8, true, true>(tmem + Lay::kColB, lS_m, lK_m, kIdDQ, 0u);
           umma_commit(dq_full);
           // dK_j += dS^T Q_i: A = dS^T K-major, B = Q_i MN-major
-          if constexpr (!kDsTmem<DROPOUT>)
-            umma_ss_group<8, false, true>(tmem + Lay::kColDK, lS_k, (it & 1) ? lQ1_m : lQ0_m,
-                                          kIdTS, idx > 0 ? 1u : 0u);
+          umma_ss_group<8, false, true>(tmem + Lay::kColDK, lS_k, (it & 1) ? lQ1_m : lQ0_m, kIdTS,
+                                        idx > 0 ? 1u : 0u);
           umma_commit(&slot_empty[it & 1]);  // Q_i: S and dK done
           umma_commit(ds_empty);             // dK and dQ have read dS^T
           FA_TRACE_AT(it, 3);
@@ -673,6 +635,7 @@ __global__ void __launch_bounds__(512, 1)
           f2unpack(fmul2(f2pack(pf[2], pf[3]), x23), gv[2], gv[3]);
           dd[(e & 31) >> 1] = pack2<BF16>(gv[0], gv[1]);
           dd[((e & 31) >> 1) + 1] = pack2<BF16>(gv[2], gv[3]);
+          if (threadIdx.x == FA_TRACE_SM_THREAD && (e & 15) == 12) FA_TRACE_AT(it, 24 + (e >> 4));
           if ((e & 31) == 28) {
             // 32 queries done: four 16-byte units of the 128-byte swizzled row
             // (units 4 cc .. 4 cc + 3 of panel `half`, cc = e / 32)
@@ -682,11 +645,8 @@ __global__ void __launch_bounds__(512, 1)
               st_shared_v4(ds_row + unit * 16, dd[4 * w4], dd[4 * w4 + 1], dd[4 * w4 + 2],
                            dd[4 * w4 + 3]);
             }
-            // and to region B beside P^T, for the dK product
-            if constexpr (kDsTmem<DROPOUT>) tmem_st_n<16>(tB + 64 * half + 32 + 16 * (e >> 5), dd);
           }
         }
-        if constexpr (kDsTmem<DROPOUT>) tmem_st_wait();
         if (threadIdx.x == FA_TRACE_SM_THREAD) FA_TRACE_AT(it, 22);
         fence_proxy_async_smem();
         tc_fence_before();
@@ -697,7 +657,7 @@ __global__ void __launch_bounds__(512, 1)
       }
     }
   } else {
-    regs_set<kBwdDqRegs, kBwdLaunchRegs>();
+    regs_increase<kBwdDqRegs>();
     // --------------------------- dQ read-out and reduce-add; dK_j, dV_j epilogue
     const int r = ((warp & 3) << 5) | lane;  // TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -727,44 +687,16 @@ __global__ void __launch_bounds__(512, 1)
         // transfer (the TMA path sustains more reduce bandwidth per SM than
         // per-thread reds); staging a round overlaps the previous transfer.
         // Rows past N are clipped by the transfer.
-        if constexpr (kDqRed<D>) {
-          // Lane r holds d index r of dQ_i^T for the tile's 128 queries: read
-          // them, release the TMEM columns, and add them into the fp32
-          // accumulator from registers; the 32 lanes of a warp cover 32
-          // consecutive d of one query row, so every reduce of a warp is one
-          // 128-byte line.  Rows past the slice's computed rows are skipped.
-          uint32_t v[128];
-          tmem_ld64x2(tmem + lane_off + Lay::kColB, v);
+        {
+          const bool leader = warp == 8 && lane == 0;
+          uint32_t v[D];
+          if constexpr (D == 128) tmem_ld64x2(tmem + lane_off + Lay::kColB, v);
+          else tmem_ld64(tmem + lane_off + Lay::kColB, v);
           if (threadIdx.x == 256) FA_TRACE_AT(it, 29);
           tc_fence_before();
           mbar_arrive(dq_empty);
-          const int qn = min(kBlockM, w.rows - i * kBlockM);
-          float* acc = p.dq_acc + (base + static_cast<size_t>(i) * kBlockM) * D + r;
-#pragma unroll
-          for (int q = 0; q < 128; ++q)
-            if (q < qn) red_add_f32(acc + static_cast<size_t>(q) * D, __uint_as_float(v[q]));
-        } else {
-          const bool leader = warp == 8 && lane == 0;
-          constexpr int kV = (kDqHalves && D == 128) ? 64 : D;  // columns held at a time
-          uint32_t v[kV];
-          if constexpr (kV == 128) tmem_ld64x2(tmem + lane_off + Lay::kColB, v);
-          else tmem_ld64(tmem + lane_off + Lay::kColB, v);
-          if constexpr (kV == D) {
-            if (threadIdx.x == 256) FA_TRACE_AT(it, 29);
-            tc_fence_before();
-            mbar_arrive(dq_empty);
-          }
 #pragma unroll
           for (int rd = 0; rd < D / 32; ++rd) {
-            if constexpr (kV < D) {
-              if (rd == kV / 32) {
-                // second half: read it, then release the TMEM columns
-                tmem_ld64(tmem + lane_off + Lay::kColB + kV, v);
-                if (threadIdx.x == 256) FA_TRACE_AT(it, 29);
-                tc_fence_before();
-                mbar_arrive(dq_empty);
-              }
-            }
             uint8_t* stg = sSTG + (stage_round & 1) * 16384;
             if (stage_round >= 2) {
               // the transfer that used this buffer two rounds ago must have
@@ -775,9 +707,8 @@ __global__ void __launch_bounds__(512, 1)
             const uint32_t row = smem_addr(stg) + r * 128;
 #pragma unroll
             for (int u = 0; u < 8; ++u)
-              st_shared_v4(row + ((u ^ (r & 7)) << 4), v[(rd * 32) % kV + 4 * u],
-                           v[(rd * 32) % kV + 4 * u + 1], v[(rd * 32) % kV + 4 * u + 2],
-                           v[(rd * 32) % kV + 4 * u + 3]);
+              st_shared_v4(row + ((u ^ (r & 7)) << 4), v[rd * 32 + 4 * u], v[rd * 32 + 4 * u + 1],
+                           v[rd * 32 + 4 * u + 2], v[rd * 32 + 4 * u + 3]);
             fence_proxy_async_smem();
             named_bar_sync(1, 128);
             if (leader) {

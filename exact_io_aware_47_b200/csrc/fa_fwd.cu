@@ -120,25 +120,9 @@ struct FwdLayout {
 // Register split: 384 threads launched at 168 registers (launch bounds 384,1);
 // the two softmax warpgroups take 184, the MMA/TMA warpgroup keeps 136:
 // 2 * 184 + 136 = 3 * 168 (no spills at this split).
-#ifndef FA_FWD_POLY_EVERY
-#define FA_FWD_POLY_EVERY 0
-#endif
-constexpr int kFwdPolyEvery = FA_FWD_POLY_EVERY;
-// P of a key tile is handed to the tensor core in this many parts (keys
-// 128 / parts each): part q is stored and signalled while the exponentials
-// of part q + 1 are computed, and P V runs part by part, so only the last
-// part's share of P V lies between the end of the softmax and the next S.
-#ifndef FA_FWD_P_PARTS
-#define FA_FWD_P_PARTS 1
-#endif
-constexpr int kPParts = FA_FWD_P_PARTS;
-static_assert(kPParts == 1 || kPParts == 2 || kPParts == 4, "P parts");
 constexpr int kFwdLaunchRegs = 168;
-#ifndef FA_FWD_SM_REGS
-#define FA_FWD_SM_REGS 184
-#endif
-constexpr int kFwdSoftmaxRegs = FA_FWD_SM_REGS;
-constexpr int kFwdOtherRegs = 3 * kFwdLaunchRegs - 2 * kFwdSoftmaxRegs;
+constexpr int kFwdSoftmaxRegs = 184;
+constexpr int kFwdOtherRegs = 136;
 static_assert(2 * kFwdSoftmaxRegs + kFwdOtherRegs <= 3 * kFwdLaunchRegs, "register split");
 
 struct FwdUnit {
@@ -209,8 +193,9 @@ __global__ void __launch_bounds__(384, 1)
   static_assert(!FP8 || (D == 128 && !PACKED && !SPARSE && !DROPOUT), "e4m3: dense, d = 128");
   constexpr int kSlots = Lay::kSlots;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // 1024-byte aligned base, derived from smem_raw by pointer arithmetic so
+  // that the compiler keeps every derived pointer in the shared space
+  uint8_t* smem = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   uint8_t* sq = smem + Lay::kQ0;        // Q0, Q1 tiles
   uint8_t* skv = smem + Lay::kSlot0;    // K/V ring
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
@@ -219,8 +204,8 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* kv_full = bars + 4;         // [kSlots]
   uint64_t* kv_empty = kv_full + kSlots;
   uint64_t* s_full = kv_empty + kSlots; // [2]
-  uint64_t* p_full = s_full + 2;        // [2][kPParts]: part q of P_t written
-  uint64_t* o_full = p_full + 2 * kPParts;  // [2]
+  uint64_t* p_full = s_full + 2;        // [2]
+  uint64_t* o_full = p_full + 2;        // [2]
   uint64_t* drain = o_full + 2;         // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -234,7 +219,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&q_full[t], 1);
       mbar_init(&q_empty[t], 1);
       mbar_init(&s_full[t], 1);
-      for (int q = 0; q < kPParts; ++q) mbar_init(&p_full[t * kPParts + q], 128);
+      mbar_init(&p_full[t], 128);
       mbar_init(&o_full[t], 1);
     }
     for (int s = 0; s < kSlots; ++s) {
@@ -363,24 +348,6 @@ __global__ void __launch_bounds__(384, 1)
           umma_ts_group8<true, false>(tmem + Lay::kColO + t * D, tmem + t * 128,
                                       lKV_m + vslot * kTileLo, kIdescPV, acc ? 1u : 0u);
       };
-      // Part q of O_t += P_t V: the K steps of keys [128 q / parts, 128 (q + 1)
-      // / parts); P_t's columns for them sit 8 per step (16-bit) or 8 per
-      // step of 32 keys (e4m3) after the tile's first column.
-      auto issue_pv_part = [&](int t, int vslot, int q, bool acc) {
-        if constexpr (kPParts == 1) {
-          issue_pv(t, vslot, acc);
-        } else {
-          constexpr int kSteps = (FP8 ? 4 : 8) / kPParts;
-#pragma unroll
-          for (int u = 0; u < kSteps; ++u) {
-            const int kk = q * kSteps + u;
-            const uint32_t b = lKV_m + vslot * kTileLo + (FP8 ? sw128_step8(true, kk) : sw128_step(true, kk));
-            umma_ts_one<FP8>(tmem + Lay::kColO + t * D, tmem + t * 128 + kk * 8, b, kIdescPV,
-                             (acc || u > 0) ? 1u : 0u);
-          }
-        }
-      };
-
       for (int k = 0; ok; ++k) {
         WorkItem wi;
         if (!next_item(k, wi)) break;
@@ -426,16 +393,12 @@ __global__ void __launch_bounds__(384, 1)
           bool k_ready = false;
           for (int t = 0; t < 2 && ok; ++t) {
             if (fwd_need<SPARSE>(p, w, t, j)) {
-#pragma unroll
-              for (int q = 0; q < kPParts; ++q) {
-                ok = mbar_wait(&p_full[t * kPParts + q], pcnt[t] & 1, wc, 6);
-                if (!ok) break;
-                tc_fence_after();
-                issue_pv_part(t, vslot, q, npv[t] > 0 || q > 0);
-              }
+              ok = mbar_wait(&p_full[t], pcnt[t] & 1, wc, 6);
               if (!ok) break;
               FA_TRACE_AT(pcnt[t], t);
               ++pcnt[t];
+              tc_fence_after();
+              issue_pv(t, vslot, npv[t] > 0);
               ++npv[t];
               if (j == jl[t]) umma_commit(&o_full[t]);
             }
@@ -580,9 +543,9 @@ __global__ void __launch_bounds__(384, 1)
         l *= alpha;
         m = m_new;
         // O_t holds the sum up to the previous key tile (its MMA completed
-        // before S_t(j) was committed) and no part of PV_t(j) is issued
-        // before the first part of P is signalled: when a row's max moved,
-        // rescale O_t before that signal; rows that did not move multiply by 1
+        // before S_t(j) was committed) and PV_t(j) waits for p_full: when a
+        // row's max moved, rescale O_t before that signal; rows that did not
+        // move multiply by 1
         const bool rescale = jj > 0 && __any_sync(0xffffffffu, moved);
         auto rescale_o = [&]() {
 #pragma unroll 1
@@ -607,11 +570,7 @@ __global__ void __launch_bounds__(384, 1)
               ffma2(f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), c2, nm2);
           float x0, x1;
           f2unpack(x2, x0, x1);
-          // every FA_FWD_POLY_EVERY-th pair on the FMA pipe, the rest on the
-          // special-function unit, which is what bounds this loop
-          const bool poly = kFwdPolyEvery > 0 && !FP8 && (i % (kFwdPolyEvery > 0 ? kFwdPolyEvery : 1)) == kFwdPolyEvery - 1;
-          const unsigned long long p2 =
-              poly ? exp2_poly2(x0, x1) : f2pack(ex2_approx(x0), ex2_approx(x1));
+          const unsigned long long p2 = f2pack(ex2_approx(x0), ex2_approx(x1));
           acc[i & 3] = fadd2(acc[i & 3], p2);
           float p0, p1;
           f2unpack(p2, p0, p1);
@@ -626,22 +585,6 @@ __global__ void __launch_bounds__(384, 1)
             pk[i] = pack2<BF16>(p0, p1);
           }
           if (r == 0 && t == 0 && (i & 15) == 15) FA_TRACE_AT(scnt - 1, 8 + (i >> 4));
-          if constexpr (kPParts > 1) {
-            // part q of P is complete: signal part q - 1 (its store has had
-            // this part's exponentials to finish), then store part q
-            constexpr int kPairs = 64 / kPParts;           // score pairs per part
-            constexpr int kCols = FP8 ? kPairs / 2 : kPairs;  // TMEM columns per part
-            if ((i % kPairs) == kPairs - 1) {
-              const int q = i / kPairs;
-              if (q == 1 && rescale) rescale_o();
-              if (q > 0) {
-                tmem_st_wait();
-                tc_fence_before();
-                mbar_arrive(&p_full[t * kPParts + q - 1]);
-              }
-              tmem_st_n<kCols>(tS + q * kCols, pk + q * kCols);
-            }
-          }
         }
         {
           float a0, a1, b0, b1, c0, c1, d0, d1;
@@ -651,16 +594,14 @@ __global__ void __launch_bounds__(384, 1)
           f2unpack(acc[3], d0, d1);
           l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
         }
-        if constexpr (kPParts == 1) {
-          if constexpr (FP8) tmem_st32(tS, pk);
-          else tmem_st64(tS, pk);
-          if (rescale) rescale_o();
-        }
+        if constexpr (FP8) tmem_st32(tS, pk);
+        else tmem_st64(tS, pk);
+        if (rescale) rescale_o();
         if (r == 0 && t == 0) FA_TRACE_AT(scnt - 1, 12);
         tmem_st_wait();
         if (r == 0 && t == 0) FA_TRACE_AT(scnt - 1, 14);
         tc_fence_before();
-        mbar_arrive(&p_full[t * kPParts + kPParts - 1]);
+        mbar_arrive(&p_full[t]);
         if (r == 0) FA_TRACE_AT(scnt - 1, 3 + 2 * t);
         ++jj;
       }

@@ -90,23 +90,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
-#if defined(FA_WAIT_SPIN)
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-#elif defined(FA_WAIT_HINT_NS)
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity), "n"(FA_WAIT_HINT_NS)
-      : "memory");
-#else
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
@@ -114,7 +97,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "=r"(ok)
       : "r"(bar), "r"(parity)
       : "memory");
-#endif
   return ok != 0;
 }
 
@@ -254,13 +236,6 @@ template <int N>
 __device__ __forceinline__ void regs_decrease() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
-// A warpgroup's share moved from the launch allocation L to N (either way).
-template <int N, int L>
-__device__ __forceinline__ void regs_set() {
-  if constexpr (N > L) regs_increase<N>();
-  else if constexpr (N < L) regs_decrease<N>();
-}
-
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -445,28 +420,6 @@ __device__ __forceinline__ void umma_ts_group4_e4m3(uint32_t d_tmem, uint32_t a_
                "n"(sw128_step8(true, 1)), "n"(sw128_step8(true, 2)), "n"(sw128_step8(true, 3))
                : "memory");
 }
-// One tcgen05.mma with A in TMEM and B in shared memory (low descriptor
-// word b_lo), kind::f16 or kind::f8f6f4.
-template <bool F8>
-__device__ __forceinline__ void umma_ts_one(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
-                                            uint32_t idesc, uint32_t accumulate) {
-  if constexpr (F8) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "mov.b64 db, {%2, %5};\n\t"
-        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], db, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(accumulate), "n"(kSdescHi)
-        : "memory");
-  } else {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "mov.b64 db, {%2, %5};\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], db, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "r"(b_lo), "r"(idesc), "r"(accumulate), "n"(kSdescHi)
-        : "memory");
-  }
-}
-
 #undef FA_MMA8_SS_FIRST
 #undef FA_MMA8_SS_STEP
 #undef FA_MMA8_TS_FIRST
@@ -718,34 +671,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-// 2^x for a pair of fp32 values on the FMA and integer pipes (no
-// special-function unit), written from the textbook method: range reduction
-// x = n + f with n = round(x) (adding 1.5 * 2^23 + 127 rounds x to an integer
-// under round-to-nearest and leaves n + 127, the biased exponent of 2^n, in
-// the low mantissa bits) and f in [-1/2, 1/2]; 2^f from a cubic
-// c0 + f (c1 + f (c2 + f c3)) whose coefficients minimise the largest
-// relative error over [-1/2, 1/2] (fitted here as a linear program over a
-// dense grid; the fp32 evaluation stays within 7.5e-5 of 2^f); then the
-// product with 2^n, built from the biased exponent.  x is clamped to >= -127,
-// where 2^n is +0, so very negative inputs give exactly 0 (as the flushing
-// ex2.approx.ftz does below 2^-126); x must stay below 127.
-__device__ __forceinline__ unsigned long long exp2_poly2(float x0, float x1) {
-  constexpr float kShift = 12583039.f;  // 1.5 * 2^23 + 127, exact in fp32
-  const unsigned long long x = f2pack(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
-  const unsigned long long t = fadd2(x, f2pack(kShift, kShift));
-  const unsigned long long n = fadd2(t, f2pack(-kShift, -kShift));        // round(x)
-  const unsigned long long f = ffma2(n, f2pack(-1.f, -1.f), x);           // x - n
-  unsigned long long p = f2pack(0.05517222f, 0.05517222f);
-  p = ffma2(p, f, f2pack(0.24261116f, 0.24261116f));
-  p = ffma2(p, f, f2pack(0.69326086f, 0.69326086f));
-  p = ffma2(p, f, f2pack(0.99992808f, 0.99992808f));
-  float t0, t1;
-  f2unpack(t, t0, t1);
-  const unsigned long long e = f2pack(__uint_as_float(__float_as_uint(t0) << 23),
-                                      __uint_as_float(__float_as_uint(t1) << 23));  // 2^n
-  return fmul2(p, e);
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -798,11 +723,6 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
                "r"(d)
                : "memory");
-}
-
-// Relaxed fp32 add into global memory (no return value: a reduction in L2).
-__device__ __forceinline__ void red_add_f32(float* p, float v) {
-  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
 }
 
 __device__ __forceinline__ void st_global_v4(void* p, uint32_t a, uint32_t b, uint32_t c,
