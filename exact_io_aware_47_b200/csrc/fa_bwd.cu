@@ -295,6 +295,7 @@ __global__ void __launch_bounds__(512, 1)
               tma_load_3d(sSlot + slot * Lay::kTileBytes + pn * Lay::kPanelBytes,
                           t == 0 ? &tmq : &tmdo, &slot_full[slot], pn * 64,
                           w.row0 + i * kBlockM, w.z);
+            FA_TRACE_AT(lt, t == 0 ? 21 : 23);
             ++issued[slot];
           }
           ++lt;
@@ -382,14 +383,15 @@ __global__ void __launch_bounds__(512, 1)
         //   dP(i) once the first softmax phase has loaded S^T(i) out of A,
         //   dV(i) once it has written P^T(i) into B,
         //   S(i+1) once the second phase has loaded dP^T(i) out of A,
-        //   dQ(i) into B (dV(i), issued before it, has read P^T(i)) and dK(i)
-        //   once dS^T(i) is in shared memory.
+        //   dK(i), then dQ(i) into B (dV(i), issued before it, has read
+        //   P^T(i)) once dS^T(i) is in shared memory.
         // No MMA waits for the exponentials of the tile it overwrites, nor for
         // the read-out of dQ (the first phase of the next tile waits for that
         // before it writes P^T into B).
         auto issue_s = [&](int t) -> bool {  // S^T(t) = K_j Q_t^T, Q_t in slot t & 1
           if (t > 0 && !mbar_wait(dp_read, (t - 1) & 1, wc, 37)) return false;
           if (!mbar_wait(&slot_full[t & 1], (t >> 1) & 1, wc, 24)) return false;
+          FA_TRACE_AT(t, 28);
           tc_fence_after();
           umma_ss_group<D / 16, false, false>(tmem + Lay::kColA, lK_k, (t & 1) ? lQ1_k : lQ0_k,
                                               kIdS, 0u);
@@ -434,14 +436,16 @@ __global__ void __launch_bounds__(512, 1)
           if (!ok) break;
           tc_fence_after();
           FA_TRACE_AT(it, 8);
+          // dK_j += dS^T Q_i: A = dS^T K-major, B = Q_i MN-major.  Issued
+          // before dQ so that Q_i's slot, the one the next-but-one query tile
+          // loads into, is released one contraction earlier.
+          umma_ss_group<8, false, true>(tmem + Lay::kColDK, lS_k, (it & 1) ? lQ1_m : lQ0_m, kIdTS,
+                                        idx > 0 ? 1u : 0u);
+          umma_commit(&slot_empty[it & 1]);  // Q_i: S and dK done
           // dQ = dS K_j into region B: A = dS^T read MN-major (queries
           // contiguous), B = K_j read MN-major (d contiguous)
           umma_ss_group<8, true, true>(tmem + Lay::kColB, lS_m, lK_m, kIdDQ, 0u);
           umma_commit(dq_full);
-          // dK_j += dS^T Q_i: A = dS^T K-major, B = Q_i MN-major
-          umma_ss_group<8, false, true>(tmem + Lay::kColDK, lS_k, (it & 1) ? lQ1_m : lQ0_m, kIdTS,
-                                        idx > 0 ? 1u : 0u);
-          umma_commit(&slot_empty[it & 1]);  // Q_i: S and dK done
           umma_commit(ds_empty);             // dK and dQ have read dS^T
           FA_TRACE_AT(it, 3);
           ++it;
@@ -512,6 +516,9 @@ __global__ void __launch_bounds__(512, 1)
     // dS^T row r, queries of this half: panel `half` of the swizzled tile
     const uint32_t ds_row = smem_addr(sDS) + half * 16384 + r * 128;
     const float cl = p.scale_log2;
+    const uint32_t u_drop = 256u - min(p.keep_t, 256u);  // dropout keep test (keep_flags4)
+    const uint32_t u_lo7 = (u_drop & 0x7Fu) * 0x01010101u, u_all = u_drop * 0x01010101u;
+    const unsigned long long inv_keep2 = f2pack(p.inv_keep, p.inv_keep);
     int it = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
@@ -525,19 +532,13 @@ __global__ void __launch_bounds__(512, 1)
       for (int idx = 0; idx < w.ni && ok; ++idx) {
         i = bwd_next_i<SPARSE>(p, w, i + 1);
         const int st = it & 1;  // LSE/D staging advances with the iteration count
-        // dropout: keep bits of this key for the half's 64 queries (bit q of
-        // drop_keep[q / 32] = query 128 i + 64 half + q), made while S^T is
-        // computed; the first phase writes only kept P^T, the second scales
-        // the kept dP^T by 256 / t
+        // dropout: keep flags of this key for the half's 64 queries
+        // (keep_flags_key64), made while S^T is computed; the first phase
+        // writes only kept P^T, the second scales the kept dP^T by 256 / t
         uint32_t drop_keep[2] = {~0u, ~0u};
-        if constexpr (DROPOUT) {
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const uint32_t m16 =
-                keep_bits_key16(p, w.bh, w.j * kBlockN + r, i * kBlockM + 64 * half + 16 * g, lane & 3);
-            drop_keep[g >> 1] = (g & 1) ? (drop_keep[g >> 1] & 0xFFFFu) | (m16 << 16) : m16;
-          }
-        }
+        if constexpr (DROPOUT)
+          keep_flags_key64(p, w.bh, w.j * kBlockN + r, i * kBlockM + 64 * half, lane & 3, u_lo7,
+                           u_all, drop_keep);
         // ---- phase 1: P^T = 2^(c S^T - LSE_i log2 e) from S^T (region A),
         // to region B as 16-bit for the dV product
         ok = mbar_wait_warp(&ld_full[st], (it >> 1) & 1, wc, 28) &&
@@ -563,20 +564,23 @@ __global__ void __launch_bounds__(512, 1)
             const int q0 = 64 * half + e;  // query inside the tile
             const float4 l4 = *reinterpret_cast<const float4*>(lse2 + q0);
             const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-            float pv[4], pd[4];
+            float pv[4];
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4) {
               const bool vis = key_ok && (q0 + k4 >= diag_lim);
               const float x = fmaf(__uint_as_float(sr[e + k4]), cl, -lv[k4]);
               pv[k4] = vis ? ex2_approx(x) : 0.f;
-              // P^T as dV sees it: dropped scores are zero
-              pd[k4] = DROPOUT && !((drop_keep[e >> 5] >> ((e & 31) + k4)) & 1u) ? 0.f : pv[k4];
             }
-            pp[e >> 1] = pack2<BF16>(pd[0], pd[1]);
-            pp[(e >> 1) + 1] = pack2<BF16>(pd[2], pd[3]);
+            pp[e >> 1] = pack2<BF16>(pv[0], pv[1]);
+            pp[(e >> 1) + 1] = pack2<BF16>(pv[2], pv[3]);
             if constexpr (DROPOUT) {
-              pu[e >> 1] = pack2<BF16>(pv[0], pv[1]);
-              pu[(e >> 1) + 1] = pack2<BF16>(pv[2], pv[3]);
+              // P^T as dV sees it: dropped scores are zero.  Queries e .. e + 3
+              // = 32 h + 16 e' + 4 s + c share one shift of the flags
+              pu[e >> 1] = pp[e >> 1];
+              pu[(e >> 1) + 1] = pp[(e >> 1) + 1];
+              const uint32_t fl = drop_keep[e >> 5] << (((e >> 2) & 3) + 4 * ((e >> 4) & 1));
+              pp[e >> 1] &= pair_keep_mask(fl, 0);
+              pp[(e >> 1) + 1] &= pair_keep_mask(fl, 1);
             }
           }
         }
@@ -615,21 +619,22 @@ __global__ void __launch_bounds__(512, 1)
         for (int e = 0; e < 64; e += 4) {
           const int q0 = 64 * half + e;
           const float4 nd = *reinterpret_cast<const float4*>(dsm + q0);  // -D
-          if constexpr (DROPOUT) {  // dP of the kept scores, scaled by 256 / t
+          if constexpr (DROPOUT) {  // dP of the kept scores (scaled by 256 / t below)
+            const uint32_t fl = drop_keep[e >> 5] << (((e >> 2) & 3) + 4 * ((e >> 4) & 1));
 #pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4)
-              dr[e + k4] = (drop_keep[e >> 5] >> ((e & 31) + k4)) & 1u
-                               ? __float_as_uint(__uint_as_float(dr[e + k4]) * p.inv_keep)
-                               : 0u;
+            for (int k4 = 0; k4 < 4; ++k4) dr[e + k4] &= word_keep_mask(fl, k4);
           }
           float pf[4];
           unpack2<BF16>(pq[e >> 1], pf[0], pf[1]);
           unpack2<BF16>(pq[(e >> 1) + 1], pf[2], pf[3]);
           // packed pairs: (dP - D) then P (dP - D)
-          const auto x01 = fadd2(f2pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])),
-                                 f2pack(nd.x, nd.y));
-          const auto x23 = fadd2(f2pack(__uint_as_float(dr[e + 2]), __uint_as_float(dr[e + 3])),
-                                 f2pack(nd.z, nd.w));
+          // (with dropout, dP of the kept scores times 256 / t, minus D)
+          const auto dr01 = f2pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1]));
+          const auto dr23 = f2pack(__uint_as_float(dr[e + 2]), __uint_as_float(dr[e + 3]));
+          const auto x01 = DROPOUT ? ffma2(dr01, inv_keep2, f2pack(nd.x, nd.y))
+                                   : fadd2(dr01, f2pack(nd.x, nd.y));
+          const auto x23 = DROPOUT ? ffma2(dr23, inv_keep2, f2pack(nd.z, nd.w))
+                                   : fadd2(dr23, f2pack(nd.z, nd.w));
           float gv[4];
           f2unpack(fmul2(f2pack(pf[0], pf[1]), x01), gv[0], gv[1]);
           f2unpack(fmul2(f2pack(pf[2], pf[3]), x23), gv[2], gv[3]);

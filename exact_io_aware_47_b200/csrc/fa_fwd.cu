@@ -439,6 +439,8 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tS = tmem + lane_off + t * 128;
     const uint32_t tO = tmem + lane_off + Lay::kColO + t * D;
     const float c = p.scale_log2;
+    const uint32_t u_drop = 256u - min(p.keep_t, 256u);  // dropout keep test (keep_flags4)
+    const uint32_t u_lo7 = (u_drop & 0x7Fu) * 0x01010101u, u_all = u_drop * 0x01010101u;
     int scnt = 0, ocnt = 0;
     bool ok = true;
     for (int k = 0; ok; ++k) {
@@ -488,15 +490,12 @@ __global__ void __launch_bounds__(384, 1)
       int jj = 0;           // key tiles processed so far
       for (int j = 0; j < jend; ++j) {
         if (!fwd_need<SPARSE>(p, w, t, j)) continue;
-        // dropout: keep bits of this row for key tile j, made while the
-        // tensor core computes S (bit c of drop_keep[c / 32] = key 128 j + c)
+        // dropout: keep flags of this row for key tile j (keep_flags_row128),
+        // made while the tensor core computes S
         uint32_t drop_keep[4] = {~0u, ~0u, ~0u, ~0u};
         if constexpr (DROPOUT) {
-#pragma unroll
-          for (int g = 0; g < 8; ++g) {
-            const uint32_t m16 = keep_bits_row16(p, w.bh, row, j, g, lane & 3);
-            drop_keep[g >> 1] = (g & 1) ? (drop_keep[g >> 1] & 0xFFFFu) | (m16 << 16) : m16;
-          }
+          keep_flags_row128(p, w.bh, row, j, lane & 3, u_lo7, u_all, drop_keep);
+          if (r == 0 && t == 0) FA_TRACE_AT(scnt, 15);
         }
         // scores of this tile are raw * cj in log2 units
         float cj = c, rho = 1.f;
@@ -574,15 +573,16 @@ __global__ void __launch_bounds__(384, 1)
           acc[i & 3] = fadd2(acc[i & 3], p2);
           float p0, p1;
           f2unpack(p2, p0, p1);
-          if constexpr (DROPOUT) {  // dropped scores leave the row sum, not P V
-            p0 = (drop_keep[i >> 4] >> ((2 * i) & 31)) & 1u ? p0 : 0.f;
-            p1 = (drop_keep[i >> 4] >> ((2 * i + 1) & 31)) & 1u ? p1 : 0.f;
-          }
           if constexpr (FP8) {
             const uint32_t h = pack_e4m3x2(p0 * rho, p1 * rho);
             pk[i >> 1] = (i & 1) ? (pk[i >> 1] | (h << 16)) : h;
           } else {
             pk[i] = pack2<BF16>(p0, p1);
+          }
+          if constexpr (DROPOUT) {  // dropped scores leave the row sum, not P V
+            // keys 2 i, 2 i + 1 = 32 h + 16 e + 4 s + c with c = 2 (i & 1)
+            const int sh = ((i >> 1) & 3) + 4 * ((i >> 3) & 1);
+            pk[i] &= pair_keep_mask(drop_keep[i >> 4] << sh, i & 1);
           }
           if (r == 0 && t == 0 && (i & 15) == 15) FA_TRACE_AT(scnt - 1, 8 + (i >> 4));
         }

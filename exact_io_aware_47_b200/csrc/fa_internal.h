@@ -147,36 +147,68 @@ __device__ __forceinline__ bool tile_allowed(const uint8_t* block_mask, int ntil
 // query row 4 qb + w and byte c of that word to key 4 kb + c; a score is kept
 // iff its byte is below keep_t.
 //
-// Forward (lanes = 4 consecutive query rows, lane w = row & 3): 16 keys
-// 16 g .. 16 g + 15 of key tile j for this thread's row; bit c of the result
-// is key 16 g + c.
+// Forward (lanes = 4 consecutive query rows, lane w = row & 3): keep flags
+// of this thread's row for the 128 keys of key tile j.  Group g of 16 keys
+// (keys 16 g + 4 s + c) is the generator call with key block 32 j + 4 g + w;
+// the eight calls run interleaved.  Key k = 32 h + 16 e + 4 s + c of the
+// tile is bit 8 c + 7 - s - 4 e of m[h] (the byte-wise flags of keep_flags4,
+// merged four words to one and two groups to one word): a pair of keys
+// 2 i, 2 i + 1 sits in bits 8 c + 7 and 8 c + 15 of m[h] << (s + 4 e), the
+// form pair_keep_mask reads.
 template <class P>
-__device__ __forceinline__ uint32_t keep_bits_row16(const P& p, int bh, int row, int j, int g,
-                                                    int w) {
-  uint32_t a[4] = {static_cast<uint32_t>(32 * j + 4 * g + w), static_cast<uint32_t>(row >> 2),
-                   static_cast<uint32_t>(bh), p.drop_offset};
-  philox4x32_10(a, p.seed_lo, p.seed_hi);
-  quad_transpose4(a, w);  // a[s] = this row's word of key block 4 g + s
-  uint32_t m = 0;
+__device__ __forceinline__ void keep_flags_row128(const P& p, int bh, int row, int j, int w,
+                                                  uint32_t u_lo7, uint32_t u_all,
+                                                  uint32_t (&m)[4]) {
+  uint32_t a[8][4];
 #pragma unroll
-  for (int s = 0; s < 4; ++s) m |= bytes_below(a[s], p.keep_t) << (4 * s);
-  return m;
+  for (int g = 0; g < 8; ++g) {
+    a[g][0] = static_cast<uint32_t>(32 * j + 4 * g + w);
+    a[g][1] = static_cast<uint32_t>(row >> 2);
+    a[g][2] = static_cast<uint32_t>(bh);
+    a[g][3] = p.drop_offset;
+  }
+  philox4x32_10_n<8>(a, p.seed_lo, p.seed_hi);
+  uint32_t grp[8];
+#pragma unroll
+  for (int g = 0; g < 8; ++g) {
+    quad_transpose4(a[g], w);  // a[g][s]: this row's word of key block 4 g + s
+    grp[g] = merge_flags4(keep_flags4(a[g][0], u_lo7, u_all), keep_flags4(a[g][1], u_lo7, u_all),
+                          keep_flags4(a[g][2], u_lo7, u_all), keep_flags4(a[g][3], u_lo7, u_all));
+  }
+#pragma unroll
+  for (int h = 0; h < 4; ++h) m[h] = bit_select(grp[2 * h], grp[2 * h + 1] >> 4, 0xF0F0F0F0u);
 }
 
-// Backward (lanes = 4 consecutive keys, lane w = key & 3): 16 queries
-// q0 .. q0 + 15 (q0 a multiple of 16) for this thread's key; bit c of the
-// result is query q0 + c.
+// Backward (lanes = 4 consecutive keys, lane w = key & 3): keep flags of
+// this thread's key for 64 queries q0 .. q0 + 63 (q0 a multiple of 64).
+// Group g of 16 queries (q0 + 16 g + 4 s + c) is the generator call with
+// query block q0 / 4 + 4 g + w.  Query
+// q0 + 32 h + 16 e + 4 s + c is bit 8 c + 7 - s - 4 e of m[h], the layout of
+// keep_flags_row128.
 template <class P>
-__device__ __forceinline__ uint32_t keep_bits_key16(const P& p, int bh, int key, int q0, int w) {
-  uint32_t a[4] = {static_cast<uint32_t>(key >> 2), static_cast<uint32_t>((q0 >> 2) + w),
-                   static_cast<uint32_t>(bh), p.drop_offset};
-  philox4x32_10(a, p.seed_lo, p.seed_hi);
-  byte_transpose4(a);     // a[c] = key c's bytes of the 4 queries
-  quad_transpose4(a, w);  // a[s] = this key's bytes of query block q0 / 4 + s
-  uint32_t m = 0;
+__device__ __forceinline__ void keep_flags_key64(const P& p, int bh, int key, int q0, int w,
+                                                 uint32_t u_lo7, uint32_t u_all,
+                                                 uint32_t (&m)[2]) {
+  uint32_t a[4][4];
 #pragma unroll
-  for (int s = 0; s < 4; ++s) m |= bytes_below(a[s], p.keep_t) << (4 * s);
-  return m;
+  for (int g = 0; g < 4; ++g) {
+    a[g][0] = static_cast<uint32_t>(key >> 2);
+    a[g][1] = static_cast<uint32_t>((q0 >> 2) + 4 * g + w);
+    a[g][2] = static_cast<uint32_t>(bh);
+    a[g][3] = p.drop_offset;
+  }
+#pragma unroll
+  for (int g = 0; g < 4; ++g) philox4x32_10(a[g], p.seed_lo, p.seed_hi);
+  uint32_t grp[4];
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    byte_transpose4(a[g]);     // a[g][c] = key c's bytes of the 4 queries
+    quad_transpose4(a[g], w);  // a[g][s] = this key's bytes of query block q0 / 4 + 4 g + s
+    grp[g] = merge_flags4(keep_flags4(a[g][0], u_lo7, u_all), keep_flags4(a[g][1], u_lo7, u_all),
+                          keep_flags4(a[g][2], u_lo7, u_all), keep_flags4(a[g][3], u_lo7, u_all));
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) m[h] = bit_select(grp[2 * h], grp[2 * h + 1] >> 4, 0xF0F0F0F0u);
 }
 
 struct WorkItem {

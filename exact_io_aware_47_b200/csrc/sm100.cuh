@@ -573,6 +573,16 @@ __device__ __forceinline__ void tmem_st_wait() {
 // One call: 128-bit counter c, 64-bit key (k0, k1), 10 rounds.  A round forms
 // the 64-bit products M0 c0 and M1 c2 and sets c = (hi1 ^ c1 ^ k0, lo1,
 // hi0 ^ c3 ^ k1, lo0); the key is bumped by (W0, W1) between rounds.
+__device__ __forceinline__ void philox_round(uint32_t (&c)[4], uint32_t k0, uint32_t k1) {
+  const uint32_t hi0 = __umulhi(0xD2511F53u, c[0]), lo0 = 0xD2511F53u * c[0];
+  const uint32_t hi1 = __umulhi(0xCD9E8D57u, c[2]), lo1 = 0xCD9E8D57u * c[2];
+  const uint32_t n0 = hi1 ^ c[1] ^ k0, n2 = hi0 ^ c[3] ^ k1;
+  c[0] = n0;
+  c[1] = lo1;
+  c[2] = n2;
+  c[3] = lo0;
+}
+
 __device__ __forceinline__ void philox4x32_10(uint32_t (&c)[4], uint32_t k0, uint32_t k1) {
 #pragma unroll
   for (int r = 0; r < 10; ++r) {
@@ -580,13 +590,26 @@ __device__ __forceinline__ void philox4x32_10(uint32_t (&c)[4], uint32_t k0, uin
       k0 += 0x9E3779B9u;
       k1 += 0xBB67AE85u;
     }
-    const uint32_t hi0 = __umulhi(0xD2511F53u, c[0]), lo0 = 0xD2511F53u * c[0];
-    const uint32_t hi1 = __umulhi(0xCD9E8D57u, c[2]), lo1 = 0xCD9E8D57u * c[2];
-    const uint32_t n0 = hi1 ^ c[1] ^ k0, n2 = hi0 ^ c[3] ^ k1;
-    c[0] = n0;
-    c[1] = lo1;
-    c[2] = n2;
-    c[3] = lo0;
+    philox_round(c, k0, k1);
+  }
+}
+
+// G independent calls with the same key, interleaved round by round.  A
+// round is a chain of dependent multiplies (one call alone leaves the
+// multiplier idle most of the time), so G calls in one stream keep it busy.
+template <int G>
+__device__ __forceinline__ void philox4x32_10_n(uint32_t (&c)[G][4], uint32_t k0, uint32_t k1) {
+  // the round keys are rebuilt at each use (two adds a round, shared by the G
+  // calls) rather than held in registers across the caller's loops
+  asm volatile("" : "+r"(k0), "+r"(k1));
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) philox_round(c[g], k0, k1);
   }
 }
 
@@ -619,15 +642,46 @@ __device__ __forceinline__ void byte_transpose4(uint32_t (&x)[4]) {
   x[3] = __byte_perm(t1, t3, 0x7632);
 }
 
-// Bit k (k = 0..3) = (byte k of a) < t, for a threshold t in 1..256: per-byte
-// unsigned compare without carries between bytes (high bit of each byte),
-// then the four flags gathered by one multiply.
-__device__ __forceinline__ uint32_t bytes_below(uint32_t a, uint32_t t) {
-  if (t >= 256u) return 0xFu;
-  const uint32_t H = 0x80808080u, T = t * 0x01010101u;
-  const uint32_t d = (a | H) - (T & ~H);
-  const uint32_t lt = ((~a & T) | (~(a ^ T) & ~d)) & H;
-  return (((lt >> 7) * 0x00204081u) >> 21) & 0xFu;
+// (x & m) | (y & ~m)
+__device__ __forceinline__ uint32_t bit_select(uint32_t x, uint32_t y, uint32_t m) {
+  return (x & m) | (y & ~m);
+}
+
+// Keep flags of the four bytes of a at once, for a threshold t in 1..256:
+// bit 8 c + 7 of the result is set iff byte c is below t; the other bits are
+// unspecified.  With u = 256 - t, byte c is below t iff byte c + u stays below
+// 256, i.e. the byte-wise sum does not carry out of bit 7: the low seven bits
+// of each byte are added without carries between bytes, and the carry out is
+// the majority of the two high bits and the carry into bit 7.
+// u_lo7 = (u & 0x7F) * 0x01010101, u_all = u * 0x01010101.
+__device__ __forceinline__ uint32_t keep_flags4(uint32_t a, uint32_t u_lo7, uint32_t u_all) {
+  const uint32_t s7 = (a & 0x7F7F7F7Fu) + u_lo7;
+  return ~((a & u_all) | (a & s7) | (u_all & s7));
+}
+
+// Four words of keep flags (bit 8 c + 7 of f_s) into one: the flag of byte c
+// of f_s goes to bit 8 c + 7 - s; bits 8 c .. 8 c + 3 are unspecified.
+__device__ __forceinline__ uint32_t merge_flags4(uint32_t f0, uint32_t f1, uint32_t f2,
+                                                 uint32_t f3) {
+  const uint32_t x = bit_select(f0, f1 >> 1, 0x80808080u);  // bits 8c+7, 8c+6
+  const uint32_t y = bit_select(f2 >> 2, f3 >> 3, 0x20202020u);  // bits 8c+5, 8c+4
+  return bit_select(x, y, 0xC0C0C0C0u);
+}
+
+// A 16-bit pair mask from keep flags: the low half is all ones iff bit 7 of
+// byte 2 k of flags is set, the high half iff bit 7 of byte 2 k + 1 is (byte
+// permute with replication of the selected byte's sign bit).
+__device__ __forceinline__ uint32_t pair_keep_mask(uint32_t flags, int k) {
+  uint32_t m;
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(m) : "r"(flags), "r"(k ? 0xBBAAu : 0x9988u));
+  return m;
+}
+
+// A 32-bit mask from keep flags: all ones iff bit 7 of byte c of flags is set.
+__device__ __forceinline__ uint32_t word_keep_mask(uint32_t flags, int c) {
+  uint32_t m;
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(m) : "r"(flags), "r"((8u | c) * 0x1111u));
+  return m;
 }
 
 // ---------------------------------------------------------------------------
