@@ -498,13 +498,14 @@ __global__ void __launch_bounds__(384, 1)
           if (r == 0 && t == 0) FA_TRACE_AT(scnt, 15);
         }
         // scores of this tile are raw * cj in log2 units
-        float cj = c, rho = 1.f;
+        float cj = c, rho = 1.f, inv_rho = 1.f;
         if constexpr (FP8) {
           const float skj = kds[j], svj = vds[j];
           if (!(skj > 0.f && skj < INFINITY && svj > 0.f && svj < INFINITY))
             record_error(kErrDeviceScale, 1);
           cj = c * sq_t * skj;
           rho = svj / sv_max;
+          inv_rho = sv_max / svj;
         }
         ok = mbar_wait_warp(&s_full[t], scnt & 1, wc, 8);
         if (!ok) break;
@@ -558,9 +559,12 @@ __global__ void __launch_bounds__(384, 1)
         };
         // p = 2^(c s - m): packed FMA on pairs, then ex2; row sum in fp32 over
         // four packed accumulators
+        // e4m3: p rho_j = 2^(c s - m + log2 rho_j) is formed directly (the V
+        // descale ratio rides in the exponent), and the row sum divides it back
         const float mu = (m == -INFINITY) ? 0.f : m;
+        const float bias = FP8 ? lg2_approx(rho) - mu : -mu;
         const unsigned long long c2 = f2pack(cj, cj);
-        const unsigned long long nm2 = f2pack(-mu, -mu);
+        const unsigned long long nm2 = f2pack(bias, bias);
         unsigned long long acc[4] = {0ull, 0ull, 0ull, 0ull};
         uint32_t pk[FP8 ? 32 : 64];  // P as the A operand: 16-bit pairs or e4m3 quads
 #pragma unroll
@@ -574,7 +578,7 @@ __global__ void __launch_bounds__(384, 1)
           float p0, p1;
           f2unpack(p2, p0, p1);
           if constexpr (FP8) {
-            const uint32_t h = pack_e4m3x2(p0 * rho, p1 * rho);
+            const uint32_t h = pack_e4m3x2(p0, p1);
             pk[i >> 1] = (i & 1) ? (pk[i >> 1] | (h << 16)) : h;
           } else {
             pk[i] = pack2<BF16>(p0, p1);
@@ -592,7 +596,8 @@ __global__ void __launch_bounds__(384, 1)
           f2unpack(acc[1], b0, b1);
           f2unpack(acc[2], c0, c1);
           f2unpack(acc[3], d0, d1);
-          l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
+          const float sum = ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
+          l += FP8 ? sum * inv_rho : sum;
         }
         if constexpr (FP8) tmem_st32(tS, pk);
         else tmem_st64(tS, pk);

@@ -725,6 +725,13 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// log2(x) (hardware approximation, relative error about 2^-22), x > 0.
+__device__ __forceinline__ float lg2_approx(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
