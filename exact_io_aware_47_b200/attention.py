@@ -327,8 +327,9 @@ def quantize_e4m3(x, out=None, descale=None):
 
 def forward_e4m3(q8, k8, v8, q_descale, k_descale, v_descale, scale=None, causal=False,
                  seqlens=None, out_dtype=torch.bfloat16, out=None, lse=None):
-    """O, LSE of attention on e4m3 inputs ([B, H, N, 128] float8_e4m3fn or
-    uint8 codes, descales [B, H, ceil(N / 128)] float32); O in out_dtype."""
+    """O, LSE of attention on e4m3 inputs ([B, H, N, d] float8_e4m3fn or
+    uint8 codes, d in {64, 128}, descales [B, H, ceil(N / 128)] float32); O
+    in out_dtype."""
     if q8.dim() != 4:
         raise ValueError("q8 must be [B, H, N, d]")
     B, H, N, d = q8.shape

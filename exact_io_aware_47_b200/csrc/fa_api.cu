@@ -96,8 +96,10 @@ int make_map(CUtensorMap* map, const void* ptr, int BH, int N, int d, int dtype)
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
-// [B*H, N, 128] e4m3 view: box = 128 columns (128 bytes) x 128 rows, 128-byte
-// swizzle; in bytes the same tiles as the 16-bit d = 64 layout.
+// [B*H, N, d] e4m3 view: box = 128 columns (128 bytes) x 128 rows, 128-byte
+// swizzle; in bytes the same tiles as the 16-bit d = 64 layout.  For d = 64
+// the box runs past the row: the load fills columns 64..127 with zeros, so
+// the d = 128 kernel computes the same S and an O whose last 64 columns are 0.
 int make_map_e4m3(CUtensorMap* map, const void* ptr, int BH, int N, int d) {
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
                               static_cast<cuuint64_t>(BH)};
@@ -187,6 +189,7 @@ int fwd_core(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.B = B;
   p.H = H;
   p.N = N;
+  p.o_cols = d;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.causal = causal ? 1 : 0;
   p.n_qtiles = (p.max_seqlen + kBlockM - 1) / kBlockM;
@@ -281,7 +284,6 @@ extern "C" int fa_fwd_e4m3(const void* q8, const void* k8, const void* v8, const
     return FA_ERR_INVALID_ARG;
   const int st = check_common(B, H, N, d, scale, out_dtype);
   if (st != FA_OK) return st;
-  if (d != 128) return FA_ERR_UNSUPPORTED;
   const uintptr_t ds_bits = reinterpret_cast<uintptr_t>(q_descale) |
                             reinterpret_cast<uintptr_t>(k_descale) |
                             reinterpret_cast<uintptr_t>(v_descale);

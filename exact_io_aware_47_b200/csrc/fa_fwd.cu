@@ -621,9 +621,13 @@ __global__ void __launch_bounds__(384, 1)
       const float inv_l = FP8 ? sv_max / l : (DROPOUT ? p.inv_keep / l : 1.f / l);
       const bool store = row < w.rows;
       const size_t orow_idx = static_cast<size_t>(w.z) * p.N + w.row0 + (store ? row : 0);
-      uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) + orow_idx * (D * 2);
+      // O rows are o_cols wide: D, or 64 for e4m3 inputs with d = 64, whose
+      // columns 64..127 of the accumulator are zero (zero-filled V columns)
+      const int o_cols = FP8 ? p.o_cols : D;
+      uint8_t* orow = reinterpret_cast<uint8_t*>(p.o) + orow_idx * (o_cols * 2);
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
+        if (FP8 && cc * 32 >= o_cols) break;
         uint32_t ro[32];
         tmem_ld32(tO + cc * 32, ro);
         uint32_t pk[16];

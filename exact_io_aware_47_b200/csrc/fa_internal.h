@@ -42,6 +42,8 @@ struct FwdParams {
   const float* k_descale;
   const float* v_descale;
   int B, H, N;
+  int o_cols;               // columns of O (d); the e4m3 kernel reads d = 64 inputs as 128
+                            // columns, the TMA load filling columns 64..127 with zeros
   float scale_log2;         // scale * log2(e)
   int causal;
   int n_qtiles;             // ceil(N / 128)

@@ -177,16 +177,19 @@ int fa_bwd_dropout(const void* q, const void* k, const void* v, const void* o,
  *     d in {64, 128}.  An infinite or NaN input is reported as
  *     FA_ERR_DEVICE_SCALE (that tile's descale and codes are then unspecified).
  *   fa_fwd_e4m3: forward attention of Q, K, V given as e4m3 codes
- *     [B, H, N, 128] with descales [B, H, ceil(N/128)] (any positive finite
+ *     [B, H, N, d] with descales [B, H, ceil(N/128)] (any positive finite
  *     values; the quantiser's output is one choice): the tensors stand for
  *     code * descale of the row's tile.  Scores, masks, seqlens and LSE are
  *     as in fa_fwd, on those values.  For the product with V the
  *     probabilities of key tile j (against the running row max, which moves
  *     only by more than 8 in log2 units) are multiplied by
- *     sv_j / max sv (the largest V descale of the slice's valid key tiles)
- *     and rounded to e4m3; the row sum uses them before rounding; O =
- *     max sv * sum / l in out_dtype (FA_BF16 or FA_FP16) [B, H, N, 128].
- *     d must be 128 (FA_ERR_UNSUPPORTED otherwise).  Descale pointers must be
+ *     sv_j / max sv (the largest V descale of the slice's valid key tiles;
+ *     formed as 2^(c s - m + log2(sv_j / max sv))) and rounded to e4m3; the
+ *     row sum uses them before rounding, divided back by sv_j / max sv; O =
+ *     max sv * sum / l in out_dtype (FA_BF16 or FA_FP16) [B, H, N, d].
+ *     d in {64, 128}: d = 64 runs the d = 128 kernel, whose loads fill
+ *     columns 64..127 with zeros (same results, the d = 128 time).
+ *     FA_ERR_UNSUPPORTED for other d.  Descale pointers must be
  *     4-byte aligned, the others 16-byte aligned.  A descale that is not
  *     finite and positive is reported as FA_ERR_DEVICE_SCALE (the results are
  *     then unspecified).

@@ -135,8 +135,7 @@ def test_e4m3_rejections_before_any_cuda_call(lib):
     assert fwd8(B=0) == _lib.FA_ERR_INVALID_ARG
     assert fwd8(scale=-1.0) == _lib.FA_ERR_INVALID_ARG
     assert fwd8(dtype=5) == _lib.FA_ERR_INVALID_ARG
-    assert fwd8(d=64) == _lib.FA_ERR_UNSUPPORTED                # 8-bit path: d = 128 only
-    assert fwd8(d=96) == _lib.FA_ERR_UNSUPPORTED
+    assert fwd8(d=96) == _lib.FA_ERR_UNSUPPORTED                # 8-bit path: d in {64, 128}
     assert fwd8(ds=P + 2) == _lib.FA_ERR_ALIGNMENT              # descales: 4-byte aligned
     assert fwd8(q=P + 8) == _lib.FA_ERR_ALIGNMENT               # codes: 16-byte aligned
     assert fwd8(o=P + 4) == _lib.FA_ERR_ALIGNMENT

@@ -86,9 +86,9 @@ def test_quantizer_is_the_oracle_bit_for_bit(fa, dtype, d):
     assert np.array_equal(ds.cpu().numpy(), rds)
 
 
-def _fwd_case(fa, B, H, N, causal, seed, seqlens=None, out_dtype=torch.bfloat16, v_scales=None):
+def _fwd_case(fa, B, H, N, causal, seed, seqlens=None, out_dtype=torch.bfloat16, v_scales=None,
+              d=128):
     from exact_io_aware_47_b200.inputs import make_inputs_shape
-    d = 128
     inp = make_inputs_shape(B, H, N, d, torch.bfloat16, seed=seed, seqlens=seqlens)
     v = inp["v"].float()
     if v_scales is not None:                                   # V tiles on different scales
@@ -108,11 +108,15 @@ def _fwd_case(fa, B, H, N, causal, seed, seqlens=None, out_dtype=torch.bfloat16,
     return (qc, kc, vc, sq, sk, sv), f64(o), f64(lse), scale
 
 
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("N", [128, 300, 515])
-def test_forward_against_oracle(fa, N, causal):
+def test_forward_against_oracle(fa, N, causal, d):
+    """d = 64 runs the d = 128 kernel on zero-filled columns 64..127."""
     B, H = 2, 2
-    (qc, kc, vc, sq, sk, sv), o, lse, scale = _fwd_case(fa, B, H, N, causal, seed=N + causal)
+    (qc, kc, vc, sq, sk, sv), o, lse, scale = _fwd_case(fa, B, H, N, causal, seed=N + causal + d,
+                                                        d=d)
+    assert o.shape == (B, H, N, d)
     for b in range(B):
         for h in range(H):
             a = (qc[b, h], kc[b, h], vc[b, h], sq[b, h], sk[b, h], sv[b, h])
@@ -167,8 +171,8 @@ def test_rejections_and_device_scale_status(fa):
     lse = torch.empty((1, 1, 128), dtype=torch.float32, device="cuda")
     args = lambda qp, dsp, d: (qp, qp, qp, dsp, dsp, dsp, o.data_ptr(), lse.data_ptr(), 1, 1, 128,
                                d, 0.1, 0, None, _lib.FA_BF16, s)
-    q64 = torch.zeros((1, 1, 128, 64), dtype=torch.uint8, device="cuda")
-    assert _lib.fa_fwd_e4m3(*args(q64.data_ptr(), ds.data_ptr(), 64)) == _lib.FA_ERR_UNSUPPORTED
+    q96 = torch.zeros((1, 1, 128, 96), dtype=torch.uint8, device="cuda")
+    assert _lib.fa_fwd_e4m3(*args(q96.data_ptr(), ds.data_ptr(), 96)) == _lib.FA_ERR_UNSUPPORTED
     assert _lib.fa_fwd_e4m3(*args(q8.data_ptr(), ds.data_ptr() + 2, 128)) == _lib.FA_ERR_ALIGNMENT
     assert _lib.fa_fwd_e4m3(*args(q8.data_ptr(), None, 128)) == _lib.FA_ERR_INVALID_ARG
     bad = torch.full((1, 1, 1), -1.0, dtype=torch.float32, device="cuda")
