@@ -61,3 +61,28 @@ def test_reference_arm_other_ranks_exit_without_work(workload):
                          capture_output=True, text=True, timeout=120, cwd=ROOT, env=env)
     assert out.returncode == 0, out.stderr[-2000:]
     assert not [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+
+
+def test_cpu_baseline_cuts_long_slices(monkeypatch):
+    """Slices longer than max_rows are cut to their first max_rows queries and
+    keys before the oracle sees them; shorter ones go whole."""
+    import types
+    import torch
+    import oracle
+    seen = []
+    real = oracle.ref_fwd_slice
+
+    def spy(q, k, v, *a, **kw):
+        seen.append((q.shape, k.shape, v.shape))
+        return real(q, k, v, *a, **kw)
+    monkeypatch.setattr(oracle, "ref_fwd_slice", spy)
+    B, H, N, d = 1, 2, 96, 16
+    w = types.SimpleNamespace(B=B, H=H, N=N, d=d, scale=d ** -0.5, causal=True, name="cut")
+    g = torch.Generator().manual_seed(0)
+    q, k, v, do = (torch.randn(B, H, N, d, generator=g) for _ in range(4))
+    whole = bench.cpu_baseline_slices(w, q, k, v, do, None, budget_s=60.0)
+    assert "whole" in whole["sample"] and seen == [((N, d),) * 3] * H
+    seen.clear()
+    cut = bench.cpu_baseline_slices(w, q, k, v, do, None, budget_s=60.0, max_rows=32)
+    assert "cut to its first 32" in cut["sample"] and seen == [((32, d),) * 3] * H
+    assert whole["kind"] == cut["kind"] == "oracle" and cut["value"] > 0 and cut["cores"] >= 1
