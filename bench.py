@@ -601,36 +601,90 @@ def _timed_steps(torch, step, n_marks, args, world, dev, stream, lib):
     return warmup, total_ms, seg, clk
 
 
-def _e2e(torch, dev_inputs, dev_outputs, api_step, K, world, dev, stream, step_flops):
+def _e2e(torch, dev_inputs, dev_outputs, make_step, K, world, dev, stream, step_flops):
     """End to end through the public API: every step copies its inputs from
-    pinned host memory, runs api_step and copies its results back."""
-    ins = [(t.cpu().pin_memory(), t) for t in dev_inputs]
-    outs = [(t, torch.empty(t.shape, dtype=t.dtype, pin_memory=True)) for t in dev_outputs]
-    h2d = sum(src.numel() * src.element_size() for src, _ in ins)
-    d2h = sum(dst.numel() * dst.element_size() for _, dst in outs)
+    pinned host memory, runs the step (``make_step(inputs, outputs)`` returns
+    it for one set of device buffers) and copies its results back.
 
-    def e2e_step():
-        for src, dst in ins:
-            dst.copy_(src, non_blocking=True)
-        api_step()
-        for src, dst in outs:
-            dst.copy_(src, non_blocking=True)
-
-    for _ in range(2):
-        e2e_step()
+    Timed twice, both with every step's copies inside the timed region:
+    serially (copy in, compute, copy out on one stream), and pipelined as a
+    caller streaming batches would run it: two sets of device buffers, the
+    input copy of step k + 1 on its own stream overlapping step k, and the
+    output copy of step k on a third stream overlapping step k + 1."""
+    ins_h = [t.cpu().pin_memory() for t in dev_inputs]
+    outs_h = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in dev_outputs]
+    h2d = sum(t.numel() * t.element_size() for t in ins_h)
+    d2h = sum(t.numel() * t.element_size() for t in outs_h)
+    sets = [(list(dev_inputs), list(dev_outputs)),
+            ([torch.empty_like(t) for t in dev_inputs], [torch.empty_like(t) for t in dev_outputs])]
+    steps = [make_step(i, o) for i, o in sets]
     ke = max(3, min(K, 10))
-    dist_barrier(world)
-    torch.cuda.synchronize(dev)
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(ke):
-        e2e_step()
-    b.record(stream)
-    torch.cuda.synchronize(dev)
-    dist_barrier(world)
-    e_ms = dist_max(a.elapsed_time(b), world)
-    return {"value": world * step_flops * ke / (e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms / ke}
+
+    def timed(run):
+        run(2)  # warm-up
+        dist_barrier(world)
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        run(ke, a)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        dist_barrier(world)
+        return dist_max(a.elapsed_time(b), world)
+
+    def serial(n, start=None):
+        ins_d, outs_d = sets[0]
+        for _ in range(n):
+            for src, dst in zip(ins_h, ins_d):
+                dst.copy_(src, non_blocking=True)
+            steps[0]()
+            for src, dst in zip(outs_d, outs_h):
+                dst.copy_(src, non_blocking=True)
+
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = lambda: [torch.cuda.Event() for _ in range(2)]
+    in_ready, done, out_done = ev(), ev(), ev()
+
+    def pipelined(n, start=None):
+        if start is not None:  # the copy streams start with the timed region
+            s_in.wait_event(start)
+            s_out.wait_event(start)
+        for k in range(n):
+            j = k % 2
+            ins_d, outs_d = sets[j]
+            if k >= 2:
+                s_in.wait_event(done[j])         # step k-2 has read input set j
+            with torch.cuda.stream(s_in):
+                for src, dst in zip(ins_h, ins_d):
+                    dst.copy_(src, non_blocking=True)
+                in_ready[j].record(s_in)
+            stream.wait_event(in_ready[j])
+            if k >= 2:
+                stream.wait_event(out_done[j])   # output set j has been copied out
+            steps[j]()
+            done[j].record(stream)
+            s_out.wait_event(done[j])
+            with torch.cuda.stream(s_out):
+                for src, dst in zip(outs_d, outs_h):
+                    dst.copy_(src, non_blocking=True)
+                out_done[j].record(s_out)
+        for j in range(2):                       # the region ends with the last copies
+            stream.wait_event(out_done[j])
+
+    ser_ms = timed(serial)
+    pip_ms = timed(pipelined)
+    tf = lambda ms: world * step_flops * ke / (ms / 1e3) / 1e12
+    # the line's figure is the faster schedule (for tiny steps the stream
+    # hand-offs cost more than the copies they overlap); both are reported
+    pip = pip_ms < ser_ms
+    ms = pip_ms if pip else ser_ms
+    return {"value": tf(ms), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms / ke,
+            "mode": ("pipelined: two device buffer sets; the input copy of step k + 1 and the "
+                     "output copy of step k overlap the compute of steps k and k + 1") if pip else
+                    "serial: copy in, compute, copy out on one stream",
+            "serial": {"value": tf(ser_ms), "ms_per_step": ser_ms / ke},
+            "pipelined": {"value": tf(pip_ms), "ms_per_step": pip_ms / ke}}
 
 
 def _roof(kernel, flops, ms, peak, peak_src, traffic=None, sustained=None):
@@ -771,11 +825,16 @@ def run_ours(args, w):
 
     e2e = None
     if not args.no_e2e:
-        def api_step():
-            fa.forward(q, k, v, scale=scale, causal=causal, seqlens=sl, out=o, lse=lse)
-            fa.backward(q, k, v, o, lse, do, scale=scale, causal=causal, seqlens=sl,
-                        workspace=ws, dq=dq, dk=dk, dv=dv)
-        e2e = _e2e(torch, (q, k, v, do), (o, lse, dq, dk, dv), api_step, K, world, dev, stream,
+        def make_step(ins, outs):
+            q_, k_, v_, do_ = ins
+            o_, lse_, dq_, dk_, dv_ = outs
+
+            def api_step():
+                fa.forward(q_, k_, v_, scale=scale, causal=causal, seqlens=sl, out=o_, lse=lse_)
+                fa.backward(q_, k_, v_, o_, lse_, do_, scale=scale, causal=causal, seqlens=sl,
+                            workspace=ws, dq=dq_, dk=dk_, dv=dv_)
+            return api_step
+        e2e = _e2e(torch, (q, k, v, do), (o, lse, dq, dk, dv), make_step, K, world, dev, stream,
                    step_flops)
 
     cpu = None
@@ -859,11 +918,17 @@ def run_ours_packed(args, w):
 
     e2e = None
     if not args.no_e2e:
-        def api_step():
-            fa.forward_varlen(q, k, v, cu, ms, scale=scale, causal=causal, out=o, lse=lse)
-            fa.backward_varlen(q, k, v, o, lse, do, cu, ms, scale=scale, causal=causal,
-                               workspace=ws, dq=dq, dk=dk, dv=dv)
-        e2e = _e2e(torch, (q, k, v, do, cu), (o, lse, dq, dk, dv), api_step, K, world, dev,
+        def make_step(ins, outs):
+            q_, k_, v_, do_, cu_ = ins
+            o_, lse_, dq_, dk_, dv_ = outs
+
+            def api_step():
+                fa.forward_varlen(q_, k_, v_, cu_, ms, scale=scale, causal=causal, out=o_,
+                                  lse=lse_)
+                fa.backward_varlen(q_, k_, v_, o_, lse_, do_, cu_, ms, scale=scale, causal=causal,
+                                   workspace=ws, dq=dq_, dk=dk_, dv=dv_)
+            return api_step
+        e2e = _e2e(torch, (q, k, v, do, cu), (o, lse, dq, dk, dv), make_step, K, world, dev,
                    stream, step_flops)
 
     cpu = None
@@ -947,10 +1012,16 @@ def run_ours_variant(args, spec):
                                            mask.data_ptr(), B, H, N, d, scale, int(causal), None,
                                            dt_code, sh)
 
-        def api_step():
-            fa.forward_blocksparse(q, k, v, mask, scale=scale, causal=causal, out=o, lse=lse)
-            fa.backward_blocksparse(q, k, v, o, lse, do, mask, scale=scale, causal=causal,
-                                    workspace=ws, dq=dq, dk=dk, dv=dv)
+        def make_step(ins, outs):
+            q_, k_, v_, do_, mask_ = ins
+            o_, lse_, dq_, dk_, dv_ = outs
+
+            def api_step():
+                fa.forward_blocksparse(q_, k_, v_, mask_, scale=scale, causal=causal, out=o_,
+                                       lse=lse_)
+                fa.backward_blocksparse(q_, k_, v_, o_, lse_, do_, mask_, scale=scale,
+                                        causal=causal, workspace=ws, dq=dq_, dk=dk_, dv=dv_)
+            return api_step
         cfg = {"tiles_computed": sum(1 for i in range(nt) for j in range(nt)
                                      if mask_list[i][j] and not (causal and j > i)),
                "tiles_total": nt * nt}
@@ -968,11 +1039,16 @@ def run_ours_variant(args, spec):
                                        P["dk"], P["dv"], P["ws"], ws_bytes, B, H, N, d, scale,
                                        int(causal), None, p_drop, seed, 0, dt_code, sh)
 
-        def api_step():
-            fa.forward_dropout(q, k, v, p_drop, seed, 0, scale=scale, causal=causal, out=o,
-                               lse=lse)
-            fa.backward_dropout(q, k, v, o, lse, do, p_drop, seed, 0, scale=scale,
-                                causal=causal, workspace=ws, dq=dq, dk=dk, dv=dv)
+        def make_step(ins, outs):
+            q_, k_, v_, do_ = ins
+            o_, lse_, dq_, dk_, dv_ = outs
+
+            def api_step():
+                fa.forward_dropout(q_, k_, v_, p_drop, seed, 0, scale=scale, causal=causal,
+                                   out=o_, lse=lse_)
+                fa.backward_dropout(q_, k_, v_, o_, lse_, do_, p_drop, seed, 0, scale=scale,
+                                    causal=causal, workspace=ws, dq=dq_, dk=dk_, dv=dv_)
+            return api_step
         cfg = {"p_drop": p_drop, "seed": seed}
 
     def step(ev=None):
@@ -999,7 +1075,7 @@ def run_ours_variant(args, spec):
 
     e2e = None
     if not args.no_e2e:
-        e2e = _e2e(torch, (q, k, v, do) + extra_inputs, (o, lse, dq, dk, dv), api_step, K,
+        e2e = _e2e(torch, (q, k, v, do) + extra_inputs, (o, lse, dq, dk, dv), make_step, K,
                    world, dev, stream, step_flops)
 
     cpu = None
@@ -1083,11 +1159,16 @@ def run_ours_fp8(args, spec):
 
     e2e = None
     if not args.no_e2e:
-        def api_step():
-            for x, x8, ds in trio:
-                fa.quantize_e4m3(x, out=x8, descale=ds)
-            fa.forward_e4m3(q8, k8, v8, sq, sk, sv, scale=scale, causal=causal, out=o, lse=lse)
-        e2e = _e2e(torch, (q, k, v), (o, lse), api_step, K, world, dev, stream, f_fwd)
+        def make_step(ins, outs):
+            o_, lse_ = outs
+
+            def api_step():  # the codes and descales are per-step scratch on the device
+                for x, (_, x8, ds) in zip(ins, trio):
+                    fa.quantize_e4m3(x, out=x8, descale=ds)
+                fa.forward_e4m3(q8, k8, v8, sq, sk, sv, scale=scale, causal=causal, out=o_,
+                                lse=lse_)
+            return api_step
+        e2e = _e2e(torch, (q, k, v), (o, lse), make_step, K, world, dev, stream, f_fwd)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
